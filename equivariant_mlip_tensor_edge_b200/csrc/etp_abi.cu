@@ -1,0 +1,368 @@
+// C ABI of libetp: handle lifecycle, argument checks, workspace carving and kernel dispatch.
+// The operation and conventions are documented in include/etp.h.
+#include <cctype>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "etp_internal.h"
+#include "generated/etp_paths.h"
+
+struct etp_ctx {
+  etp::Ctx c;
+};
+
+namespace etp {
+
+static thread_local std::string g_last_error;
+
+void set_error(const std::string& msg) { g_last_error = msg; }
+
+etp_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ETP_OK;
+  set_error(std::string(what) + ": " + cudaGetErrorString(e));
+  return ETP_ERR_CUDA;
+}
+
+namespace {
+
+struct Block {
+  int mul, l, parity;
+};
+
+// "64x0e+64x1o" -> blocks. Returns false on a malformed string.
+bool parse_irreps(const char* s, std::vector<Block>* out) {
+  if (!s) return false;
+  std::string str;
+  for (const char* p = s; *p; ++p)
+    if (!std::isspace(static_cast<unsigned char>(*p))) str.push_back(*p);
+  if (str.empty()) return false;
+  size_t pos = 0;
+  while (pos <= str.size()) {
+    size_t end = str.find('+', pos);
+    if (end == std::string::npos) end = str.size();
+    std::string term = str.substr(pos, end - pos);
+    if (term.empty()) return false;
+    int mul = 1;
+    size_t x = term.find('x');
+    std::string lp = term;
+    if (x != std::string::npos) {
+      std::string m = term.substr(0, x);
+      if (m.empty() || m.size() > 6) return false;
+      for (char ch : m)
+        if (!std::isdigit(static_cast<unsigned char>(ch))) return false;
+      mul = std::atoi(m.c_str());
+      lp = term.substr(x + 1);
+    }
+    if (lp.size() < 2 || lp.size() > 3) return false;
+    char par = lp.back();
+    if (par != 'e' && par != 'o') return false;
+    std::string ls = lp.substr(0, lp.size() - 1);
+    for (char ch : ls)
+      if (!std::isdigit(static_cast<unsigned char>(ch))) return false;
+    out->push_back({mul, std::atoi(ls.c_str()), par == 'e' ? 1 : -1});
+    pos = end + 1;
+    if (end == str.size()) break;
+  }
+  return true;
+}
+
+// Paths (block_in, l2, block_out) in lexicographic order with the triangle and parity rules.
+std::vector<int> enumerate_paths(const std::vector<Block>& in, int sh_lmax, const std::vector<Block>& out) {
+  std::vector<int> ls;
+  for (const Block& a : in)
+    for (int l2 = 0; l2 <= sh_lmax; ++l2)
+      for (const Block& b : out) {
+        int sh_par = (l2 % 2) ? -1 : 1;
+        if (std::abs(a.l - l2) <= b.l && b.l <= a.l + l2 && a.parity * sh_par == b.parity) {
+          ls.push_back(a.l);
+          ls.push_back(l2);
+          ls.push_back(b.l);
+        }
+      }
+  return ls;
+}
+
+template <int L>
+bool fill_from_table(Ctx* c, const std::vector<int>& ls) {
+  using PS = etp_gen::PathSet<L>;
+  const int* tab = L == 1 ? etp_gen::kPathL_1 : (L == 2 ? etp_gen::kPathL_2 : etp_gen::kPathL_3);
+  if (static_cast<int>(ls.size()) != 3 * PS::P) return false;
+  for (int i = 0; i < 3 * PS::P; ++i)
+    if (ls[i] != tab[i]) return false;
+  c->n_paths = PS::P;
+  c->cg_nnz = PS::NNZ;
+  c->sum_2l3p1 = PS::SUM_2L3P1;
+  return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+}  // namespace etp
+
+using namespace etp;
+
+extern "C" {
+
+const char* etp_status_string(etp_status s) {
+  switch (s) {
+    case ETP_OK: return "ok";
+    case ETP_ERR_INVALID_ARG: return "invalid argument";
+    case ETP_ERR_IRREPS: return "malformed irreps string";
+    case ETP_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ETP_ERR_BAD_GRAPH: return "invalid CSR graph";
+    case ETP_ERR_CUDA: return "CUDA error";
+    case ETP_ERR_CAPACITY: return "output capacity exceeded";
+  }
+  return "unknown status";
+}
+
+const char* etp_last_error(void) { return g_last_error.c_str(); }
+
+etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_basis,
+                      float r_cut, etp_handle* out) {
+  if (!out) {
+    set_error("etp_create: out is NULL");
+    return ETP_ERR_INVALID_ARG;
+  }
+  *out = nullptr;
+  std::vector<Block> bin, bout;
+  if (!parse_irreps(irreps_in, &bin) || !parse_irreps(irreps_out, &bout)) {
+    set_error("etp_create: malformed irreps string");
+    return ETP_ERR_IRREPS;
+  }
+  if (!(r_cut > 0.f) || n_basis <= 0 || sh_lmax < 0) {
+    set_error("etp_create: r_cut must be > 0, n_basis > 0, sh_lmax >= 0");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_basis != kNumBasis) {
+    set_error("etp_create: only n_basis == 8 is implemented");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  const int L = static_cast<int>(bin.size()) - 1;
+  if (L < 1 || L > kMaxL || bin.size() != bout.size() || sh_lmax != L) {
+    set_error("etp_create: need irreps_in == irreps_out == C x (0e..Le), sh_lmax == L, 1 <= L <= 3");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  const int C = bin[0].mul;
+  for (int l = 0; l <= L; ++l) {
+    const int par = (l % 2) ? -1 : 1;
+    const Block& a = bin[l];
+    const Block& b = bout[l];
+    if (a.l != l || b.l != l || a.parity != par || b.parity != par || a.mul != C || b.mul != C) {
+      set_error("etp_create: blocks must be l = 0..L in order, parity (-1)^l, one multiplicity");
+      return ETP_ERR_UNSUPPORTED;
+    }
+  }
+  if (C % kBatch != 0 || C < kBatch || C > 256) {
+    set_error("etp_create: channel count must be a multiple of 4 in [4, 256]");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  Ctx c;
+  c.lmax = L;
+  c.channels = C;
+  c.dim = C * (L + 1) * (L + 1);
+  c.r_cut = r_cut;
+  const std::vector<int> ls = enumerate_paths(bin, sh_lmax, bout);
+  bool ok = L == 1 ? fill_from_table<1>(&c, ls) : (L == 2 ? fill_from_table<2>(&c, ls) : fill_from_table<3>(&c, ls));
+  if (!ok) {
+    set_error("etp_create: path enumeration does not match the generated path tables");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  etp_ctx* h = new (std::nothrow) etp_ctx;
+  if (!h) {
+    set_error("etp_create: out of host memory");
+    return ETP_ERR_INVALID_ARG;
+  }
+  h->c = c;
+  *out = h;
+  return ETP_OK;
+}
+
+etp_status etp_destroy(etp_handle h) {
+  delete h;
+  return ETP_OK;
+}
+
+etp_status etp_get_info(etp_handle h, etp_info_t* info) {
+  if (!h || !info) {
+    set_error("etp_get_info: NULL argument");
+    return ETP_ERR_INVALID_ARG;
+  }
+  const Ctx& c = h->c;
+  info->lmax = c.lmax;
+  info->channels = c.channels;
+  info->dim_in = c.dim;
+  info->dim_out = c.dim;
+  info->n_paths = c.n_paths;
+  info->n_basis = kNumBasis;
+  info->weight_numel = kNumBasis * c.n_paths * c.channels;
+  info->cg_nnz = c.cg_nnz;
+  info->sum_2l3p1 = c.sum_2l3p1;
+  info->r_cut = c.r_cut;
+  return ETP_OK;
+}
+
+// Workspace: [recv_map: n_edges ints][validation scratch: n_edges + 1 ints]
+size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
+  (void)h;
+  (void)n_nodes;
+  if (n_edges < 0) return 0;
+  return align256(sizeof(int) * static_cast<size_t>(n_edges)) +
+         align256(sizeof(int) * (static_cast<size_t>(n_edges) + 1));
+}
+
+static etp_status check_common(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                               const int* sender, const float* edge_vec, const float* x,
+                               const float* W, const char* who) {
+  if (!h) {
+    set_error(std::string(who) + ": NULL handle");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_nodes < 0 || n_edges < 0) {
+    set_error(std::string(who) + ": negative size");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(n_nodes) * h->c.dim >= (1LL << 31)) {
+    set_error(std::string(who) + ": n_nodes * dim must stay below 2^31");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  if (!row_ptr || (n_edges > 0 && (!sender || !edge_vec || !x || !W))) {
+    set_error(std::string(who) + ": NULL array");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if ((x && !aligned16(x)) || (W && !aligned16(W))) {
+    set_error(std::string(who) + ": x and W must be 16-byte aligned");
+    return ETP_ERR_INVALID_ARG;
+  }
+  return ETP_OK;
+}
+
+static bool validate_requested() {
+  const char* v = std::getenv("ETP_VALIDATE");
+  return v && v[0] == '1';
+}
+
+etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                       const int* sender, const float* edge_vec, const float* x, const float* W,
+                       float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_forward");
+  if (st != ETP_OK) return st;
+  if (!out || !aligned16(out)) {
+    set_error("etp_forward: out must be a 16-byte aligned device pointer");
+    return ETP_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (validate_requested()) {
+    if (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges)) {
+      set_error("etp_forward: ETP_VALIDATE=1 needs the workspace");
+      return ETP_ERR_INVALID_ARG;
+    }
+    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) +
+                                          align256(sizeof(int) * static_cast<size_t>(n_edges)));
+    st = validate_graph(n_nodes, n_edges, row_ptr, sender, nullptr, nullptr, scratch, s);
+    if (st != ETP_OK) return st;
+  }
+  if (n_nodes == 0) return ETP_OK;
+  return launch_forward(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, s);
+}
+
+etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                        const int* sender, const float* edge_vec, const int* t_row_ptr,
+                        const int* t_perm, const float* x, const float* W, const float* grad_out,
+                        float* grad_x, float* grad_edge_vec, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_backward");
+  if (st != ETP_OK) return st;
+  if (!t_row_ptr || (n_edges > 0 && (!t_perm || !grad_out)) || (!grad_x && !grad_edge_vec)) {
+    set_error("etp_backward: NULL array (grad_x and grad_edge_vec may not both be NULL)");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if ((grad_x && !aligned16(grad_x)) || (grad_out && !aligned16(grad_out))) {
+    set_error("etp_backward: grad_x and grad_out must be 16-byte aligned");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_edges > 0 && (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges))) {
+    set_error("etp_backward: workspace missing or smaller than etp_workspace_bytes()");
+    return ETP_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* recv_map = static_cast<int*>(workspace);
+  if (validate_requested()) {
+    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) +
+                                          align256(sizeof(int) * static_cast<size_t>(n_edges)));
+    st = validate_graph(n_nodes, n_edges, row_ptr, sender, t_row_ptr, t_perm, scratch, s);
+    if (st != ETP_OK) return st;
+  }
+  if (n_nodes == 0) return ETP_OK;
+  return launch_backward(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, t_row_ptr, t_perm, x,
+                         W, grad_out, grad_x, grad_edge_vec, recv_map, s);
+}
+
+etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, const float* W,
+                              float* w_out, void* stream) {
+  if (!h || n_edges < 0 || (n_edges > 0 && (!edge_vec || !W || !w_out))) {
+    set_error("etp_radial_weights: bad argument");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_edges == 0) return ETP_OK;
+  return launch_radial_weights(h->c, n_edges, edge_vec, W, w_out, static_cast<cudaStream_t>(stream));
+}
+
+etp_status etp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* t_row_ptr,
+                      const int* t_perm, const float* grad_edge_vec, float* forces, void* stream) {
+  if (n_nodes < 0 || n_edges < 0 || !row_ptr || !t_row_ptr || !forces ||
+      (n_edges > 0 && (!t_perm || !grad_edge_vec))) {
+    set_error("etp_forces: bad argument");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_nodes == 0) return ETP_OK;
+  return launch_forces(n_nodes, n_edges, row_ptr, t_row_ptr, t_perm, grad_edge_vec, forces,
+                       static_cast<cudaStream_t>(stream));
+}
+
+size_t etp_graph_workspace_bytes(int n_nodes, int max_edges) {
+  if (n_nodes < 0 || max_edges < 0) return 0;
+  return graph_workspace_bytes(n_nodes, max_edges);
+}
+
+etp_status etp_neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,
+                         float r_cut, int max_edges, int* n_edges, int* row_ptr, int* sender,
+                         float* edge_vec, int* shift, int* t_row_ptr, int* t_perm,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_nodes < 0 || max_edges < 0 || !n_edges || !row_ptr || !t_row_ptr || !(r_cut > 0.f) ||
+      (n_nodes > 0 && !pos) || (max_edges > 0 && (!sender || !edge_vec || !t_perm))) {
+    set_error("etp_neighbors: bad argument");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (workspace_bytes < graph_workspace_bytes(n_nodes, max_edges) || (!workspace && workspace_bytes)) {
+    set_error("etp_neighbors: workspace smaller than etp_graph_workspace_bytes()");
+    return ETP_ERR_INVALID_ARG;
+  }
+  return neighbors(pos, n_nodes, cell, pbc, r_cut, max_edges, n_edges, row_ptr, sender, edge_vec,
+                   shift, t_row_ptr, t_perm, workspace, workspace_bytes,
+                   static_cast<cudaStream_t>(stream));
+}
+
+etp_status etp_build_csr(int n_nodes, int n_edges, const int* receiver, const int* sender_in,
+                         const float* edge_vec_in, int* row_ptr, int* sender, float* edge_vec,
+                         int* perm, int* t_row_ptr, int* t_perm, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (n_nodes < 0 || n_edges < 0 || !row_ptr || !t_row_ptr ||
+      (n_edges > 0 && (!receiver || !sender_in || !edge_vec_in || !sender || !edge_vec || !t_perm))) {
+    set_error("etp_build_csr: bad argument");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (workspace_bytes < graph_workspace_bytes(n_nodes, n_edges) || (!workspace && workspace_bytes)) {
+    set_error("etp_build_csr: workspace smaller than etp_graph_workspace_bytes()");
+    return ETP_ERR_INVALID_ARG;
+  }
+  return build_csr(n_nodes, n_edges, receiver, sender_in, edge_vec_in, row_ptr, sender, edge_vec,
+                   perm, t_row_ptr, t_perm, workspace, workspace_bytes,
+                   static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,328 @@
+// Graph construction: brute-force neighbour list with a fixed float64 inclusion test, canonical
+// receiver-sorted CSR, and the transposed (sender-sorted) order. Integer outputs are
+// deterministic and bit-exact against any implementation of the same test (include/etp.h).
+#include <cub/cub.cuh>
+
+#include <cmath>
+#include <string>
+
+#include "etp_internal.h"
+
+namespace etp {
+namespace {
+
+struct CellParams {
+  double c[9];       // rows = lattice vectors
+  int n[3];          // images scanned per axis: S_a in [-n_a, n_a]
+  double rc2;        // float64(r_cut)^2 (exact: a float squared fits in a double)
+};
+
+// r = (pos[j] - pos[i]) + ((S0 c0 + S1 c1) + S2 c2); d2 = (rx rx + ry ry) + rz rz, no FMA.
+__device__ __forceinline__ bool pair_test(float3 pi, float3 pj, int s0, int s1, int s2,
+                                          const CellParams& cp, double* rx, double* ry, double* rz) {
+  const double a0 = static_cast<double>(s0), a1 = static_cast<double>(s1), a2 = static_cast<double>(s2);
+  const double sx = __dadd_rn(__dadd_rn(__dmul_rn(a0, cp.c[0]), __dmul_rn(a1, cp.c[3])), __dmul_rn(a2, cp.c[6]));
+  const double sy = __dadd_rn(__dadd_rn(__dmul_rn(a0, cp.c[1]), __dmul_rn(a1, cp.c[4])), __dmul_rn(a2, cp.c[7]));
+  const double sz = __dadd_rn(__dadd_rn(__dmul_rn(a0, cp.c[2]), __dmul_rn(a1, cp.c[5])), __dmul_rn(a2, cp.c[8]));
+  const double dx = __dadd_rn(__dsub_rn(static_cast<double>(pj.x), static_cast<double>(pi.x)), sx);
+  const double dy = __dadd_rn(__dsub_rn(static_cast<double>(pj.y), static_cast<double>(pi.y)), sy);
+  const double dz = __dadd_rn(__dsub_rn(static_cast<double>(pj.z), static_cast<double>(pi.z)), sz);
+  const double d2 = __dadd_rn(__dadd_rn(__dmul_rn(dx, dx), __dmul_rn(dy, dy)), __dmul_rn(dz, dz));
+  *rx = dx;
+  *ry = dy;
+  *rz = dz;
+  return d2 < cp.rc2;
+}
+
+__device__ __forceinline__ float3 load_pos(const float* pos, int i) {
+  return make_float3(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2]);
+}
+
+// Number of kept images for receiver i and sender j (S in lexicographic order).
+__device__ __forceinline__ int count_pair(float3 pi, float3 pj, bool same, const CellParams& cp) {
+  int c = 0;
+  double rx, ry, rz;
+  for (int s0 = -cp.n[0]; s0 <= cp.n[0]; ++s0)
+    for (int s1 = -cp.n[1]; s1 <= cp.n[1]; ++s1)
+      for (int s2 = -cp.n[2]; s2 <= cp.n[2]; ++s2) {
+        if (same && s0 == 0 && s1 == 0 && s2 == 0) continue;
+        c += pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz) ? 1 : 0;
+      }
+  return c;
+}
+
+// One warp per receiver: counts[i] = number of neighbours.
+__global__ void k_nbr_count(const float* __restrict__ pos, int n, CellParams cp, int* __restrict__ counts) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (i >= n) return;
+  const float3 pi = load_pos(pos, i);
+  int c = 0;
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    if (j < n) c += count_pair(pi, load_pos(pos, j), j == i, cp);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  if (lane == 0) counts[i] = c;
+}
+
+// One warp per receiver: writes the row in canonical (sender, S) order.
+__global__ void k_nbr_emit(const float* __restrict__ pos, int n, CellParams cp,
+                           const int* __restrict__ row_ptr, int* __restrict__ sender,
+                           float* __restrict__ edge_vec, int* __restrict__ shift) {
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (i >= n) return;
+  const float3 pi = load_pos(pos, i);
+  int base = row_ptr[i];
+  for (int j0 = 0; j0 < n; j0 += 32) {
+    const int j = j0 + lane;
+    const float3 pj = j < n ? load_pos(pos, j) : pi;
+    const int c = j < n ? count_pair(pi, pj, j == i, cp) : 0;
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (c > 0) {
+      int at = base + incl - c;
+      double rx, ry, rz;
+      for (int s0 = -cp.n[0]; s0 <= cp.n[0]; ++s0)
+        for (int s1 = -cp.n[1]; s1 <= cp.n[1]; ++s1)
+          for (int s2 = -cp.n[2]; s2 <= cp.n[2]; ++s2) {
+            if (j == i && s0 == 0 && s1 == 0 && s2 == 0) continue;
+            if (pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz)) {
+              sender[at] = j;
+              edge_vec[3 * at + 0] = static_cast<float>(rx);
+              edge_vec[3 * at + 1] = static_cast<float>(ry);
+              edge_vec[3 * at + 2] = static_cast<float>(rz);
+              if (shift) {
+                shift[3 * at + 0] = s0;
+                shift[3 * at + 1] = s1;
+                shift[3 * at + 2] = s2;
+              }
+              ++at;
+            }
+          }
+    }
+    base += total;
+  }
+}
+
+__global__ void k_iota(int* __restrict__ v, int n) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) v[k] = k;
+}
+
+// ptr[r] = first k with keys[k] >= r (keys sorted), r = 0..n_nodes.
+__global__ void k_lower_bound_ptr(const int* __restrict__ keys, int n_keys, int n_nodes, int* __restrict__ ptr) {
+  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r <= n_nodes; r += gridDim.x * blockDim.x) {
+    int lo = 0, hi = n_keys;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (keys[mid] < r) lo = mid + 1; else hi = mid;
+    }
+    ptr[r] = lo;
+  }
+}
+
+__global__ void k_gather_key(const int* __restrict__ key_src, const int* __restrict__ idx, int n,
+                             int* __restrict__ out) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) out[k] = key_src[idx[k]];
+}
+
+__global__ void k_gather_edges(const int* __restrict__ perm, int n, const int* __restrict__ sender_in,
+                               const float* __restrict__ vec_in, int* __restrict__ sender,
+                               float* __restrict__ vec) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
+    const int e = perm[k];
+    sender[k] = sender_in[e];
+    vec[3 * k + 0] = vec_in[3 * e + 0];
+    vec[3 * k + 1] = vec_in[3 * e + 1];
+    vec[3 * k + 2] = vec_in[3 * e + 2];
+  }
+}
+
+__global__ void k_check_range(const int* __restrict__ a, const int* __restrict__ b, int n, int n_nodes,
+                              int* __restrict__ flag) {
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) {
+    if (a[k] < 0 || a[k] >= n_nodes || b[k] < 0 || b[k] >= n_nodes) atomicOr(flag, 1);
+  }
+}
+
+int key_bits(int n_nodes) {
+  int b = 1;
+  while ((1LL << b) <= n_nodes) ++b;
+  return b;
+}
+
+struct GraphWs {
+  int* counts;   // n_nodes + 1
+  int* ka;
+  int* kb;
+  int* va;
+  int* vb;
+  int* pm;
+  int* flag;
+  void* cub_tmp;
+  size_t cub_bytes;
+};
+
+size_t cub_temp_bytes(int n_nodes, int max_edges) {
+  size_t scan_b = 0, sort_b = 0;
+  cub::DeviceScan::InclusiveSum(nullptr, scan_b, static_cast<const int*>(nullptr),
+                                static_cast<int*>(nullptr), n_nodes > 0 ? n_nodes : 1);
+  cub::DeviceRadixSort::SortPairs(nullptr, sort_b, static_cast<const int*>(nullptr),
+                                  static_cast<int*>(nullptr), static_cast<const int*>(nullptr),
+                                  static_cast<int*>(nullptr), max_edges > 0 ? max_edges : 1, 0,
+                                  key_bits(n_nodes));
+  return scan_b > sort_b ? scan_b : sort_b;
+}
+
+GraphWs carve(void* ws, int n_nodes, int max_edges) {
+  char* p = static_cast<char*>(ws);
+  GraphWs g;
+  const size_t eb = align256(sizeof(int) * static_cast<size_t>(max_edges > 0 ? max_edges : 1));
+  g.counts = reinterpret_cast<int*>(p);
+  p += align256(sizeof(int) * (static_cast<size_t>(n_nodes) + 1));
+  g.ka = reinterpret_cast<int*>(p); p += eb;
+  g.kb = reinterpret_cast<int*>(p); p += eb;
+  g.va = reinterpret_cast<int*>(p); p += eb;
+  g.vb = reinterpret_cast<int*>(p); p += eb;
+  g.pm = reinterpret_cast<int*>(p); p += eb;
+  g.flag = reinterpret_cast<int*>(p); p += 256;
+  g.cub_tmp = p;
+  g.cub_bytes = cub_temp_bytes(n_nodes, max_edges);
+  return g;
+}
+
+int grid_for(long long n, int threads) {
+  long long b = (n + threads - 1) / threads;
+  if (b < 1) b = 1;
+  if (b > 148 * 32) b = 148 * 32;
+  return static_cast<int>(b);
+}
+
+// t_perm = stable sort of canonical edge ids by sender; t_row_ptr from the sorted keys.
+etp_status transpose(int n_nodes, int n_edges, const int* sender, int* t_row_ptr, int* t_perm,
+                     GraphWs& g, cudaStream_t s) {
+  if (n_edges > 0) {
+    k_iota<<<grid_for(n_edges, 256), 256, 0, s>>>(g.va, n_edges);
+    size_t tb = g.cub_bytes;
+    cudaError_t e = cub::DeviceRadixSort::SortPairs(g.cub_tmp, tb, sender, g.kb, g.va, t_perm, n_edges,
+                                                    0, key_bits(n_nodes), s);
+    if (e != cudaSuccess) return cuda_status(e, "transpose sort");
+  }
+  k_lower_bound_ptr<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.kb, n_edges, n_nodes, t_row_ptr);
+  return cuda_status(cudaGetLastError(), "transpose");
+}
+
+}  // namespace
+
+size_t graph_workspace_bytes(int n_nodes, int max_edges) {
+  const size_t eb = align256(sizeof(int) * static_cast<size_t>(max_edges > 0 ? max_edges : 1));
+  return align256(sizeof(int) * (static_cast<size_t>(n_nodes) + 1)) + 5 * eb + 256 +
+         align256(cub_temp_bytes(n_nodes, max_edges));
+}
+
+etp_status neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,
+                     float r_cut, int max_edges, int* n_edges, int* row_ptr, int* sender,
+                     float* edge_vec, int* shift, int* t_row_ptr, int* t_perm, void* ws,
+                     size_t ws_bytes, cudaStream_t s) {
+  (void)ws_bytes;
+  CellParams cp;
+  for (int k = 0; k < 9; ++k) cp.c[k] = cell ? cell[k] : 0.0;
+  const double rc = static_cast<double>(r_cut);
+  cp.rc2 = rc * rc;
+  if (cell) {
+    const double* c = cell;
+    const double vol = std::fabs(c[0] * (c[4] * c[8] - c[5] * c[7]) - c[1] * (c[3] * c[8] - c[5] * c[6]) +
+                                 c[2] * (c[3] * c[7] - c[4] * c[6]));
+    for (int a = 0; a < 3; ++a) {
+      cp.n[a] = 0;
+      if (!pbc || !pbc[a]) continue;
+      const double* b = c + 3 * ((a + 1) % 3);
+      const double* d = c + 3 * ((a + 2) % 3);
+      const double cx = b[1] * d[2] - b[2] * d[1], cy = b[2] * d[0] - b[0] * d[2], cz = b[0] * d[1] - b[1] * d[0];
+      const double spacing = vol / std::sqrt(cx * cx + cy * cy + cz * cz);
+      if (!(spacing > 0.0)) {
+        set_error("etp_neighbors: degenerate cell");
+        return ETP_ERR_INVALID_ARG;
+      }
+      cp.n[a] = static_cast<int>(std::ceil(rc / spacing));
+    }
+  } else {
+    if (pbc && (pbc[0] || pbc[1] || pbc[2])) {
+      set_error("etp_neighbors: periodic axes need a cell");
+      return ETP_ERR_INVALID_ARG;
+    }
+    cp.n[0] = cp.n[1] = cp.n[2] = 0;
+  }
+  GraphWs g = carve(ws, n_nodes, max_edges);
+  cudaError_t e;
+  if (n_nodes > 0) {
+    const int warps = 4;
+    k_nbr_count<<<(n_nodes + warps - 1) / warps, 32 * warps, 0, s>>>(pos, n_nodes, cp, g.counts);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour count");
+    size_t tb = g.cub_bytes;
+    e = cub::DeviceScan::InclusiveSum(g.cub_tmp, tb, g.counts, row_ptr + 1, n_nodes, s);
+    if (e != cudaSuccess) return cuda_status(e, "neighbour scan");
+  }
+  if ((e = cudaMemsetAsync(row_ptr, 0, sizeof(int), s)) != cudaSuccess) return cuda_status(e, "memset");
+  int total = 0;
+  if ((e = cudaMemcpyAsync(&total, row_ptr + n_nodes, sizeof(int), cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_status(e, "read edge count");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_status(e, "neighbour count sync");
+  *n_edges = total;
+  if (total > max_edges) {
+    set_error("etp_neighbors: " + std::to_string(total) + " edges exceed max_edges");
+    return ETP_ERR_CAPACITY;
+  }
+  if (n_nodes > 0 && total > 0) {
+    const int warps = 4;
+    k_nbr_emit<<<(n_nodes + warps - 1) / warps, 32 * warps, 0, s>>>(pos, n_nodes, cp, row_ptr, sender,
+                                                                   edge_vec, shift);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour emit");
+  }
+  return transpose(n_nodes, total, sender, t_row_ptr, t_perm, g, s);
+}
+
+etp_status build_csr(int n_nodes, int n_edges, const int* receiver, const int* sender_in,
+                     const float* edge_vec_in, int* row_ptr, int* sender, float* edge_vec,
+                     int* perm, int* t_row_ptr, int* t_perm, void* ws, size_t ws_bytes,
+                     cudaStream_t s) {
+  (void)ws_bytes;
+  GraphWs g = carve(ws, n_nodes, n_edges);
+  cudaError_t e;
+  int* pm = perm ? perm : g.pm;
+  if (n_edges > 0) {
+    if ((e = cudaMemsetAsync(g.flag, 0, sizeof(int), s)) != cudaSuccess) return cuda_status(e, "memset");
+    k_check_range<<<grid_for(n_edges, 256), 256, 0, s>>>(receiver, sender_in, n_edges, n_nodes, g.flag);
+    int bad = 0;
+    if ((e = cudaMemcpyAsync(&bad, g.flag, sizeof(int), cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+      return cuda_status(e, "read flag");
+    if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_status(e, "build_csr sync");
+    if (bad) {
+      set_error("etp_build_csr: receiver or sender index out of [0, n_nodes)");
+      return ETP_ERR_BAD_GRAPH;
+    }
+    const int bits = key_bits(n_nodes);
+    k_iota<<<grid_for(n_edges, 256), 256, 0, s>>>(g.va, n_edges);
+    size_t tb = g.cub_bytes;
+    // LSD: stable by sender, then stable by receiver -> (receiver, sender, input index)
+    e = cub::DeviceRadixSort::SortPairs(g.cub_tmp, tb, sender_in, g.kb, g.va, g.vb, n_edges, 0, bits, s);
+    if (e != cudaSuccess) return cuda_status(e, "csr sort 1");
+    k_gather_key<<<grid_for(n_edges, 256), 256, 0, s>>>(receiver, g.vb, n_edges, g.ka);
+    tb = g.cub_bytes;
+    e = cub::DeviceRadixSort::SortPairs(g.cub_tmp, tb, g.ka, g.kb, g.vb, pm, n_edges, 0, bits, s);
+    if (e != cudaSuccess) return cuda_status(e, "csr sort 2");
+    k_gather_edges<<<grid_for(n_edges, 256), 256, 0, s>>>(pm, n_edges, sender_in, edge_vec_in, sender, edge_vec);
+  }
+  k_lower_bound_ptr<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.kb, n_edges, n_nodes, row_ptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "build_csr");
+  return transpose(n_nodes, n_edges, sender, t_row_ptr, t_perm, g, s);
+}
+
+}  // namespace etp

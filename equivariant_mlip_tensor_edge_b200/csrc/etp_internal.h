@@ -1,0 +1,62 @@
+// Internal declarations shared by the library's translation units (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "etp.h"
+
+namespace etp {
+
+constexpr int kNumBasis = 8;     // radial basis functions (fixed at compile time)
+constexpr int kBatch = 4;        // channels per register batch (one float4 per component)
+constexpr int kMaxL = 3;
+
+struct Ctx {
+  int lmax = 0;
+  int channels = 0;
+  int dim = 0;
+  int n_paths = 0;
+  int cg_nnz = 0;
+  int sum_2l3p1 = 0;
+  float r_cut = 0.f;
+};
+
+// Error message of the last failing call on this host thread.
+void set_error(const std::string& msg);
+etp_status cuda_status(cudaError_t e, const char* what);
+
+// ---- conv kernels (etp_conv.cu)
+etp_status launch_forward(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr,
+                          const int* sender, const float* edge_vec, const float* x,
+                          const float* W, float* out, cudaStream_t s);
+etp_status launch_backward(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr,
+                           const int* sender, const float* edge_vec, const int* t_row_ptr,
+                           const int* t_perm, const float* x, const float* W,
+                           const float* grad_out, float* grad_x, float* grad_edge_vec,
+                           int* recv_map, cudaStream_t s);
+etp_status launch_radial_weights(const Ctx& c, int n_edges, const float* edge_vec,
+                                 const float* W, float* w_out, cudaStream_t s);
+etp_status launch_forces(int n_nodes, int n_edges, const int* row_ptr, const int* t_row_ptr,
+                         const int* t_perm, const float* grad_edge_vec, float* forces,
+                         cudaStream_t s);
+// Returns ETP_OK or ETP_ERR_BAD_GRAPH (synchronises s). scratch: >= n_edges ints + 1.
+etp_status validate_graph(int n_nodes, int n_edges, const int* row_ptr, const int* sender,
+                          const int* t_row_ptr, const int* t_perm, int* scratch, cudaStream_t s);
+
+// ---- graph kernels (etp_graph.cu)
+size_t graph_workspace_bytes(int n_nodes, int max_edges);
+etp_status neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,
+                     float r_cut, int max_edges, int* n_edges, int* row_ptr, int* sender,
+                     float* edge_vec, int* shift, int* t_row_ptr, int* t_perm, void* ws,
+                     size_t ws_bytes, cudaStream_t s);
+etp_status build_csr(int n_nodes, int n_edges, const int* receiver, const int* sender_in,
+                     const float* edge_vec_in, int* row_ptr, int* sender, float* edge_vec,
+                     int* perm, int* t_row_ptr, int* t_perm, void* ws, size_t ws_bytes,
+                     cudaStream_t s);
+
+inline size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+}  // namespace etp

@@ -1,0 +1,293 @@
+"""Build-time generator of the unrolled per-path device code (``generated/etp_paths.h``).
+
+Emits, for every supported l_max (in = SH = out = L):
+  * the real spherical harmonics Y_lm(n) of a unit vector as explicit polynomials
+    (component normalisation, sum_m Y_lm^2 = 2l + 1, m = -l..l, z polar), and the
+    contraction sum_m gY_m dY_m/dr needed by the backward pass;
+  * the path list (l1, l2, l3), lexicographic, triangle rule, l1 + l2 + l3 even;
+  * per path, the real-basis Clebsch-Gordan nonzeros as float immediates inside
+    straight-line forward and backward contraction code.
+
+Independent of the float64 oracle by construction: Clebsch-Gordan values come
+from ``sympy.physics.wigner.clebsch_gordan`` and the harmonic polynomials from a
+least-squares fit of homogeneous polynomials to ``scipy.special.sph_harm_y``
+(a homogeneous polynomial of degree l is fixed by its values on the sphere),
+each moved to the real basis by the change of basis written out below.
+
+Run:  python gen_paths.py  (writes generated/etp_paths.h next to this file)
+"""
+import itertools
+import math
+import os
+import struct
+import sys
+
+import numpy as np
+import scipy.special as sps
+from sympy import N as sym_n
+from sympy.physics.wigner import clebsch_gordan
+
+LMAX_SUPPORTED = (1, 2, 3)
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+# ---------------------------------------------------------------- bases
+
+def complex_to_real(l):
+    """U with Y_real = U Y_complex; real m>0 ~ cos(m phi), m<0 ~ sin(|m| phi)."""
+    u = np.zeros((2 * l + 1, 2 * l + 1), dtype=complex)
+    r = math.sqrt(0.5)
+    u[l, l] = 1.0
+    for m in range(1, l + 1):
+        sgn = -1.0 if m % 2 else 1.0
+        u[l + m, l + m] = sgn * r
+        u[l + m, l - m] = r
+        u[l - m, l - m] = 1j * r
+        u[l - m, l + m] = -1j * sgn * r
+    return u
+
+
+def real_cg(l1, l2, l3):
+    c = np.zeros((2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1), dtype=complex)
+    for m1 in range(-l1, l1 + 1):
+        for m2 in range(-l2, l2 + 1):
+            m3 = m1 + m2
+            if abs(m3) <= l3:
+                c[m1 + l1, m2 + l2, m3 + l3] = float(sym_n(clebsch_gordan(l1, l2, l3, m1, m2, m3), 30))
+    u1, u2, u3 = complex_to_real(l1), complex_to_real(l2), complex_to_real(l3)
+    r = np.einsum("ai,bj,ck,ijk->abc", u1.conj(), u2.conj(), u3, c)
+    assert np.abs(r.imag).max() < 1e-12
+    r = r.real
+    r[np.abs(r) < 1e-12] = 0.0
+    return r
+
+
+def monomials(l):
+    return [(a, b, l - a - b) for a in range(l, -1, -1) for b in range(l - a, -1, -1)]
+
+
+def sh_polynomials(l):
+    """Coefficients over ``monomials(l)`` of Y_lm (component normalised), rows m=-l..l."""
+    rng = np.random.default_rng(1234 + l)
+    v = rng.standard_normal((400, 3))
+    v /= np.linalg.norm(v, axis=1, keepdims=True)
+    theta, phi = np.arccos(np.clip(v[:, 2], -1, 1)), np.arctan2(v[:, 1], v[:, 0])
+    yc = np.stack([sps.sph_harm_y(l, m, theta, phi) for m in range(-l, l + 1)], axis=0)
+    yr = (complex_to_real(l) @ yc).real * math.sqrt(4.0 * math.pi)
+    mons = monomials(l)
+    a = np.stack([v[:, 0] ** p * v[:, 1] ** q * v[:, 2] ** s for p, q, s in mons], axis=1)
+    coef, *_ = np.linalg.lstsq(a, yr.T, rcond=None)
+    assert np.abs(a @ coef - yr.T).max() < 1e-12, l
+    coef[np.abs(coef) < 1e-12] = 0.0
+    return coef.T  # [2l+1, n_monomials]
+
+
+# ---------------------------------------------------------------- emit helpers
+
+def repr_f32(f):
+    # hexadecimal float literal, exact for float32 values
+    return float.hex(float(f)) + "f"
+
+
+def idx(l, m):
+    return l * l + l + m
+
+
+def paths_for(lmax):
+    return [(l1, l2, l3) for l1 in range(lmax + 1) for l2 in range(lmax + 1) for l3 in range(lmax + 1)
+            if abs(l1 - l2) <= l3 <= l1 + l2 and (l1 + l2 + l3) % 2 == 0]
+
+
+def mono_expr(p, q, s, names=("nx", "ny", "nz")):
+    parts = []
+    for n, e in zip(names, (p, q, s)):
+        parts += [n] * e
+    return "*".join(parts) if parts else "1.0f"
+
+
+# ---------------------------------------------------------------- SH code
+
+def emit_sh(out, lmax):
+    out.append(f"// real spherical harmonics up to l = {lmax}: Y[l*l + l + m] of the unit vector (nx, ny, nz)")
+    out.append(f"__device__ __forceinline__ void sh_eval_{lmax}(float nx, float ny, float nz, float* Y) {{")
+    out.append("  Y[0] = 1.0f;")
+    for l in range(1, lmax + 1):
+        coef = sh_polynomials(l)
+        mons = monomials(l)
+        for m in range(-l, l + 1):
+            terms = [(coef[m + l, k], mons[k]) for k in range(len(mons)) if coef[m + l, k] != 0.0]
+            expr = " + ".join(f"{repr_f32(np.float32(c))}*({mono_expr(*mo)})" for c, mo in terms)
+            out.append(f"  Y[{idx(l, m)}] = {expr};")
+    out.append("}")
+    # gradient contraction: given gY (dL/dY), returns G = sum_m gY_m grad P_m(n) and
+    # S = sum_m gY_m l P_m(n); then dL/dr = (G - S n) / d
+    out.append(f"__device__ __forceinline__ void sh_grad_{lmax}(float nx, float ny, float nz, const float* gY,")
+    out.append("                                              float& Gx, float& Gy, float& Gz, float& S) {")
+    out.append("  Gx = 0.0f; Gy = 0.0f; Gz = 0.0f; S = 0.0f;")
+    for l in range(1, lmax + 1):
+        coef = sh_polynomials(l)
+        mons = monomials(l)
+        for m in range(-l, l + 1):
+            i = idx(l, m)
+            terms = [(coef[m + l, k], mons[k]) for k in range(len(mons)) if coef[m + l, k] != 0.0]
+            gx, gy, gz, pv = [], [], [], []
+            for c, (p, q, s) in terms:
+                pv.append(f"{repr_f32(np.float32(c))}*({mono_expr(p, q, s)})")
+                if p:
+                    gx.append(f"{repr_f32(np.float32(c * p))}*({mono_expr(p - 1, q, s)})")
+                if q:
+                    gy.append(f"{repr_f32(np.float32(c * q))}*({mono_expr(p, q - 1, s)})")
+                if s:
+                    gz.append(f"{repr_f32(np.float32(c * s))}*({mono_expr(p, q, s - 1)})")
+            out.append(f"  {{ const float g = gY[{i}];")
+            for name, lst in (("Gx", gx), ("Gy", gy), ("Gz", gz)):
+                if lst:
+                    out.append(f"    {name} = fmaf(g, {' + '.join(lst)}, {name});")
+            out.append(f"    S = fmaf(g * {float(l):.1f}f, {' + '.join(pv)}, S); }}")
+    out.append("}")
+
+
+# ---------------------------------------------------------------- path code
+
+def emit_paths(out, lmax):
+    paths = paths_for(lmax)
+    P = len(paths)
+    D = (lmax + 1) ** 2
+    cgs = [real_cg(*p) for p in paths]
+    nnz = sum(int(np.count_nonzero(c)) for c in cgs)
+    s3 = sum(2 * l3 + 1 for _, _, l3 in paths)
+    out.append(f"// ---- l_max = {lmax}: {P} paths, {nnz} real-CG nonzeros")
+    out.append(f"template <> struct PathSet<{lmax}> {{")
+    out.append(f"  static constexpr int L = {lmax};")
+    out.append(f"  static constexpr int P = {P};")
+    out.append(f"  static constexpr int D = {D};")
+    out.append(f"  static constexpr int NNZ = {nnz};")
+    out.append(f"  static constexpr int SUM_2L3P1 = {s3};")
+    out.append("};")
+    trip = ", ".join(f"{a},{b},{c}" for a, b, c in paths)
+    out.append(f"static const int kPathL_{lmax}[{3 * P}] = {{{trip}}};")
+
+    # forward: acc[l3 m3][k] += w_p[k] * sum_{m1,m2} C Y[l2 m2] x[l1 m1][k]
+    out.append("template <int K, class WF>")
+    out.append(f"__device__ __forceinline__ void tp_fwd_{lmax}(const float* Y, WF&& wfetch,")
+    out.append(f"    const float (&x)[{D}][K], float (&acc)[{D}][K]) {{")
+    for p, ((l1, l2, l3), c) in enumerate(zip(paths, cgs)):
+        out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
+        out.append("    float wp[K]; wfetch(" + str(p) + ", wp);")
+        # M[m3][m1] = sum_m2 C[m1,m2,m3] Y[l2,m2]
+        mnz = []
+        for m3 in range(2 * l3 + 1):
+            for m1 in range(2 * l1 + 1):
+                terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
+                if not terms:
+                    continue
+                if l2 == 0:
+                    e = repr_f32(np.float32(terms[0][0]))
+                else:
+                    e = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                out.append(f"    const float M{m3}_{m1} = {e};")
+                mnz.append((m3, m1))
+        scale_x = (2 * l1 + 1) < (2 * l3 + 1)
+        out.append("    #pragma unroll")
+        out.append("    for (int k = 0; k < K; ++k) {")
+        if scale_x:
+            for m1 in range(2 * l1 + 1):
+                out.append(f"      const float xs{m1} = wp[k] * x[{idx(l1, m1 - l1)}][k];")
+            for m3 in range(2 * l3 + 1):
+                for (a, b) in mnz:
+                    if a == m3:
+                        out.append(f"      acc[{idx(l3, m3 - l3)}][k] = fmaf(M{a}_{b}, xs{b}, acc[{idx(l3, m3 - l3)}][k]);")
+        else:
+            for m3 in range(2 * l3 + 1):
+                row = [(a, b) for (a, b) in mnz if a == m3]
+                if not row:
+                    continue
+                a, b = row[0]
+                out.append(f"      float s{m3} = M{a}_{b} * x[{idx(l1, b - l1)}][k];")
+                for a, b in row[1:]:
+                    out.append(f"      s{m3} = fmaf(M{a}_{b}, x[{idx(l1, b - l1)}][k], s{m3});")
+                out.append(f"      acc[{idx(l3, m3 - l3)}][k] = fmaf(wp[k], s{m3}, acc[{idx(l3, m3 - l3)}][k]);")
+        out.append("    }")
+        out.append("  }")
+    out.append("}")
+
+    # backward (one edge, K channels):
+    #   v[m1]   = sum_m3 M[m3][m1] g[l3 m3]
+    #   gx      += w v;   gw = sum_m1 x[l1 m1] v[m1];   accd += wd gw
+    #   gY[l2 m2] += w sum_{m1,m3} C[m1,m2,m3] x[l1 m1] g[l3 m3]
+    out.append("template <int K, class WF>")
+    out.append(f"__device__ __forceinline__ void tp_bwd_{lmax}(const float* Y, WF&& wfetch,")
+    out.append(f"    const float (&x)[{D}][K], const float (&g)[{D}][K], float (&gx)[{D}][K],")
+    out.append(f"    float* gY, float& accd) {{")
+    for p, ((l1, l2, l3), c) in enumerate(zip(paths, cgs)):
+        out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
+        out.append("    float wp[K], wdp[K]; wfetch(" + str(p) + ", wp, wdp);")
+        mnz = []
+        for m3 in range(2 * l3 + 1):
+            for m1 in range(2 * l1 + 1):
+                terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
+                if not terms:
+                    continue
+                if l2 == 0:
+                    e = repr_f32(np.float32(terms[0][0]))
+                else:
+                    e = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                out.append(f"    const float M{m3}_{m1} = {e};")
+                mnz.append((m3, m1))
+        out.append("    #pragma unroll")
+        out.append("    for (int k = 0; k < K; ++k) {")
+        for m1 in range(2 * l1 + 1):
+            col = [(a, b) for (a, b) in mnz if b == m1]
+            if not col:
+                out.append(f"      const float v{m1} = 0.0f;")
+                continue
+            a, b = col[0]
+            out.append(f"      float v{m1} = M{a}_{b} * g[{idx(l3, a - l3)}][k];")
+            for a, b in col[1:]:
+                out.append(f"      v{m1} = fmaf(M{a}_{b}, g[{idx(l3, a - l3)}][k], v{m1});")
+        for m1 in range(2 * l1 + 1):
+            out.append(f"      gx[{idx(l1, m1 - l1)}][k] = fmaf(wp[k], v{m1}, gx[{idx(l1, m1 - l1)}][k]);")
+        out.append(f"      float gw = x[{idx(l1, -l1)}][k] * v0;")
+        for m1 in range(1, 2 * l1 + 1):
+            out.append(f"      gw = fmaf(x[{idx(l1, m1 - l1)}][k], v{m1}, gw);")
+        out.append("      accd = fmaf(wdp[k], gw, accd);")
+        if l2 > 0:
+            # gY[l2 m2] += w * sum C x g
+            for m2 in range(2 * l2 + 1):
+                terms = [(c[m1, m2, m3], m1, m3) for m1 in range(2 * l1 + 1) for m3 in range(2 * l3 + 1)
+                         if c[m1, m2, m3] != 0.0]
+                if not terms:
+                    continue
+                v, a, b = terms[0]
+                out.append(f"      float q{m2} = {repr_f32(np.float32(v))} * (x[{idx(l1, a - l1)}][k] * g[{idx(l3, b - l3)}][k]);")
+                for v, a, b in terms[1:]:
+                    out.append(f"      q{m2} = fmaf({repr_f32(np.float32(v))}, x[{idx(l1, a - l1)}][k] * g[{idx(l3, b - l3)}][k], q{m2});")
+                out.append(f"      gY[{idx(l2, m2 - l2)}] = fmaf(wp[k], q{m2}, gY[{idx(l2, m2 - l2)}]);")
+        out.append("    }")
+        out.append("  }")
+    out.append("}")
+    return P, nnz, s3
+
+
+def generate():
+    out = ["// GENERATED by gen_paths.py -- do not edit.",
+           "// Real-basis Clebsch-Gordan contractions and real spherical harmonics, unrolled per path.",
+           "#pragma once",
+           "namespace etp_gen {",
+           "template <int L> struct PathSet;"]
+    for lmax in LMAX_SUPPORTED:
+        emit_sh(out, lmax)
+        emit_paths(out, lmax)
+    out.append("}  // namespace etp_gen")
+    return "\n".join(out) + "\n"
+
+
+if __name__ == "__main__":
+    dst = os.path.join(HERE, "generated", "etp_paths.h")
+    os.makedirs(os.path.dirname(dst), exist_ok=True)
+    text = generate()
+    if len(sys.argv) > 1 and sys.argv[1] == "--check":
+        sys.exit(0 if os.path.exists(dst) and open(dst).read() == text else 1)
+    with open(dst, "w") as f:
+        f.write(text)
+    print("wrote", dst)

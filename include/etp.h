@@ -1,0 +1,164 @@
+/*
+ * etp.h -- C ABI of the B200 equivariant edge tensor-product convolution library (libetp.so).
+ *
+ * The operation (see "Fast and Accurate Foundation Models for Equivariant MLIPs", section VII,
+ * and "FlashCart", Fig. 3 caption, Table C1 and Fig. D1, for the pages that name it; the
+ * formulas are the textbook ones):
+ *
+ *   for each receiver i and each edge e = (i <- j, S) of its CSR row:
+ *     r_e = pos[j] - pos[i] + S . cell        (receiver -> sender),  d = |r_e|,  n = r_e / d
+ *     Y_l2(n)  real spherical harmonics, component normalisation (sum_m Y_lm^2 = 2l+1), z polar
+ *     R_b(d)   = (2/r_c) sin(b pi d / r_c) / d * u(d / r_c),  b = 1..n_basis,
+ *     u(t)     = 1 - 28 t^6 + 48 t^7 - 21 t^8 for t < 1, else 0          (p = 6 envelope)
+ *     w_{e,p,u} = sum_b R_b(d) W[b, p, u]                                 (radial projection)
+ *     out[i, l3, m3, u] += w_{e,p,u} sum_{m1,m2} C^{l1 l2 l3}_{m1 m2 m3} x[j, l1, m1, u] Y_{l2 m2}(n)
+ *
+ *   with C the real-basis Clebsch-Gordan coefficients, paths p = (l1, l2, l3) enumerated
+ *   lexicographically over (input block, l2 = 0..sh_lmax, output block) with the triangle rule
+ *   and parity p1 (-1)^l2 = p3, and "uvu" channel pairing (output channel = input channel).
+ *
+ * Layouts (all row-major, 32-bit):
+ *   node features x, out, grad_x, grad_out : [n_nodes][dim], dim = C (L+1)^2; the row holds the
+ *       blocks l = 0..L in order, block l is [m = -l..l][u = 0..C-1] (channels contiguous):
+ *       element (l, m, u) sits at (l*l + l + m) * C + u.
+ *   W           : [n_basis][n_paths][C]
+ *   edge arrays : receiver-sorted CSR. row_ptr [n_nodes+1], sender [n_edges], edge_vec [n_edges][3]
+ *                 (float32 r_e). Canonical edge order: (receiver, sender, S0, S1, S2).
+ *   transposed  : t_row_ptr [n_nodes+1] (edges per sender), t_perm [n_edges]: the edge ids in
+ *                 (sender, receiver, S) order.
+ *
+ * Conventions.
+ *   Pointers: every array argument is a CUDA DEVICE pointer owned by the caller unless the
+ *   comment says "host". The library allocates no device memory; scratch comes from the caller
+ *   through `workspace` (size from the matching *_workspace_bytes query, 256-byte aligned).
+ *   Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Calls are
+ *   asynchronous on that stream unless documented otherwise.
+ *   Outputs are overwritten, never accumulated into.
+ *   Errors: every call returns an etp_status; no call throws or traps. ETP_ERR_CUDA reports a
+ *   launch error (no implicit synchronisation). etp_last_error() returns a thread-local message
+ *   for the last failing call on the calling host thread.
+ *   Thread safety: a handle is immutable after etp_create; concurrent calls on different
+ *   streams with distinct output and workspace buffers are safe.
+ *   Graph validation: with the environment variable ETP_VALIDATE=1, etp_forward and etp_backward
+ *   first check the CSR arrays on the device (monotone row pointers, indices in range, t_perm a
+ *   permutation) and return ETP_ERR_BAD_GRAPH without touching the outputs; this synchronises
+ *   the stream.
+ */
+#ifndef ETP_H
+#define ETP_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct etp_ctx* etp_handle;
+
+typedef enum {
+  ETP_OK = 0,
+  ETP_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned pointer, workspace too small */
+  ETP_ERR_IRREPS = 2,        /* malformed irreps string */
+  ETP_ERR_UNSUPPORTED = 3,   /* well-formed but outside what the kernels implement */
+  ETP_ERR_BAD_GRAPH = 4,     /* CSR arrays failed validation (ETP_VALIDATE=1) */
+  ETP_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
+  ETP_ERR_CAPACITY = 6       /* an output buffer is smaller than the result (n_edges reported) */
+} etp_status;
+
+typedef struct {
+  int lmax;          /* L: irreps_in = irreps_out = C x (0e + 1o + ... ), SH lmax = L */
+  int channels;      /* C */
+  int dim_in;        /* C (L+1)^2 */
+  int dim_out;       /* C (L+1)^2 */
+  int n_paths;       /* P */
+  int n_basis;
+  int weight_numel;  /* n_basis * P * C */
+  int cg_nnz;        /* real-CG nonzeros summed over the path set */
+  int sum_2l3p1;     /* sum over paths of 2 l3 + 1 */
+  float r_cut;
+} etp_info_t;
+
+/* Create a convolution handle. Host-only, synchronous, allocates host memory only.
+ * irreps_in / irreps_out: "CxL1p+CxL2p+..." strings, e.g. "64x0e+64x1o+64x2e".
+ * Supported: every block has the same multiplicity C (C % 4 == 0, 4 <= C <= 256), blocks are
+ * l = 0..L in order with parity (-1)^l, irreps_out == irreps_in, sh_lmax == L, L in {1,2,3},
+ * n_basis == 8, r_cut > 0. Malformed strings -> ETP_ERR_IRREPS; anything else outside the
+ * supported set -> ETP_ERR_UNSUPPORTED. The path list is the enumeration described above. */
+etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_basis,
+                      float r_cut, etp_handle* out);
+
+/* Release a handle (host memory only). NULL is accepted. */
+etp_status etp_destroy(etp_handle h);
+
+/* Dimensions and path statistics of a handle (info: host pointer). */
+etp_status etp_get_info(etp_handle h, etp_info_t* info);
+
+/* Static text for a status code, and the last detailed error message of this host thread. */
+const char* etp_status_string(etp_status s);
+const char* etp_last_error(void);
+
+/* Bytes of device workspace etp_forward / etp_backward need for a graph of this size. */
+size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges);
+
+/* Fused forward: out[n_nodes][dim_out] = convolution of x[n_nodes][dim_in] over the CSR graph.
+ * Spherical harmonics, radial basis, radial projection, Clebsch-Gordan contraction and the
+ * per-receiver segmented sum run in one kernel pass; receivers without edges get zero rows.
+ * Edges with d >= r_cut contribute zero (u = 0). workspace may be NULL when
+ * etp_workspace_bytes returns 0. */
+etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                       const int* sender, const float* edge_vec, const float* x, const float* W,
+                       float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Fused backward (vector-Jacobian product of etp_forward for the cotangent grad_out):
+ *   grad_x[n_nodes][dim_in]        = dL/dx,        L = <grad_out, out>
+ *   grad_edge_vec[n_edges][3]      = dL/dr_e       (indexed by canonical edge id)
+ * Runs over the transposed (sender-sorted) order so grad_x is a segmented sum per sender.
+ * grad_x or grad_edge_vec may be NULL to skip that output (not both). */
+etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                        const int* sender, const float* edge_vec, const int* t_row_ptr,
+                        const int* t_perm, const float* x, const float* W, const float* grad_out,
+                        float* grad_x, float* grad_edge_vec, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Radial projection alone: w_out[n_edges][n_paths][C] = sum_b R_b(|r_e|) W[b][p][u]. */
+etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, const float* W,
+                              float* w_out, void* stream);
+
+/* Forces from edge-vector gradients, F = -dL/dpos with r_e = pos[sender] - pos[receiver] + S:
+ *   F[k] = sum_{e: receiver(e)=k} grad_edge_vec[e] - sum_{e: sender(e)=k} grad_edge_vec[e],
+ * summed in canonical (row) order and transposed (t_perm) order respectively. */
+etp_status etp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* t_row_ptr,
+                      const int* t_perm, const float* grad_edge_vec, float* forces, void* stream);
+
+/* ---- graph construction (integer outputs are bit-exact against a float64 brute force) ---- */
+
+/* Device workspace for etp_neighbors / etp_build_csr with up to max_edges edges. */
+size_t etp_graph_workspace_bytes(int n_nodes, int max_edges);
+
+/* Neighbour list and canonical CSR. pos: [n_nodes][3] float32 (device). cell: 9 doubles,
+ * rows = lattice vectors (HOST pointer; NULL for no cell). pbc: 3 ints (HOST pointer; NULL = none
+ * periodic). An edge (i <- j, S) is kept iff, in float64 without fused multiply-add,
+ *     s = (S0 cell[0] + S1 cell[1]) + S2 cell[2];  r = (pos[j] - pos[i]) + s;
+ *     (r_x r_x + r_y r_y) + r_z r_z < r_cut^2,  and not (i == j and S == 0),
+ * scanning every image with |S_a| <= ceil(r_cut / plane spacing_a) on periodic axes.
+ * Outputs (device, capacity max_edges): row_ptr, sender, edge_vec (= float32(r)), shift
+ * [max_edges][3] (may be NULL), t_row_ptr, t_perm. *n_edges (HOST) receives the edge count;
+ * this call synchronises `stream` once to read it. If the count exceeds max_edges the call
+ * returns ETP_ERR_CAPACITY after filling row_ptr only. */
+etp_status etp_neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,
+                         float r_cut, int max_edges, int* n_edges, int* row_ptr, int* sender,
+                         float* edge_vec, int* shift, int* t_row_ptr, int* t_perm,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Canonical CSR from a given edge list in any order (receiver[e], sender[e], edge_vec_in[e]):
+ * stable sort by (receiver, sender); perm[k] = input index of canonical edge k (may be NULL). */
+etp_status etp_build_csr(int n_nodes, int n_edges, const int* receiver, const int* sender_in,
+                         const float* edge_vec_in, int* row_ptr, int* sender, float* edge_vec,
+                         int* perm, int* t_row_ptr, int* t_perm, void* workspace,
+                         size_t workspace_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ETP_H */

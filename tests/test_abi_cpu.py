@@ -1,0 +1,93 @@
+"""C-ABI checks that need no GPU: the library loads, exports every declared symbol, and its
+host-side logic (irreps parsing, path enumeration, argument checks) behaves as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import equivariant_mlip_tensor_edge_b200 as etp
+from oracle.conv import ConvSpec, flop_counts
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "etp.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(etp_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return etp.load_library()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in etp.SIGNATURES, f"{n} has no ctypes signature in the binding"
+
+
+def _create(irin, lmax, irout, nb=8, rc=5.0):
+    lib = etp.load_library()
+    h = ctypes.c_void_p()
+    st = lib.etp_create(irin.encode() if irin is not None else None, lmax,
+                        irout.encode() if irout is not None else None, nb, rc, ctypes.byref(h))
+    if st == 0:
+        lib.etp_destroy(h)
+    return st
+
+
+def test_create_status_codes():
+    assert _create("64x0e+64x1o+64x2e", 2, "64x0e+64x1o+64x2e") == 0
+    assert _create("8x0e + 8x1o", 1, "8x0e+8x1o") == 0
+    assert _create("64x0e+64x1q", 1, "64x0e+64x1o") == 2        # malformed
+    assert _create("64x0e++64x1o", 1, "64x0e+64x1o") == 2
+    assert _create(None, 1, "64x0e+64x1o") == 2
+    assert _create("64x0e+64x1e", 1, "64x0e+64x1e") == 3        # parity not (-1)^l
+    assert _create("64x0e+32x1o", 1, "64x0e+32x1o") == 3        # mixed multiplicity
+    assert _create("6x0e+6x1o", 1, "6x0e+6x1o") == 3            # C % 4 != 0
+    assert _create("8x0e+8x1o", 1, "8x0e+8x1o", nb=6) == 3      # n_basis != 8
+    assert _create("8x0e+8x1o", 2, "8x0e+8x1o") == 3            # sh_lmax != L
+    assert _create("8x0e+8x1o+8x2e+8x3o+8x4e", 4, "8x0e+8x1o+8x2e+8x3o+8x4e") == 3
+    assert _create("8x0e+8x1o", 1, "8x0e+8x1o", rc=-1.0) == 1
+
+
+@pytest.mark.parametrize("lmax,c", [(1, 8), (2, 64), (3, 128)])
+def test_info_matches_independent_path_enumeration(lmax, c):
+    irr = "+".join(f"{c}x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
+    conv = etp.EdgeConv(irr, lmax, irr, 8, 5.0)
+    spec = ConvSpec(irr, lmax, irr, 8, 5.0)
+    fc = flop_counts(spec)
+    assert conv.info["n_paths"] == len(spec.paths)
+    assert conv.info["cg_nnz"] == fc["nnz"]
+    assert conv.info["sum_2l3p1"] == fc["sum_2l3p1"]
+    assert conv.info["dim_in"] == spec.dim_in == conv.info["dim_out"]
+    assert conv.info["weight_numel"] == 8 * len(spec.paths) * c
+    assert conv.workspace_bytes(100, 1000) >= 2 * 4 * 1000
+
+
+def test_status_strings_and_errors(lib):
+    for s in range(7):
+        assert lib.etp_status_string(s)
+    with pytest.raises(etp.EtpError) as ei:
+        etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x2o", 8, 5.0)
+    assert ei.value.status == 3
+    assert "etp_create" in str(ei.value)
+
+
+def test_null_arguments_rejected_without_cuda(lib):
+    # argument checks happen on the host before any CUDA call
+    conv = etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x1o", 8, 4.0)
+    st = lib.etp_forward(conv._h, 10, 5, None, None, None, None, None, None, None, 0, None)
+    assert st == 1
+    st = lib.etp_forward(None, 10, 5, None, None, None, None, None, None, None, 0, None)
+    assert st == 1
+    st = lib.etp_backward(conv._h, 10, 5, None, None, None, None, None, None, None, None, None, None, None, 0, None)
+    assert st == 1
+    assert lib.etp_forces(-1, 0, None, None, None, None, None, None) == 1
+    assert lib.etp_neighbors(None, -1, None, None, 1.0, 0, None, None, None, None, None, None, None, None, 0,
+                             None) == 1

@@ -1,0 +1,330 @@
+"""GPU parity: every kernel of libetp against the float64 oracle, through the C ABI.
+
+Integer graph arrays must match bit for bit; floating outputs within the per-irrep-block bound
+max|gpu - ref| <= 1e-5 max|ref| (grad_edge_vec and forces: over the whole array). Full outputs
+on the small workloads (several 32-edge tiles with a ragged tail); sampled receivers/senders,
+computed one by one by the oracle, on the full-size ones, in the launch configuration the
+benchmark uses.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import workloads
+from oracle.conv import conv_forward, conv_vjp
+from oracle.graph import forces_from_edge_grads
+from oracle.radial import radial
+from tests._oracle_side import (assert_blocks_close, assert_close_rel, forward_ref, full_graph, given_graph,
+                                rows_subgraph, sampled_rows, sender_edges, spec_of)
+
+torch = pytest.importorskip("torch")
+etp = pytest.importorskip("equivariant_mlip_tensor_edge_b200")
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+N_SAMPLE = 48
+
+
+@pytest.fixture(scope="module")
+def wls():
+    cache = {}
+
+    def get(name):
+        if name not in cache:
+            cache[name] = workloads.make(name)
+        return cache[name]
+    return get
+
+
+def _gpu_graph(wl):
+    if wl.given_receiver is not None:
+        return etp.build_csr(wl.n_nodes, torch.from_numpy(wl.given_receiver).to(DEV),
+                             torch.from_numpy(wl.given_sender).to(DEV), torch.from_numpy(wl.given_edge_vec).to(DEV))
+    return etp.neighbors(torch.from_numpy(wl.pos).to(DEV), float(wl.r_cut), cell=wl.cell, pbc=wl.pbc)
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _conv(wl):
+    return etp.EdgeConv(wl.irreps, wl.lmax, wl.irreps, wl.n_basis, float(wl.r_cut))
+
+
+def _edge_keys(receiver, sender, shift, n_nodes):
+    s = np.asarray(shift, np.int64) + 2
+    return ((np.asarray(receiver, np.int64) * n_nodes + np.asarray(sender, np.int64)) * 125
+            + s[:, 0] * 25 + s[:, 1] * 5 + s[:, 2])
+
+
+def _gpu_receivers(g):
+    return np.repeat(np.arange(g.n_nodes), np.diff(_np(g.row_ptr)))
+
+
+# ------------------------------------------------------------------ graph
+
+@pytest.mark.parametrize("name", ["tiny", "diamond1k"])
+def test_neighbors_bit_exact_full(wls, name):
+    wl = wls(name)
+    ref = full_graph(wl)
+    g = _gpu_graph(wl)
+    assert g.n_edges == len(ref["sender"])
+    assert np.array_equal(_np(g.row_ptr), ref["row_ptr"])
+    assert np.array_equal(_np(g.sender), ref["sender"])
+    assert np.array_equal(_np(g.shift), ref["shift"])
+    assert np.array_equal(_np(g.edge_vec).view(np.uint32), ref["edge_vec"].view(np.uint32))
+    assert np.array_equal(_np(g.t_row_ptr), ref["t_row_ptr"])
+    assert np.array_equal(_np(g.t_perm), ref["t_perm"])
+
+
+@pytest.mark.parametrize("name", ["diamond8k", "melt32k"])
+def test_neighbors_bit_exact_sampled(wls, name):
+    wl = wls(name)
+    g = _gpu_graph(wl)
+    rng = np.random.default_rng(7)
+    sample = np.sort(rng.choice(wl.n_nodes, size=N_SAMPLE, replace=False))
+    rows = sampled_rows(wl, sample)
+    rp = _np(g.row_ptr)
+    snd, shf, vec = _np(g.sender), _np(g.shift), _np(g.edge_vec)
+    for i in sample:
+        m = rows["receiver"] == i
+        a, b = rp[i], rp[i + 1]
+        assert b - a == m.sum()
+        assert np.array_equal(snd[a:b], rows["sender"][m])
+        assert np.array_equal(shf[a:b], rows["shift"][m])
+        assert np.array_equal(vec[a:b].view(np.uint32), rows["edge_vec"][m].view(np.uint32))
+    # transposed order: edges sent by j = mirror of row j (symmetric test), so counts agree
+    trp = _np(g.t_row_ptr)
+    for i in sample:
+        assert trp[i + 1] - trp[i] == rp[i + 1] - rp[i]
+    # t_perm: the stable sort of the canonical edge ids by sender
+    tp = _np(g.t_perm)
+    s_sorted = snd[tp]
+    assert np.all(np.diff(s_sorted) >= 0)
+    same = np.diff(s_sorted) == 0
+    assert np.all(np.diff(tp)[same] > 0)
+    assert np.array_equal(np.sort(tp), np.arange(g.n_edges))
+
+
+@pytest.mark.parametrize("name", ["sweep1", "sweep2", "sweep3"])
+def test_build_csr_bit_exact(wls, name):
+    wl = wls(name)
+    ref = given_graph(wl)
+    g = _gpu_graph(wl)
+    assert np.array_equal(_np(g.perm), ref["perm"])
+    assert np.array_equal(_np(g.row_ptr), ref["row_ptr"])
+    assert np.array_equal(_np(g.sender), ref["sender"])
+    assert np.array_equal(_np(g.edge_vec).view(np.uint32), ref["edge_vec"].view(np.uint32))
+    assert np.array_equal(_np(g.t_row_ptr), ref["t_row_ptr"])
+    assert np.array_equal(_np(g.t_perm), ref["t_perm"])
+
+
+# ------------------------------------------------------------------ forward
+
+def _inputs(wl, conv):
+    x = wl.features()
+    W = wl.weights(conv.n_paths)
+    return x, W
+
+
+@pytest.mark.parametrize("name", ["tiny", "diamond1k"])
+def test_forward_parity_full(wls, name):
+    wl = wls(name)
+    conv = _conv(wl)
+    spec = spec_of(wl)
+    x, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    out = conv.forward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV))
+    ref = forward_ref(wl, spec, x, W, graph=full_graph(wl))
+    assert_blocks_close(_np(out), ref, wl.channels, wl.lmax, f"{name} forward")
+
+
+@pytest.mark.parametrize("name", ["sweep1", "sweep2", "sweep3", "diamond8k", "melt32k"])
+def test_forward_parity_sampled(wls, name):
+    wl = wls(name)
+    conv = _conv(wl)
+    spec = spec_of(wl)
+    x, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    out = _np(conv.forward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)))
+    rng = np.random.default_rng(11)
+    sample = np.sort(rng.choice(wl.n_nodes, size=N_SAMPLE, replace=False))
+    if wl.given_receiver is not None:
+        ref_g = given_graph(wl)
+        ref = conv_forward(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, receivers=sample)
+    else:
+        ref, _ = forward_ref(wl, spec, x, W, sample=sample)
+    assert_blocks_close(out[sample], ref, wl.channels, wl.lmax, f"{name} forward (sampled)")
+
+
+def test_forward_bitwise_deterministic(wls):
+    wl = wls("diamond1k")
+    conv = _conv(wl)
+    x, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    xt, Wt = torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)
+    a = conv.forward(g, xt, Wt).clone()
+    b = conv.forward(g, xt, Wt)
+    assert torch.equal(a, b)
+
+
+def test_radial_weights_parity(wls):
+    wl = wls("diamond1k")
+    conv = _conv(wl)
+    _, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    w = _np(conv.radial_weights(g.edge_vec, torch.from_numpy(W).to(DEV)))
+    ref_g = full_graph(wl)
+    vec = ref_g["edge_vec"].astype(np.float64)
+    rad = radial(np.linalg.norm(vec, axis=1), 8, np.float64(np.float32(wl.r_cut)))
+    ref = np.einsum("eb,bpc->epc", rad, W.astype(np.float64))
+    assert_close_rel(w, ref, "radial weights")
+
+
+# ------------------------------------------------------------------ backward
+
+@pytest.mark.parametrize("name", ["tiny", "diamond1k"])
+def test_backward_parity_full(wls, name):
+    wl = wls(name)
+    conv = _conv(wl)
+    spec = spec_of(wl)
+    x, W = _inputs(wl, conv)
+    gout = wl.cotangent()
+    g = _gpu_graph(wl)
+    gx, gv = conv.backward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV),
+                           torch.from_numpy(gout).to(DEV))
+    ref_g = full_graph(wl)
+    rgx, rgv = conv_vjp(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, gout)
+    assert_blocks_close(_np(gx), rgx, wl.channels, wl.lmax, f"{name} grad_x")
+    assert_close_rel(_np(gv), rgv, f"{name} grad_edge_vec")
+    # forces from the edge gradients
+    f = _np(etp.forces(g, gv))
+    rf = forces_from_edge_grads(rgv, ref_g["receiver"], ref_g["sender"], wl.n_nodes)
+    assert_close_rel(f, rf, f"{name} forces")
+    # only one of the two outputs
+    gx2, none = conv.backward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV),
+                              torch.from_numpy(gout).to(DEV), want_grad_vec=False)
+    assert none is None and torch.equal(gx2, gx)
+    none, gv2 = conv.backward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV),
+                              torch.from_numpy(gout).to(DEV), want_grad_x=False)
+    assert none is None and torch.equal(gv2, gv)
+
+
+@pytest.mark.parametrize("name", ["diamond8k", "melt32k"])
+def test_backward_parity_sampled(wls, name):
+    wl = wls(name)
+    conv = _conv(wl)
+    spec = spec_of(wl)
+    x, W = _inputs(wl, conv)
+    gout = wl.cotangent()
+    g = _gpu_graph(wl)
+    gx, gv = conv.backward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV),
+                           torch.from_numpy(gout).to(DEV))
+    gx, gv = _np(gx), _np(gv)
+    rng = np.random.default_rng(13)
+    sample = np.sort(rng.choice(wl.n_nodes, size=N_SAMPLE // 2, replace=False))
+    rows = sampled_rows(wl, sample)
+    recv, send, shift, vec = sender_edges(rows)
+    rp, snd, v = rows_subgraph(wl.n_nodes, recv, send, vec)
+    rgx, rgv = conv_vjp(spec, rp, snd, v, x, W, gout)
+    assert_blocks_close(gx[sample], rgx[sample], wl.channels, wl.lmax, f"{name} grad_x (sampled)")
+    keys = _edge_keys(_gpu_receivers(g), _np(g.sender), _np(g.shift), wl.n_nodes)
+    want = _edge_keys(recv, send, shift, wl.n_nodes)
+    pos = np.searchsorted(keys, want)
+    assert np.array_equal(keys[pos], want)
+    assert_close_rel(gv[pos], rgv, f"{name} grad_edge_vec (sampled)")
+
+
+def test_autograd_function_matches_backward(wls):
+    wl = wls("tiny")
+    conv = _conv(wl)
+    x, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    fn = etp.edge_conv_function()
+    xt = torch.from_numpy(x).to(DEV).requires_grad_(True)
+    vt = g.edge_vec.clone().requires_grad_(True)
+    Wt = torch.from_numpy(W).to(DEV)
+    out = fn.apply(conv, g, xt, vt, Wt)
+    gout = torch.from_numpy(wl.cotangent()).to(DEV)
+    (out * gout).sum().backward()
+    gx, gv = conv.backward(g, xt.detach(), Wt, gout)
+    assert torch.equal(xt.grad, gx) and torch.equal(vt.grad, gv)
+
+
+# ------------------------------------------------------------------ edge cases
+
+def test_empty_graph_and_isolated_nodes():
+    conv = etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x1o", 8, 4.0)
+    pos = torch.tensor([[0.0, 0.0, 0.0], [10.0, 0.0, 0.0], [20.0, 0.0, 0.0]], device=DEV)
+    g = etp.neighbors(pos, 4.0)
+    assert g.n_edges == 0
+    x = torch.randn(3, 32, device=DEV)
+    W = torch.randn(8, conv.n_paths, 8, device=DEV)
+    out = conv.forward(g, x, W, out=torch.full((3, 32), 7.0, device=DEV))
+    assert torch.count_nonzero(out) == 0
+    gx, gv = conv.backward(g, x, W, torch.randn(3, 32, device=DEV),
+                           grad_x=torch.full((3, 32), 7.0, device=DEV))
+    assert torch.count_nonzero(gx) == 0 and gv.numel() == 0
+    f = etp.forces(g, gv)
+    assert torch.count_nonzero(f) == 0
+    # one node, no edges
+    g1 = etp.neighbors(pos[:1], 4.0)
+    assert g1.n_edges == 0 and torch.count_nonzero(conv.forward(g1, x[:1], W)) == 0
+
+
+def test_edges_beyond_cutoff_contribute_zero():
+    conv = etp.EdgeConv("4x0e+4x1o", 1, "4x0e+4x1o", 8, 3.0)
+    recv = torch.tensor([0, 0, 1], device=DEV)
+    send = torch.tensor([1, 1, 0], device=DEV)
+    vec = torch.tensor([[3.0, 0.0, 0.0], [0.0, 4.0, 0.0], [0.0, 0.0, -3.5]], device=DEV)
+    g = etp.build_csr(2, recv, send, vec)
+    out = conv.forward(g, torch.randn(2, 16, device=DEV), torch.randn(8, conv.n_paths, 4, device=DEV))
+    assert torch.count_nonzero(out) == 0
+
+
+def test_validation_rejects_corrupt_graph(wls, monkeypatch):
+    wl = wls("tiny")
+    conv = _conv(wl)
+    x, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    bad_ptr = g.row_ptr.clone()
+    bad_ptr[5] = bad_ptr[6] + 3          # not monotone
+    bad = etp.Graph(g.n_nodes, g.n_edges, bad_ptr, g.sender, g.edge_vec, g.t_row_ptr, g.t_perm)
+    monkeypatch.setenv("ETP_VALIDATE", "1")
+    out = torch.full((wl.n_nodes, wl.dim), 3.0, device=DEV)
+    with pytest.raises(etp.EtpError) as ei:
+        conv.forward(bad, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV), out=out)
+    assert ei.value.status == 4
+    assert bool((out == 3.0).all())
+    bad_sender = g.sender.clone()
+    bad_sender[0] = wl.n_nodes + 5
+    bad2 = etp.Graph(g.n_nodes, g.n_edges, g.row_ptr, bad_sender, g.edge_vec, g.t_row_ptr, g.t_perm)
+    with pytest.raises(etp.EtpError):
+        conv.backward(bad2, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV),
+                      torch.from_numpy(wl.cotangent()).to(DEV))
+    bad_tp = g.t_perm.clone()
+    bad_tp[0] = bad_tp[1]
+    bad3 = etp.Graph(g.n_nodes, g.n_edges, g.row_ptr, g.sender, g.edge_vec, g.t_row_ptr, bad_tp)
+    with pytest.raises(etp.EtpError):
+        conv.backward(bad3, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV),
+                      torch.from_numpy(wl.cotangent()).to(DEV))
+    monkeypatch.delenv("ETP_VALIDATE")
+    conv.forward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV), out=out)
+    torch.cuda.synchronize()
+
+
+def test_build_csr_rejects_out_of_range():
+    recv = torch.tensor([0, 3], device=DEV)
+    send = torch.tensor([1, 0], device=DEV)
+    vec = torch.zeros(2, 3, device=DEV)
+    with pytest.raises(etp.EtpError) as ei:
+        etp.build_csr(2, recv, send, vec)
+    assert ei.value.status == 4
+
+
+def test_no_cpu_fallback():
+    conv = etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x1o", 8, 4.0)
+    with pytest.raises(ValueError):
+        conv.radial_weights(torch.zeros(3, 3), torch.zeros(8, conv.n_paths, 8))
+    assert os.path.exists(etp.LIB_PATH)
