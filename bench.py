@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the fused equivariant edge tensor-product convolution on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input: neighbour list and
+canonical CSR from the atom positions, fused forward convolution, fused backward (VJP to node
+features and edge vectors) and force assembly. Workload: the 1000-atom periodic diamond cell
+(5x5x5 conventional cells, a = 3.567 A, jitter N(0, 0.05 A), r_cut 5 A, 64x0e+64x1o+64x2e,
+SH lmax 2, 8 Bessel functions), synthetic seeded inputs, fp32 throughout.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {etp,reference}] [--workload NAME]
+
+Multi-GPU (torchrun, one rank per GPU): independent replicas (the path does not shard on one
+GPU's workload; weak scaling), no data-path collective; the timed region is the max over ranks.
+The reference arm (--impl reference) times the float64 CPU oracle on a bounded sample of the
+same workload (rank 0 only).
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "edges/sec for TP conv fwd and fwd+bwd (fp32), % of HBM/FP32 roofline"
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------- peaks and counts
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS, "sm_max_mhz": 1965.0}, "fallback"
+
+
+def fp32_peak_tflops(sm_mhz):
+    """Plain FP32 ALU peak: 148 SMs x 128 FP32 lanes x 2 flop (FMA) x SM clock."""
+    return SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+
+
+def algorithmic_counts(info, n_nodes, n_edges):
+    """Per-launch algorithmic flops / bytes of the plain definition (see the design notes).
+
+    forward  FP32: 2 (nnz + sum_p(2 l3 + 1)) C per edge   (CG contraction with c = C Y, then w s)
+    backward FP32: 2 (3 nnz + 2 sum_p(2 l3 + 1)) C per edge (grad_x, grad_w, grad_Y contractions)
+    radial projection (tensor-core class work, not counted as FP32): 2 n_basis P C per edge
+    (forward), twice that in the backward.
+    Compulsory HBM bytes: node rows read/written once, edge arrays once.
+    """
+    c, nnz, s3 = info["channels"], info["cg_nnz"], info["sum_2l3p1"]
+    dim = info["dim_in"]
+    fwd_flop = 2.0 * (nnz + s3) * c * n_edges
+    bwd_flop = 2.0 * (3 * nnz + 2 * s3) * c * n_edges
+    radial = 2.0 * info["n_basis"] * info["n_paths"] * c * n_edges
+    fwd_bytes = 4.0 * (2 * n_nodes * dim + 4 * n_edges + n_nodes + 1)
+    bwd_bytes = 4.0 * (3 * n_nodes * dim + 4 * n_edges + 3 * n_edges + 2 * (n_nodes + 1) + n_edges)
+    return dict(fwd_flop=fwd_flop, bwd_flop=bwd_flop, fwd_radial_flop=radial, bwd_radial_flop=2 * radial,
+                fwd_bytes=fwd_bytes, bwd_bytes=bwd_bytes)
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, ValueError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import equivariant_mlip_tensor_edge_b200 as etp
+    import workloads
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = workloads.make(args.workload)
+    conv = etp.EdgeConv(wl.irreps, wl.lmax, wl.irreps, wl.n_basis, float(wl.r_cut))
+    info = conv.info
+    pos_h = torch.from_numpy(wl.pos).pin_memory()
+    x_h = torch.from_numpy(wl.features()).pin_memory()
+    W_h = torch.from_numpy(wl.weights(conv.n_paths)).pin_memory()
+    g_h = torch.from_numpy(wl.cotangent()).pin_memory()
+    pos, x, W, gout = (t.to(dev) for t in (pos_h, x_h, W_h, g_h))
+    n = wl.n_nodes
+
+    g0 = etp.neighbors(pos, float(wl.r_cut), cell=wl.cell, pbc=wl.pbc)
+    cap = int(g0.n_edges * 1.25) + 1024
+    # persistent buffers (capacity cap) so a step allocates nothing
+    bufs = dict(
+        row_ptr=torch.empty(n + 1, dtype=torch.int32, device=dev),
+        t_row_ptr=torch.empty(n + 1, dtype=torch.int32, device=dev),
+        sender=torch.empty(cap, dtype=torch.int32, device=dev),
+        edge_vec=torch.empty((cap, 3), dtype=torch.float32, device=dev),
+        t_perm=torch.empty(cap, dtype=torch.int32, device=dev),
+        gws=torch.empty(etp.graph_workspace_bytes(n, cap), dtype=torch.uint8, device=dev),
+        ws=torch.empty(conv.workspace_bytes(n, cap), dtype=torch.uint8, device=dev),
+        out=torch.empty((n, info["dim_out"]), dtype=torch.float32, device=dev),
+        gx=torch.empty((n, info["dim_in"]), dtype=torch.float32, device=dev),
+        gv=torch.empty((cap, 3), dtype=torch.float32, device=dev),
+        f=torch.empty((n, 3), dtype=torch.float32, device=dev),
+    )
+    lib = etp.load_library()
+    import ctypes
+    cell_arr = (ctypes.c_double * 9)(*[float(v) for row in wl.cell for v in row]) if wl.cell is not None else None
+    pbc_arr = (ctypes.c_int * 3)(*[int(bool(p)) for p in wl.pbc])
+    P = etp._ptr
+    stream = etp._stream(dev)
+    n_edges_c = ctypes.c_int(0)
+
+    def graph_step(pos_d):
+        st = lib.etp_neighbors(P(pos_d), n, ctypes.cast(cell_arr, etp._dp) if cell_arr is not None else None,
+                               pbc_arr, float(wl.r_cut), cap, ctypes.byref(n_edges_c), P(bufs["row_ptr"]),
+                               P(bufs["sender"]), P(bufs["edge_vec"]), None, P(bufs["t_row_ptr"]), P(bufs["t_perm"]),
+                               P(bufs["gws"]), bufs["gws"].numel(), stream)
+        etp._check(st, "etp_neighbors")
+        e = n_edges_c.value
+        return etp.Graph(n, e, bufs["row_ptr"], bufs["sender"][:e], bufs["edge_vec"][:e], bufs["t_row_ptr"],
+                         bufs["t_perm"][:e])
+
+    def conv_fwd(gr, xx, WW):
+        return conv.forward(gr, xx, WW, out=bufs["out"], workspace=bufs["ws"])
+
+    def conv_bwd(gr, xx, WW, gg):
+        return conv.backward(gr, xx, WW, gg, grad_x=bufs["gx"], grad_vec=bufs["gv"][:gr.n_edges],
+                             workspace=bufs["ws"])
+
+    def step(pos_d, xx, WW, gg):
+        gr = graph_step(pos_d)
+        conv_fwd(gr, xx, WW)
+        conv_bwd(gr, xx, WW, gg)
+        etp.forces(gr, bufs["gv"][:gr.n_edges], out=bufs["f"])
+        return gr
+
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # > 126 MB L2
+
+    def timed(fn, k):
+        total = 0.0
+        for _ in range(k):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            total += a.elapsed_time(b)
+        return total / k
+
+    # warm-up
+    for _ in range(args.warmup):
+        step(pos, x, W, gout)
+    torch.cuda.synchronize()
+    gr = graph_step(pos)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local_rank if os.environ.get("CUDA_VISIBLE_DEVICES") is None else 0)
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms_step = timed(lambda: step(pos, x, W, gout), args.steps)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    # per-kernel timings on the same stream (dominant kernels), same flush discipline
+    reps = max(args.steps, 5)
+    ms_fwd = timed(lambda: conv_fwd(gr, x, W), reps)
+    ms_bwd = timed(lambda: conv_bwd(gr, x, W, gout), reps)
+    ms_graph = timed(lambda: graph_step(pos), reps)
+    clocks = sampler.stop() if rank == 0 else None
+
+    # end to end through the public API with host buffers (copies inside the timed region)
+    out_h = torch.empty_like(bufs["out"], device="cpu").pin_memory()
+    f_h = torch.empty((n, 3), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        pd, xd, Wd, gd = (t.to(dev, non_blocking=True) for t in (pos_h, x_h, W_h, g_h))
+        step(pd, xd, Wd, gd)
+        out_h.copy_(bufs["out"], non_blocking=True)
+        f_h.copy_(bufs["f"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    ms_e2e = timed(e2e_step, args.steps)
+    h2d = sum(t.numel() * t.element_size() for t in (pos_h, x_h, W_h, g_h))
+    d2h = out_h.numel() * 4 + f_h.numel() * 4
+
+    e = gr.n_edges
+    t_local = torch.tensor([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph], dtype=torch.float64, device=dev)
+    edges_local = torch.tensor([float(e)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
+        dist.all_reduce(edges_local, op=dist.ReduceOp.SUM)
+    ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph = t_local.tolist()
+    total_edges = edges_local.item()
+    if rank != 0:
+        return None
+
+    peaks, peak_kind = measured_peaks()
+    sm_max = peaks.get("sm_max_mhz", 1965.0)
+    fp32_peak = fp32_peak_tflops(sm_max)
+    cnt = algorithmic_counts(info, n, e)
+    dominant = "bwd" if ms_bwd >= ms_fwd else "fwd"
+
+    def roof(kind, ms):
+        flop = cnt[f"{kind}_flop"]
+        ach = flop / (ms * 1e-3) / 1e12
+        return {"bound": "alu", "achieved": round(ach, 3), "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
+                "frac": round(ach / fp32_peak, 4), "traffic": None,
+                "kernel": "k_conv_bwd" if kind == "bwd" else "k_conv_fwd",
+                "peak_source": f"derived: 148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz ({peak_kind} sm_max_mhz)",
+                "ms_per_launch": round(ms, 5),
+                "hbm_frac_of_" + peak_kind: round(cnt[f"{kind}_bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+
+    line = {
+        "metric": METRIC,
+        "value": round(total_edges / (ms_step * 1e-3), 1),
+        "unit": "edges/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded workload generator)",
+        "config": {"workload": f"{wl.name}: {n} atoms, {e} edges, {wl.irreps}, SH lmax {wl.lmax}, "
+                               f"r_cut {float(wl.r_cut)}, 8 Bessel",
+                   "step": "neighbour list + CSR + fused forward + fused backward + forces",
+                   "parallelism": f"replicas x{world}", "l2": "flushed (256 MB write) before every timed step"},
+        "fwd_edges_per_s": round(total_edges / (ms_fwd * 1e-3), 1),
+        "conv_fwd_bwd_edges_per_s": round(total_edges / ((ms_fwd + ms_bwd) * 1e-3), 1),
+        "ms_fwd": round(ms_fwd, 5), "ms_bwd": round(ms_bwd, 5), "ms_graph": round(ms_graph, 5),
+        "roofline": roof(dominant, ms_bwd if dominant == "bwd" else ms_fwd),
+        "roofline_fwd": roof("fwd", ms_fwd),
+        "e2e": {"value": round(total_edges / (ms_e2e * 1e-3), 1), "unit": "edges/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 8 * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
+    return line
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+
+def _oracle_sample_step(wl, sample):
+    import numpy as np
+
+    from oracle.conv import ConvSpec, conv_forward, conv_vjp
+    from oracle.graph import forces_from_edge_grads, neighbors
+
+    spec = ConvSpec(wl.irreps, wl.lmax, wl.irreps, wl.n_basis, float(wl.r_cut))
+    x, W, g = wl.features(), wl.weights(len(spec.paths)), wl.cotangent()
+    rows = neighbors(wl.pos, wl.cell, wl.pbc, wl.r_cut, receivers=sample)
+    row_ptr = np.zeros(wl.n_nodes + 1, dtype=np.int64)
+    np.add.at(row_ptr, rows["receiver"] + 1, 1)
+    row_ptr = np.cumsum(row_ptr)
+    conv_forward(spec, row_ptr, rows["sender"], rows["edge_vec"], x, W, receivers=sample)
+    _, gv = conv_vjp(spec, row_ptr, rows["sender"], rows["edge_vec"], x, W, g)
+    forces_from_edge_grads(gv, rows["receiver"], rows["sender"], wl.n_nodes)
+    return len(rows["sender"])
+
+
+def cpu_baseline(wl, budget_s=15.0, steps=1):
+    """The float64 oracle, as it stands, on a bounded sample of receivers; one BLAS thread."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    frac = 0.25
+    n_s = max(1, int(wl.n_nodes * frac))
+    sample = sorted(np.random.default_rng(0).choice(wl.n_nodes, size=n_s, replace=False).tolist())
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        edges = 0
+        for _ in range(steps):
+            edges += _oracle_sample_step(wl, sample)
+        dt = time.perf_counter() - t0
+    return {"value": round(edges / dt, 1), "unit": "edges/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_s} of {wl.n_nodes} receivers ({edges // steps} edges): neighbour rows, forward, VJP, "
+                      f"forces in float64 numpy, {steps} step(s), {dt:.1f} s",
+            "seconds": round(dt, 3)}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import workloads
+    wl = workloads.make(args.workload)
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm-up state; kept for the CLI contract
+    cb = cpu_baseline(wl, budget_s=args.cpu_budget, steps=max(1, args.steps))
+    ms = 1000.0 * cb["seconds"] / max(1, args.steps)
+    return {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "edges/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded workload generator)",
+            "config": {"workload": wl.name, "step": "neighbour rows + forward + VJP + forces (float64 oracle)",
+                       "parallelism": "host cores, rank 0 only"},
+            "cpu_baseline": cb,
+            "e2e": {"value": cb["value"], "unit": "edges/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="etp", choices=["etp", "reference"])
+    ap.add_argument("--workload", default="diamond1k")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_gpu(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

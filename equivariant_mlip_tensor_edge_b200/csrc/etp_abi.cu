@@ -206,13 +206,23 @@ etp_status etp_get_info(etp_handle h, etp_info_t* info) {
   return ETP_OK;
 }
 
-// Workspace: [recv_map: n_edges ints][validation scratch: n_edges + 1 ints]
+// Workspace: [recv_map: n_edges ints][validation scratch: n_edges + 1 ints][tensor-core forward:
+// pre-split weights + status word]
+static size_t ws_scratch_offset(int n_edges) { return align256(sizeof(int) * static_cast<size_t>(n_edges)); }
+static size_t ws_tc_offset(int n_edges) {
+  return ws_scratch_offset(n_edges) + align256(sizeof(int) * (static_cast<size_t>(n_edges) + 1));
+}
+
 size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
-  (void)h;
   (void)n_nodes;
-  if (n_edges < 0) return 0;
-  return align256(sizeof(int) * static_cast<size_t>(n_edges)) +
-         align256(sizeof(int) * (static_cast<size_t>(n_edges) + 1));
+  if (!h || n_edges < 0) return 0;
+  return ws_tc_offset(n_edges) + tc::forward_tc_workspace_bytes(h->c);
+}
+
+// The tensor-core forward is the default; ETP_FORWARD=generic selects the all-FP32 kernel.
+static bool use_tc_forward() {
+  const char* v = std::getenv("ETP_FORWARD");
+  return !(v && std::strcmp(v, "generic") == 0);
 }
 
 static etp_status check_common(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
@@ -261,12 +271,21 @@ etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_pt
       set_error("etp_forward: ETP_VALIDATE=1 needs the workspace");
       return ETP_ERR_INVALID_ARG;
     }
-    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) +
-                                          align256(sizeof(int) * static_cast<size_t>(n_edges)));
+    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_scratch_offset(n_edges));
     st = validate_graph(n_nodes, n_edges, row_ptr, sender, nullptr, nullptr, scratch, s);
     if (st != ETP_OK) return st;
   }
   if (n_nodes == 0) return ETP_OK;
+  if (use_tc_forward()) {
+    if (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges)) {
+      set_error("etp_forward: workspace missing or smaller than etp_workspace_bytes()");
+      return ETP_ERR_INVALID_ARG;
+    }
+    void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
+    st = tc::launch_forward_tc(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);
+    if (st == ETP_OK && validate_requested()) st = tc::forward_tc_status(h->c, tcws, s);
+    return st;
+  }
   return launch_forward(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, s);
 }
 
@@ -292,8 +311,7 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   int* recv_map = static_cast<int*>(workspace);
   if (validate_requested()) {
-    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) +
-                                          align256(sizeof(int) * static_cast<size_t>(n_edges)));
+    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_scratch_offset(n_edges));
     st = validate_graph(n_nodes, n_edges, row_ptr, sender, t_row_ptr, t_perm, scratch, s);
     if (st != ETP_OK) return st;
   }

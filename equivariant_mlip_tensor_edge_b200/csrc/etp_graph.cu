@@ -15,6 +15,12 @@ struct CellParams {
   double c[9];       // rows = lattice vectors
   int n[3];          // images scanned per axis: S_a in [-n_a, n_a]
   double rc2;        // float64(r_cut)^2 (exact: a float squared fits in a double)
+  // Orthorhombic cell whose periodic lengths all exceed 2 r_cut: two images of a pair differ by
+  // more than 2 r_cut along some axis, so at most one image can be within r_cut and it is the
+  // nearest one. Testing only that image (clamped to the scanned range) keeps exactly the set of
+  // edges the full scan keeps, with the same arithmetic for the kept edge.
+  int min_image;
+  double len[3];
 };
 
 // r = (pos[j] - pos[i]) + ((S0 c0 + S1 c1) + S2 c2); d2 = (rx rx + ry ry) + rz rz, no FMA.
@@ -38,10 +44,24 @@ __device__ __forceinline__ float3 load_pos(const float* pos, int i) {
   return make_float3(pos[3 * i], pos[3 * i + 1], pos[3 * i + 2]);
 }
 
+__device__ __forceinline__ int nearest_image(float pi, float pj, double len, int n) {
+  if (n == 0) return 0;
+  const double d = static_cast<double>(pj) - static_cast<double>(pi);
+  int k = -static_cast<int>(rint(d / len));
+  return k < -n ? -n : (k > n ? n : k);
+}
+
 // Number of kept images for receiver i and sender j (S in lexicographic order).
 __device__ __forceinline__ int count_pair(float3 pi, float3 pj, bool same, const CellParams& cp) {
   int c = 0;
   double rx, ry, rz;
+  if (cp.min_image) {
+    const int s0 = nearest_image(pi.x, pj.x, cp.len[0], cp.n[0]);
+    const int s1 = nearest_image(pi.y, pj.y, cp.len[1], cp.n[1]);
+    const int s2 = nearest_image(pi.z, pj.z, cp.len[2], cp.n[2]);
+    if (same && s0 == 0 && s1 == 0 && s2 == 0) return 0;
+    return pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz) ? 1 : 0;
+  }
   for (int s0 = -cp.n[0]; s0 <= cp.n[0]; ++s0)
     for (int s1 = -cp.n[1]; s1 <= cp.n[1]; ++s1)
       for (int s2 = -cp.n[2]; s2 <= cp.n[2]; ++s2) {
@@ -87,7 +107,23 @@ __global__ void k_nbr_emit(const float* __restrict__ pos, int n, CellParams cp,
       if (lane >= o) incl += t;
     }
     const int total = __shfl_sync(0xffffffffu, incl, 31);
-    if (c > 0) {
+    if (c > 0 && cp.min_image) {
+      const int s0 = nearest_image(pi.x, pj.x, cp.len[0], cp.n[0]);
+      const int s1 = nearest_image(pi.y, pj.y, cp.len[1], cp.n[1]);
+      const int s2 = nearest_image(pi.z, pj.z, cp.len[2], cp.n[2]);
+      double rx, ry, rz;
+      pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz);
+      const int at = base + incl - c;
+      sender[at] = j;
+      edge_vec[3 * at + 0] = static_cast<float>(rx);
+      edge_vec[3 * at + 1] = static_cast<float>(ry);
+      edge_vec[3 * at + 2] = static_cast<float>(rz);
+      if (shift) {
+        shift[3 * at + 0] = s0;
+        shift[3 * at + 1] = s1;
+        shift[3 * at + 2] = s2;
+      }
+    } else if (c > 0) {
       int at = base + incl - c;
       double rx, ry, rz;
       for (int s0 = -cp.n[0]; s0 <= cp.n[0]; ++s0)
@@ -253,7 +289,15 @@ etp_status neighbors(const float* pos, int n_nodes, const double* cell, const in
       }
       cp.n[a] = static_cast<int>(std::ceil(rc / spacing));
     }
+    const bool ortho = c[1] == 0.0 && c[2] == 0.0 && c[3] == 0.0 && c[5] == 0.0 && c[6] == 0.0 && c[7] == 0.0;
+    cp.min_image = ortho ? 1 : 0;
+    for (int a = 0; a < 3; ++a) {
+      cp.len[a] = c[4 * a];   // signed: the image shift along axis a is S_a * c[a][a]
+      if (cp.n[a] > 0 && !(std::fabs(cp.len[a]) > 2.0 * rc)) cp.min_image = 0;
+    }
   } else {
+    cp.min_image = 0;
+    cp.len[0] = cp.len[1] = cp.len[2] = 0.0;
     if (pbc && (pbc[0] || pbc[1] || pbc[2])) {
       set_error("etp_neighbors: periodic axes need a cell");
       return ETP_ERR_INVALID_ARG;

@@ -46,6 +46,15 @@ etp_status launch_forces(int n_nodes, int n_edges, const int* row_ptr, const int
 etp_status validate_graph(int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                           const int* t_row_ptr, const int* t_perm, int* scratch, cudaStream_t s);
 
+// ---- forward with the radial projection on tcgen05 tensor cores (etp_fwd_tc.cu)
+namespace tc {
+size_t forward_tc_workspace_bytes(const Ctx& c);
+etp_status forward_tc_status(const Ctx& c, const void* ws, cudaStream_t s);
+etp_status launch_forward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
+                             const float* edge_vec, const float* x, const float* W, float* out, void* ws,
+                             cudaStream_t s);
+}  // namespace tc
+
 // ---- graph kernels (etp_graph.cu)
 size_t graph_workspace_bytes(int n_nodes, int max_edges);
 etp_status neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,

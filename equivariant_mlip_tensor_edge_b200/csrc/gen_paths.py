@@ -173,7 +173,7 @@ def emit_paths(out, lmax):
     out.append(f"    const float (&x)[{D}][K], float (&acc)[{D}][K]) {{")
     for p, ((l1, l2, l3), c) in enumerate(zip(paths, cgs)):
         out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
-        out.append("    float wp[K]; wfetch(" + str(p) + ", wp);")
+        out.append(f"    float wp[K]; wfetch(IC<{p}>{{}}, wp);")
         # M[m3][m1] = sum_m2 C[m1,m2,m3] Y[l2,m2]
         mnz = []
         for m3 in range(2 * l3 + 1):
@@ -221,7 +221,7 @@ def emit_paths(out, lmax):
     out.append(f"    float* gY, float& accd) {{")
     for p, ((l1, l2, l3), c) in enumerate(zip(paths, cgs)):
         out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
-        out.append("    float wp[K], wdp[K]; wfetch(" + str(p) + ", wp, wdp);")
+        out.append(f"    float wp[K], wdp[K]; wfetch(IC<{p}>{{}}, wp, wdp);")
         mnz = []
         for m3 in range(2 * l3 + 1):
             for m1 in range(2 * l1 + 1):
@@ -274,6 +274,11 @@ def generate():
            "// Real-basis Clebsch-Gordan contractions and real spherical harmonics, unrolled per path.",
            "#pragma once",
            "namespace etp_gen {",
+           "// compile-time path index handed to the weight-fetch callback",
+           "template <int N> struct IC {",
+           "  static constexpr int value = N;",
+           "  __host__ __device__ constexpr operator int() const { return N; }",
+           "};",
            "template <int L> struct PathSet;"]
     for lmax in LMAX_SUPPORTED:
         emit_sh(out, lmax)

@@ -328,3 +328,53 @@ def test_no_cpu_fallback():
     with pytest.raises(ValueError):
         conv.radial_weights(torch.zeros(3, 3), torch.zeros(8, conv.n_paths, 8))
     assert os.path.exists(etp.LIB_PATH)
+
+
+# ------------------------------------------------------------------ forward kernels: both implementations
+
+@pytest.mark.parametrize("impl", ["tc", "generic"])
+@pytest.mark.parametrize("name", ["tiny", "diamond1k"])
+def test_forward_both_kernels(wls, name, impl, monkeypatch):
+    if impl == "generic":
+        monkeypatch.setenv("ETP_FORWARD", "generic")
+    monkeypatch.setenv("ETP_VALIDATE", "1")      # graph checks + device pipeline status word
+    wl = wls(name)
+    conv = _conv(wl)
+    x, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    out = conv.forward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV))
+    ref = forward_ref(wl, spec_of(wl), x, W, graph=full_graph(wl))
+    assert_blocks_close(_np(out), ref, wl.channels, wl.lmax, f"{name} forward ({impl})")
+
+
+def _random_graph(n_nodes, degrees, seed, r_max=4.5):
+    rng = np.random.default_rng(seed)
+    recv = np.repeat(np.arange(n_nodes), degrees)
+    send = rng.integers(0, n_nodes, size=len(recv))
+    d = rng.standard_normal((len(recv), 3))
+    d /= np.linalg.norm(d, axis=1, keepdims=True)
+    vec = (d * rng.uniform(0.5, r_max, size=(len(recv), 1))).astype(np.float32)
+    return recv, send, vec
+
+
+@pytest.mark.parametrize("lmax,c", [(1, 20), (2, 24), (3, 8)])
+def test_forward_ragged_degrees_and_channels(lmax, c):
+    """Degrees 0..300 (several 128-edge rounds, empty rows, ragged tiles) and C not a multiple of 16."""
+    from oracle.conv import ConvSpec
+    irr = "+".join(f"{c}x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
+    n = 13
+    degrees = np.array([0, 1, 31, 32, 33, 127, 128, 129, 300, 5, 0, 64, 97])
+    recv, send, vec = _random_graph(n, degrees, seed=lmax)
+    conv = etp.EdgeConv(irr, lmax, irr, 8, 5.0)
+    spec = ConvSpec(irr, lmax, irr, 8, 5.0)
+    rng = np.random.default_rng(100 + lmax)
+    x = rng.standard_normal((n, spec.dim_in)).astype(np.float32)
+    W = (rng.standard_normal((8, len(spec.paths), c)) / np.sqrt(8)).astype(np.float32)
+    g = etp.build_csr(n, torch.from_numpy(recv).to(DEV), torch.from_numpy(send).to(DEV),
+                      torch.from_numpy(vec).to(DEV))
+    out = _np(conv.forward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)))
+    order = np.lexsort((send, recv))
+    rp = np.concatenate([[0], np.cumsum(degrees)])
+    ref = conv_forward(spec, rp, send[order], vec[order], x, W)
+    assert np.all(out[degrees == 0] == 0.0)
+    assert_blocks_close(out, ref, c, lmax, f"ragged forward lmax={lmax} C={c}")
