@@ -17,7 +17,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libetp.so")
 SOURCES = ["etp_abi.cu", "etp_graph.cu", "etp_conv.cu", "etp_fwd_tc.cu"]
 HEADERS = [os.path.join(ROOT, "include", "etp.h"), os.path.join(CSRC, "etp_internal.h"),
-           os.path.join(CSRC, "generated", "etp_paths.h"), os.path.join(CSRC, "etp_device.h")]
+           os.path.join(CSRC, "generated", "etp_paths.h"), os.path.join(CSRC, "etp_device.h"), os.path.join(CSRC, "etp_tc_common.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
          "-Xcompiler", "-fPIC", "-I" + os.path.join(ROOT, "include"), "-I" + CSRC]

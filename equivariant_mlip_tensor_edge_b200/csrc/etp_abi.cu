@@ -214,9 +214,8 @@ static size_t ws_tc_offset(int n_edges) {
 }
 
 size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
-  (void)n_nodes;
-  if (!h || n_edges < 0) return 0;
-  return ws_tc_offset(n_edges) + tc::forward_tc_workspace_bytes(h->c);
+  if (!h || n_edges < 0 || n_nodes < 0) return 0;
+  return ws_tc_offset(n_edges) + tc::forward_tc_workspace_bytes(h->c, n_nodes);
 }
 
 // The tensor-core forward is the default; ETP_FORWARD=generic selects the all-FP32 kernel.

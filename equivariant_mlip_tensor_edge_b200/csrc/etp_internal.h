@@ -48,7 +48,7 @@ etp_status validate_graph(int n_nodes, int n_edges, const int* row_ptr, const in
 
 // ---- forward with the radial projection on tcgen05 tensor cores (etp_fwd_tc.cu)
 namespace tc {
-size_t forward_tc_workspace_bytes(const Ctx& c);
+size_t forward_tc_workspace_bytes(const Ctx& c, int n_nodes);
 etp_status forward_tc_status(const Ctx& c, const void* ws, cudaStream_t s);
 etp_status launch_forward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                              const float* edge_vec, const float* x, const float* W, float* out, void* ws,
