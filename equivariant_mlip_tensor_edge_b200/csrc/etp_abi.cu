@@ -206,8 +206,8 @@ etp_status etp_get_info(etp_handle h, etp_info_t* info) {
   return ETP_OK;
 }
 
-// Workspace: [recv_map: n_edges ints][validation scratch: n_edges + 1 ints][tensor-core forward:
-// pre-split weights + status word]
+// Workspace: [recv_map: n_edges ints][validation scratch: n_edges + 1 ints][tensor-core forward
+// or backward: pre-split weights + status word (+ per-unit edge-gradient partials)]
 static size_t ws_scratch_offset(int n_edges) { return align256(sizeof(int) * static_cast<size_t>(n_edges)); }
 static size_t ws_tc_offset(int n_edges) {
   return ws_scratch_offset(n_edges) + align256(sizeof(int) * (static_cast<size_t>(n_edges) + 1));
@@ -215,12 +215,20 @@ static size_t ws_tc_offset(int n_edges) {
 
 size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   if (!h || n_edges < 0 || n_nodes < 0) return 0;
-  return ws_tc_offset(n_edges) + tc::forward_tc_workspace_bytes(h->c, n_nodes);
+  const size_t f = tc::forward_tc_workspace_bytes(h->c, n_nodes);
+  const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
+  return ws_tc_offset(n_edges) + (f > b ? f : b);
 }
 
 // The tensor-core forward is the default; ETP_FORWARD=generic selects the all-FP32 kernel.
 static bool use_tc_forward() {
   const char* v = std::getenv("ETP_FORWARD");
+  return !(v && std::strcmp(v, "generic") == 0);
+}
+
+// Likewise for the backward: ETP_BACKWARD=generic selects the all-FP32 kernel.
+static bool use_tc_backward() {
+  const char* v = std::getenv("ETP_BACKWARD");
   return !(v && std::strcmp(v, "generic") == 0);
 }
 
@@ -315,6 +323,13 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
     if (st != ETP_OK) return st;
   }
   if (n_nodes == 0) return ETP_OK;
+  if (n_edges > 0 && use_tc_backward()) {
+    void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
+    st = tc::launch_backward_tc(h->c, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W, grad_out,
+                                grad_x, grad_edge_vec, recv_map, tcws, s);
+    if (st == ETP_OK && validate_requested()) st = tc::backward_tc_status(h->c, tcws, s);
+    return st;
+  }
   return launch_backward(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, t_row_ptr, t_perm, x,
                          W, grad_out, grad_x, grad_edge_vec, recv_map, s);
 }

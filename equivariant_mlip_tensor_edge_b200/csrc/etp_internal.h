@@ -46,13 +46,22 @@ etp_status launch_forces(int n_nodes, int n_edges, const int* row_ptr, const int
 etp_status validate_graph(int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                           const int* t_row_ptr, const int* t_perm, int* scratch, cudaStream_t s);
 
-// ---- forward with the radial projection on tcgen05 tensor cores (etp_fwd_tc.cu)
 namespace tc {
+// ---- forward with the radial projection on tcgen05 tensor cores (etp_fwd_tc.cu)
 size_t forward_tc_workspace_bytes(const Ctx& c, int n_nodes);
 etp_status forward_tc_status(const Ctx& c, const void* ws, cudaStream_t s);
 etp_status launch_forward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                              const float* edge_vec, const float* x, const float* W, float* out, void* ws,
                              cudaStream_t s);
+
+// ---- backward with the radial projections on tcgen05 tensor cores (etp_bwd_tc.cu)
+size_t backward_tc_workspace_bytes(const Ctx& c, int n_edges);
+etp_status backward_tc_status(const Ctx& c, const void* ws, cudaStream_t s);
+// recv: n_edges ints of scratch (filled with the receiver of every edge)
+etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const float* edge_vec,
+                              const int* t_row_ptr, const int* t_perm, const float* x, const float* W,
+                              const float* grad_out, float* grad_x, float* grad_edge_vec, int* recv, void* ws,
+                              cudaStream_t s);
 }  // namespace tc
 
 // ---- graph kernels (etp_graph.cu)

@@ -378,3 +378,66 @@ def test_forward_ragged_degrees_and_channels(lmax, c):
     ref = conv_forward(spec, rp, send[order], vec[order], x, W)
     assert np.all(out[degrees == 0] == 0.0)
     assert_blocks_close(out, ref, c, lmax, f"ragged forward lmax={lmax} C={c}")
+
+
+# ------------------------------------------------------------------ backward kernels: both implementations
+
+@pytest.mark.parametrize("impl", ["tc", "generic"])
+@pytest.mark.parametrize("name", ["tiny", "diamond1k"])
+def test_backward_both_kernels(wls, name, impl, monkeypatch):
+    if impl == "generic":
+        monkeypatch.setenv("ETP_BACKWARD", "generic")
+    monkeypatch.setenv("ETP_VALIDATE", "1")      # graph checks + device pipeline status word
+    wl = wls(name)
+    conv = _conv(wl)
+    spec = spec_of(wl)
+    x, W = _inputs(wl, conv)
+    gout = wl.cotangent()
+    g = _gpu_graph(wl)
+    args = (g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV), torch.from_numpy(gout).to(DEV))
+    gx, gv = conv.backward(*args)
+    ref_g = full_graph(wl)
+    rgx, rgv = conv_vjp(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, gout)
+    assert_blocks_close(_np(gx), rgx, wl.channels, wl.lmax, f"{name} grad_x ({impl})")
+    assert_close_rel(_np(gv), rgv, f"{name} grad_edge_vec ({impl})")
+    gx2, gv2 = conv.backward(*args)
+    assert torch.equal(gx, gx2) and torch.equal(gv, gv2), "backward is not bitwise deterministic"
+
+
+def _skewed_graph(n_nodes, degrees, seed, hub, silent, r_max=4.5):
+    """Receiver degrees as given; about half of all edges sent by `hub`, none by `silent`."""
+    rng = np.random.default_rng(seed)
+    recv = np.repeat(np.arange(n_nodes), degrees)
+    others = np.array([i for i in range(n_nodes) if i != silent])
+    send = np.where(rng.random(len(recv)) < 0.5, hub, rng.choice(others, size=len(recv)))
+    d = rng.standard_normal((len(recv), 3))
+    d /= np.linalg.norm(d, axis=1, keepdims=True)
+    vec = (d * rng.uniform(0.5, r_max, size=(len(recv), 1))).astype(np.float32)
+    return recv, send, vec
+
+
+@pytest.mark.parametrize("lmax,c", [(1, 20), (2, 24), (3, 8), (3, 36)])
+def test_backward_ragged_degrees_and_channels(lmax, c):
+    """Sender degrees from 0 to several 128-edge rounds, ragged tiles, C not a multiple of 16."""
+    from oracle.conv import ConvSpec
+    irr = "+".join(f"{c}x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
+    n = 13
+    degrees = np.array([0, 1, 31, 32, 33, 127, 128, 129, 300, 5, 0, 64, 97])
+    recv, send, vec = _skewed_graph(n, degrees, seed=10 + lmax, hub=3, silent=10)
+    conv = etp.EdgeConv(irr, lmax, irr, 8, 5.0)
+    spec = ConvSpec(irr, lmax, irr, 8, 5.0)
+    rng = np.random.default_rng(200 + lmax)
+    x = rng.standard_normal((n, spec.dim_in)).astype(np.float32)
+    W = (rng.standard_normal((8, len(spec.paths), c)) / np.sqrt(8)).astype(np.float32)
+    gout = rng.standard_normal((n, spec.dim_out)).astype(np.float32)
+    g = etp.build_csr(n, torch.from_numpy(recv).to(DEV), torch.from_numpy(send).to(DEV),
+                      torch.from_numpy(vec).to(DEV))
+    gx, gv = conv.backward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV),
+                           torch.from_numpy(gout).to(DEV))
+    gx, gv = _np(gx), _np(gv)
+    order = np.lexsort((send, recv))
+    rp = np.concatenate([[0], np.cumsum(degrees)])
+    rgx, rgv = conv_vjp(spec, rp, send[order], vec[order], x, W, gout)
+    assert np.all(gx[10] == 0.0)
+    assert_blocks_close(gx, rgx, c, lmax, f"ragged grad_x lmax={lmax} C={c}")
+    assert_close_rel(gv, rgv, f"ragged grad_edge_vec lmax={lmax} C={c}")
