@@ -39,6 +39,7 @@ SIGNATURES = {
     "etp_last_error": (ctypes.c_char_p, []),
     "etp_workspace_bytes": (_sz, [_vp, _i, _i]),
     "etp_forward": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "etp_forward_noalloc": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "etp_backward": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "etp_radial_weights": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
     "etp_forces": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),

@@ -20,6 +20,8 @@ static thread_local std::string g_last_error;
 
 void set_error(const std::string& msg) { g_last_error = msg; }
 
+const Ctx* ctx_of(etp_handle h) { return h ? &h->c : nullptr; }
+
 etp_status cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return ETP_OK;
   set_error(std::string(what) + ": " + cudaGetErrorString(e));

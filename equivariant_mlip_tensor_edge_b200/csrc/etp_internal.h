@@ -24,6 +24,9 @@ struct Ctx {
   float r_cut = 0.f;
 };
 
+// Configuration behind a handle (NULL for a NULL handle).
+const Ctx* ctx_of(etp_handle h);
+
 // Error message of the last failing call on this host thread.
 void set_error(const std::string& msg);
 etp_status cuda_status(cudaError_t e, const char* what);

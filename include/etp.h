@@ -30,7 +30,8 @@
  * Conventions.
  *   Pointers: every array argument is a CUDA DEVICE pointer owned by the caller unless the
  *   comment says "host". The library allocates no device memory; scratch comes from the caller
- *   through `workspace` (size from the matching *_workspace_bytes query, 256-byte aligned).
+ *   through `workspace` (size from the matching *_workspace_bytes query, 256-byte aligned),
+ *   except for etp_forward_noalloc, which uses a fixed array of the library's device module.
  *   Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default stream). Calls are
  *   asynchronous on that stream unless documented otherwise.
  *   Outputs are overwritten, never accumulated into.
@@ -62,7 +63,7 @@ typedef enum {
   ETP_ERR_UNSUPPORTED = 3,   /* well-formed but outside what the kernels implement */
   ETP_ERR_BAD_GRAPH = 4,     /* CSR arrays failed validation (ETP_VALIDATE=1) */
   ETP_ERR_CUDA = 5,          /* a CUDA runtime call or kernel launch failed */
-  ETP_ERR_CAPACITY = 6       /* an output buffer is smaller than the result (n_edges reported) */
+  ETP_ERR_CAPACITY = 6       /* an output buffer or fixed scratch is smaller than needed (n_edges reported) */
 } etp_status;
 
 typedef struct {
@@ -108,6 +109,26 @@ size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges);
 etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
                        const int* sender, const float* edge_vec, const float* x, const float* W,
                        float* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Forward without a workspace argument: the same computation, kernels and results as
+ * etp_forward, but its scratch (the tf32-split radial weight matrix and a status word) sits in
+ * a fixed 256 KiB array inside libetp's device module, one per device, so the call allocates no
+ * memory and takes nothing from the caller but the tensors.
+ * The method has no such call; it is an interface convenience. It is for callers that cannot
+ * provide device scratch: for instance a host program that reaches the model through a fixed
+ * plugin interface that hands over only the input and output tensors, with no allocator of its
+ * own and nowhere to keep a workspace alive between calls.
+ * Limit: a handle whose scratch would exceed the 256 KiB (lmax 3 with more than 160 channels)
+ * is refused with ETP_ERR_CAPACITY and a message naming both sizes; use etp_forward for it.
+ * The first call on each device looks up the array's device address once, with that device
+ * current (cudaGetSymbolAddress); make that first call before beginning any stream capture.
+ * Nothing in the array needs to start at zero: each call rewrites the weights in full and its
+ * first kernel clears the status word.
+ * Overlapping calls on one device (different streams or host threads) share the array and race
+ * with each other; order them (one stream, or events). The ETP_VALIDATE graph checks are not run. */
+etp_status etp_forward_noalloc(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                               const int* sender, const float* edge_vec, const float* x,
+                               const float* W, float* out, void* stream);
 
 /* Fused backward (vector-Jacobian product of etp_forward for the cotangent grad_out):
  *   grad_x[n_nodes][dim_in]        = dL/dx,        L = <grad_out, out>
