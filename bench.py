@@ -49,16 +49,17 @@ def fp32_peak_tflops(sm_mhz):
     return SM_COUNT * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
 
 
-def launches_per_step(info, n_nodes):
+def launches_per_step(info, n_nodes, min_image=True):
     """Kernels of this library launched by one step (checked against the ncu launch list).
 
-    neighbour list: count, scan init, scan, emit, iota, radix histogram, radix exclusive sum,
-    one onesweep pass per 8 key bits, receiver row pointers; forward: weight split, fused
-    forward; backward: weight split, edge receivers, fused backward, unit sum (more than one
-    16-channel unit); forces: one.
+    neighbour list: chunk counts, scan init, scan, row pointers, emit, then for orthorhombic cells
+    wider than 2 r_cut (every workload here) the reverse-edge transpose, otherwise iota, radix
+    histogram, radix exclusive sum, one onesweep pass per 8 key bits and the row pointers;
+    forward: weight split, fused forward; backward: weight split, edge receivers, fused backward,
+    unit sum (more than one 16-channel unit); forces: one.
     """
     key_bits = max(1, int(n_nodes).bit_length())
-    graph = 8 + (key_bits + 7) // 8
+    graph = 6 if min_image else 5 + 4 + (key_bits + 7) // 8
     units = (info["channels"] + 15) // 16
     return graph + 2 + 3 + (1 if units > 1 else 0) + 1
 

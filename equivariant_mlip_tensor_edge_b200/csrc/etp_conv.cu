@@ -352,25 +352,37 @@ __global__ void k_radial_weights(int n_edges, int C, float inv_rc, const float* 
   }
 }
 
+// One warp per node: F_k = sum over edges received minus sum over edges sent, lane-strided over
+// the two rows, then a fixed-order warp sum.
 __global__ void k_forces(int n_nodes, const int* __restrict__ row_ptr, const int* __restrict__ t_row_ptr,
                          const int* __restrict__ t_perm, const float* __restrict__ gv,
                          float* __restrict__ f) {
-  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n_nodes; k += gridDim.x * blockDim.x) {
+  const int lane = threadIdx.x & 31;
+  const int n_warps = gridDim.x * (blockDim.x >> 5);
+  for (int k = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); k < n_nodes; k += n_warps) {
     float fx = 0.f, fy = 0.f, fz = 0.f;
-    for (int e = row_ptr[k]; e < row_ptr[k + 1]; ++e) {
+    for (int e = row_ptr[k] + lane; e < row_ptr[k + 1]; e += 32) {
       fx += gv[3 * e];
       fy += gv[3 * e + 1];
       fz += gv[3 * e + 2];
     }
-    for (int q = t_row_ptr[k]; q < t_row_ptr[k + 1]; ++q) {
+    for (int q = t_row_ptr[k] + lane; q < t_row_ptr[k + 1]; q += 32) {
       const int e = t_perm[q];
       fx -= gv[3 * e];
       fy -= gv[3 * e + 1];
       fz -= gv[3 * e + 2];
     }
-    f[3 * k] = fx;
-    f[3 * k + 1] = fy;
-    f[3 * k + 2] = fz;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      fx += __shfl_xor_sync(kFull, fx, o);
+      fy += __shfl_xor_sync(kFull, fy, o);
+      fz += __shfl_xor_sync(kFull, fz, o);
+    }
+    if (lane == 0) {
+      f[3 * k] = fx;
+      f[3 * k + 1] = fy;
+      f[3 * k + 2] = fz;
+    }
   }
 }
 
@@ -526,8 +538,8 @@ etp_status launch_radial_weights(const Ctx& c, int n_edges, const float* edge_ve
 etp_status launch_forces(int n_nodes, int n_edges, const int* row_ptr, const int* t_row_ptr, const int* t_perm,
                          const float* grad_edge_vec, float* forces, cudaStream_t s) {
   (void)n_edges;
-  k_forces<<<blocks_for(n_nodes, 128, 4096), 128, 0, s>>>(n_nodes, row_ptr, t_row_ptr, t_perm, grad_edge_vec,
-                                                         forces);
+  k_forces<<<blocks_for(static_cast<long long>(n_nodes) * 32, 128, 4096), 128, 0, s>>>(n_nodes, row_ptr, t_row_ptr,
+                                                                                       t_perm, grad_edge_vec, forces);
   return cuda_status(cudaGetLastError(), "forces launch");
 }
 

@@ -34,7 +34,6 @@ namespace {
 
 constexpr int kQuads = 4;                     // receivers per group (TMEM lane quadrants)
 constexpr int kThreads = 32 * (kQuads + 1);
-constexpr int kSMax = 4;                      // tiles per receiver round (128 edges)
 constexpr int kUnitC = 16;                    // channels per work unit
 constexpr int kStages = 2;                    // gather stages per consumer warp
 
@@ -43,6 +42,7 @@ struct Cfg {
   static constexpr int D = Gen<L>::D;
   static constexpr int P = Gen<L>::P;
   static constexpr int K = L >= 3 ? 4 : 8;                     // channels per pass
+  static constexpr int SMAX = 4;                               // 32-edge tiles per receiver round
   static constexpr int NPASS = kUnitC / K;
   static constexpr int PPC = 32 / K;                           // paths per 32-column TMEM chunk
   static constexpr int NCOL = ((K * P + 15) / 16) * 16;        // MMA N
@@ -52,18 +52,18 @@ struct Cfg {
   static constexpr int STAGEB = 32 * SLOTB;                    // one warp's stage
   static constexpr int V = D * K;                              // values per lane per pass
   static constexpr int VS = 4 * ((V / 4) | 1);                 // reduction row stride (odd float4 count)
+  static_assert(VS * 4 <= SLOTB, "the reduction rows fit a gather stage");
   static constexpr int WSLICE = 2 * NCOL * 32;                 // bytes: hi + lo of one pass
   static constexpr int WBUF = NPASS * WSLICE;                  // one unit
   static constexpr int MAXRG = 64;                             // receiver groups cached per CTA
   // shared memory map (bytes)
   static constexpr int OFF_G = 1024;                           // cached row pointers
   static constexpr int OFF_A = OFF_G + 2048;                  // row-pointer cache: <= 2048 B
-  static constexpr int OFF_W = OFF_A + kSMax * 2 * 4096;
+  static constexpr int OFF_W = OFF_A + SMAX * 2 * 4096;
   static constexpr int OFF_Y = OFF_W + 2 * WBUF;
-  static constexpr int OFF_J = OFF_Y + kQuads * kSMax * D * 32 * 4;
-  static constexpr int OFF_X = OFF_J + kQuads * kSMax * 32 * 4;
-  static constexpr int OFF_R = OFF_X + kQuads * kStages * STAGEB;
-  static constexpr int END = OFF_R + kQuads * 32 * VS * 4;
+  static constexpr int OFF_J = OFF_Y + kQuads * SMAX * D * 32 * 4;
+  static constexpr int OFF_X = OFF_J + kQuads * SMAX * 32 * 4;
+  static constexpr int END = OFF_X + kQuads * kStages * STAGEB;
   static constexpr int SMEM = END < 118 * 1024 ? 118 * 1024 : END;   // > half an SM: one CTA per SM
   static_assert(END <= 227 * 1024, "shared memory budget");
   static_assert(OFF_A % 1024 == 0, "A tiles alignment");
@@ -94,6 +94,7 @@ struct GroupInfo {
   int beg[kQuads];
 };
 
+template <int SMAX>
 __device__ __forceinline__ void group_info(const Args& a, const int* rp, int rg_beg, int g, GroupInfo* gi) {
   gi->rg = g / a.n_units;
   gi->unit = g - gi->rg * a.n_units;
@@ -109,7 +110,7 @@ __device__ __forceinline__ void group_info(const Args& a, const int* rp, int rg_
     }
     gi->beg[q] = b;
     gi->deg[q] = d;
-    const int rr = (d + 32 * kSMax - 1) / (32 * kSMax);
+    const int rr = (d + 32 * SMAX - 1) / (32 * SMAX);
     rounds = rr > rounds ? rr : rounds;
   }
   gi->rounds = rounds;
@@ -117,18 +118,20 @@ __device__ __forceinline__ void group_info(const Args& a, const int* rp, int rg_
   gi->nbatch = (left >= kUnitC ? kUnitC : left) / 4;
 }
 
+template <int SMAX>
 __device__ __forceinline__ int tiles_of(int deg, int round) {
-  const int rem = deg - round * 32 * kSMax;
+  const int rem = deg - round * 32 * SMAX;
   if (rem <= 0) return 0;
   const int t = (rem + 31) / 32;
-  return t < kSMax ? t : kSMax;
+  return t < SMAX ? t : SMAX;
 }
 
+template <int SMAX>
 __device__ __forceinline__ int group_tiles(const GroupInfo& gi, int round) {
   int S = 0;
 #pragma unroll
   for (int q = 0; q < kQuads; ++q) {
-    const int t = tiles_of(gi.deg[q], round);
+    const int t = tiles_of<SMAX>(gi.deg[q], round);
     S = t > S ? t : S;
   }
   return S;
@@ -167,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   using G = Cfg<L>;
   using Gn = Gen<L>;
   constexpr int D = G::D, K = G::K, V = G::V, VS = G::VS, NCOL = G::NCOL, NSLOT = G::NSLOT;
-  constexpr int NPASS = G::NPASS;
+  constexpr int NPASS = G::NPASS, SMAX = G::SMAX;
   extern __shared__ __align__(1024) unsigned char smem[];
   uint64_t* tfull = reinterpret_cast<uint64_t*>(smem);   // [NSLOT]
   uint64_t* tempty = tfull + NSLOT;                       // [NSLOT]
@@ -178,12 +181,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(wfree + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* rp = reinterpret_cast<int*>(smem + G::OFF_G);
-  float* Atile = reinterpret_cast<float*>(smem + G::OFF_A);     // [kSMax][hl][128 x 8 canonical]
+  float* Atile = reinterpret_cast<float*>(smem + G::OFF_A);     // [SMAX][hl][128 x 8 canonical]
   float* Wbuf = reinterpret_cast<float*>(smem + G::OFF_W);      // [2][pass][hl][NCOL x 8]
   float* Ybuf = reinterpret_cast<float*>(smem + G::OFF_Y);      // [quad][tile][D][32]
   int* Jbuf = reinterpret_cast<int*>(smem + G::OFF_J);          // [quad][tile][32]
   unsigned char* Xbuf = smem + G::OFF_X;                        // [quad][stage][lane][SLOTB]
-  float* Red = reinterpret_cast<float*>(smem + G::OFF_R);       // [quad][32][VS]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -244,14 +246,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
     if (g_beg < g_end) ok = load_w(g_beg, 0);
     for (int g = g_beg; g < g_end && ok; ++g) {
       GroupInfo gi;
-      group_info(a, rp, rg_beg, g, &gi);
+      group_info<SMAX>(a, rp, rg_beg, g, &gi);
       const int wb = n_loads & 1;
       const int npass = (gi.nbatch * 4 + K - 1) / K;
       if (lane == 0) ok = mbar_wait(wload + wb, (n_loads >> 1) & 1, abort_flag, a.err, 12);
       ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
       ++n_loads;
       for (int round = 0; round < gi.rounds && ok; ++round) {
-        const int S = group_tiles(gi, round);
+        const int S = group_tiles<SMAX>(gi, round);
         if (gi.rg != cached_rg || round != cached_round) {
           ok = warp_wait(rready, n_setup & 1, abort_flag, a.err, 13);
           ++n_setup;
@@ -296,9 +298,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   } else {
     // ---------------------------------------------------------------- consumer warps
     const int q = warp;
-    float* Yq = Ybuf + q * (kSMax * D * 32);
-    int* Jq = Jbuf + q * (kSMax * 32);
-    float* Rw = Red + q * (32 * VS);
+    float* Yq = Ybuf + q * (SMAX * D * 32);
+    int* Jq = Jbuf + q * (SMAX * 32);
     unsigned char* Xw0 = Xbuf + q * kStages * G::STAGEB;
     unsigned char* Xw = Xw0 + lane * G::SLOTB;
     uint32_t titem = 0, n_setup = 0;
@@ -306,14 +307,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
     bool ok = true;
     for (int g = g_beg; g < g_end && ok; ++g) {
       GroupInfo gi;
-      group_info(a, rp, rg_beg, g, &gi);
+      group_info<SMAX>(a, rp, rg_beg, g, &gi);
       const int r = gi.rg * kQuads + q;
       const int deg = gi.deg[q];
       const int npass = (gi.nbatch * 4 + K - 1) / K;
       const int cbase = gi.unit * kUnitC;
       for (int round = 0; round < gi.rounds && ok; ++round) {
-        const int S = group_tiles(gi, round);
-        const int Sq = tiles_of(deg, round);
+        const int S = group_tiles<SMAX>(gi, round);
+        const int Sq = tiles_of<SMAX>(deg, round);
         if (gi.rg != cached_rg || round != cached_round) {
           // all consumers must be done with setup n-1 (its items consumed, hence the MMAs and
           // gathers that read the old tiles complete) before anyone overwrites it
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
             if (!ok) break;
           }
           for (int s = 0; s < Sq; ++s) {
-            const int le = round * 32 * kSMax + s * 32 + lane;
+            const int le = round * 32 * SMAX + s * 32 + lane;
             float Y[D];
             float R[kNumBasis], dR[kNumBasis];
 #pragma unroll
@@ -363,19 +364,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
           cached_round = round;
           if (!ok) break;
         }
-        // this lane's sender row for (pass, tile s): D components x K channels (whole sectors)
+        // the sender rows of tile s for a pass, D components x K channels each, into a stage.
+        // The K channels of a component are whole 32-byte sectors; the (K / 4) lanes that share an
+        // edge fetch its sectors' 16-byte halves in one instruction, so a sector is requested once.
         auto prefetch = [&](int pass, int s, int st) {
+          constexpr int PARTS = K / 4;                // 16-byte chunks per component
+          constexpr int EPI = 32 / PARTS;             // edges per instruction
           const int jj = Jq[s * 32 + lane];
           const int ch = cbase + pass * K;
-          const float* src = a.x + static_cast<size_t>(jj < 0 ? 0 : jj) * a.dim + ch;
-          unsigned char* dst = Xw + st * G::STAGEB;
-          const int nvalid = a.C - ch;        // channels of the pass inside C (multiple of 4)
+          const int part = lane % PARTS;
+          const bool in_c = 4 * part < a.C - ch;      // chunk inside C (C is a multiple of 4)
+          unsigned char* stage_base = Xw0 + st * G::STAGEB;
 #pragma unroll
-          for (int c = 0; c < D; ++c)
+          for (int it = 0; it < PARTS; ++it) {
+            const int e = it * EPI + lane / PARTS;
+            const int js = __shfl_sync(kFull, jj, e);
+            const float* src = a.x + static_cast<size_t>(js < 0 ? 0 : js) * a.dim + ch + 4 * part;
+            unsigned char* dst = stage_base + e * G::SLOTB + part * 16;
+            const uint32_t nb = (js >= 0 && in_c) ? 16u : 0u;
 #pragma unroll
-            for (int k4 = 0; k4 < K / 4; ++k4)
-              cp_async16(dst + (c * (K / 4) + k4) * 16, src + c * a.C + 4 * k4,
-                         (jj < 0 || 4 * k4 >= nvalid) ? 0u : 16u);
+            for (int c = 0; c < D; ++c) cp_async16(dst + c * K * 4, src + c * a.C, nb);
+          }
           cp_async_commit();
         };
         int stage = 0;
@@ -391,7 +400,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
             const bool mine = s < Sq;
             float xv[D][K];
             if (mine) {
-              cp_async_wait<0>();    // this item's row (the only copy in flight)
+              // this item's rows (the only copies in flight); the lanes that fetched this lane's
+              // row are others, and the stage the next copies target was read by every lane before
+              cp_async_wait<0>();
+              __syncwarp();
               const float4* xs = reinterpret_cast<const float4*>(Xw + stage * G::STAGEB);
 #pragma unroll
               for (int c = 0; c < D; ++c)
@@ -440,8 +452,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
             ++titem;
           }
           if (!ok) break;
-          // cross-lane sum of acc through shared memory, then one store (or add, later rounds)
+          // cross-lane sum of acc through shared memory, then one store (or add, later rounds).
+          // The rows go to the gather stage this warp consumed last (no copy targets it; the next
+          // one is issued after this sum).
           if (Sq > 0 || round == 0) {
+            float* Rw = reinterpret_cast<float*>(Xw0 + (stage ^ 1) * G::STAGEB);
 #pragma unroll
             for (int c = 0; c < D; ++c)
 #pragma unroll

@@ -71,80 +71,121 @@ __device__ __forceinline__ int count_pair(float3 pi, float3 pj, bool same, const
   return c;
 }
 
-// One warp per receiver: counts[i] = number of neighbours.
-__global__ void k_nbr_count(const float* __restrict__ pos, int n, CellParams cp, int* __restrict__ counts) {
+constexpr int kChunk = 256;   // senders per warp task
+
+// One warp per (receiver i, chunk c of kChunk senders): counts[i * n_chunks + c] = kept pairs.
+__global__ void k_nbr_count(const float* __restrict__ pos, int n, int n_chunks, CellParams cp,
+                            int* __restrict__ counts) {
   const int lane = threadIdx.x & 31;
-  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (i >= n) return;
-  const float3 pi = load_pos(pos, i);
-  int c = 0;
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const int j = j0 + lane;
-    if (j < n) c += count_pair(pi, load_pos(pos, j), j == i, cp);
-  }
+  const long long n_tasks = static_cast<long long>(n) * n_chunks;
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long t = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); t < n_tasks;
+       t += stride) {
+    const int i = static_cast<int>(t / n_chunks);
+    const int j_beg = static_cast<int>(t % n_chunks) * kChunk;
+    const int j_end = j_beg + kChunk < n ? j_beg + kChunk : n;
+    const float3 pi = load_pos(pos, i);
+    int c = 0;
+    for (int j = j_beg + lane; j < j_end; j += 32) c += count_pair(pi, load_pos(pos, j), j == i, cp);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
-  if (lane == 0) counts[i] = c;
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+    if (lane == 0) counts[t] = c;
+  }
 }
 
-// One warp per receiver: writes the row in canonical (sender, S) order.
-__global__ void k_nbr_emit(const float* __restrict__ pos, int n, CellParams cp,
-                           const int* __restrict__ row_ptr, int* __restrict__ sender,
-                           float* __restrict__ edge_vec, int* __restrict__ shift) {
+// row_ptr[0] = 0, row_ptr[i + 1] = inclusive chunk sum at the last chunk of receiver i.
+__global__ void k_row_ptr_chunks(const int* __restrict__ incl, int n, int n_chunks, int* __restrict__ row_ptr) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i <= n; i += gridDim.x * blockDim.x)
+    row_ptr[i] = i == 0 ? 0 : incl[static_cast<long long>(i) * n_chunks - 1];
+}
+
+// One warp per (receiver, chunk): writes the chunk's pairs in canonical (sender, S) order at the
+// chunk's offset (exclusive chunk sum), and the receiver of every written edge.
+__global__ void k_nbr_emit(const float* __restrict__ pos, int n, int n_chunks, CellParams cp,
+                           const int* __restrict__ counts, const int* __restrict__ incl,
+                           int* __restrict__ sender, float* __restrict__ edge_vec, int* __restrict__ shift,
+                           int* __restrict__ receiver) {
   const int lane = threadIdx.x & 31;
-  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (i >= n) return;
-  const float3 pi = load_pos(pos, i);
-  int base = row_ptr[i];
-  for (int j0 = 0; j0 < n; j0 += 32) {
-    const int j = j0 + lane;
-    const float3 pj = j < n ? load_pos(pos, j) : pi;
-    const int c = j < n ? count_pair(pi, pj, j == i, cp) : 0;
-    int incl = c;
+  const long long n_tasks = static_cast<long long>(n) * n_chunks;
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long t = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); t < n_tasks;
+       t += stride) {
+    if (counts[t] == 0) continue;
+    const int i = static_cast<int>(t / n_chunks);
+    const int j_beg = static_cast<int>(t % n_chunks) * kChunk;
+    const int j_end = j_beg + kChunk < n ? j_beg + kChunk : n;
+    const float3 pi = load_pos(pos, i);
+    int base = incl[t] - counts[t];
+    for (int j0 = j_beg; j0 < j_end; j0 += 32) {
+      const int j = j0 + lane;
+      const float3 pj = j < j_end ? load_pos(pos, j) : pi;
+      const int c = j < j_end ? count_pair(pi, pj, j == i, cp) : 0;
+      int incl_c = c;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    if (c > 0 && cp.min_image) {
-      const int s0 = nearest_image(pi.x, pj.x, cp.len[0], cp.n[0]);
-      const int s1 = nearest_image(pi.y, pj.y, cp.len[1], cp.n[1]);
-      const int s2 = nearest_image(pi.z, pj.z, cp.len[2], cp.n[2]);
-      double rx, ry, rz;
-      pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz);
-      const int at = base + incl - c;
-      sender[at] = j;
-      edge_vec[3 * at + 0] = static_cast<float>(rx);
-      edge_vec[3 * at + 1] = static_cast<float>(ry);
-      edge_vec[3 * at + 2] = static_cast<float>(rz);
-      if (shift) {
-        shift[3 * at + 0] = s0;
-        shift[3 * at + 1] = s1;
-        shift[3 * at + 2] = s2;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl_c, o);
+        if (lane >= o) incl_c += v;
       }
-    } else if (c > 0) {
-      int at = base + incl - c;
-      double rx, ry, rz;
-      for (int s0 = -cp.n[0]; s0 <= cp.n[0]; ++s0)
-        for (int s1 = -cp.n[1]; s1 <= cp.n[1]; ++s1)
-          for (int s2 = -cp.n[2]; s2 <= cp.n[2]; ++s2) {
-            if (j == i && s0 == 0 && s1 == 0 && s2 == 0) continue;
-            if (pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz)) {
-              sender[at] = j;
-              edge_vec[3 * at + 0] = static_cast<float>(rx);
-              edge_vec[3 * at + 1] = static_cast<float>(ry);
-              edge_vec[3 * at + 2] = static_cast<float>(rz);
-              if (shift) {
-                shift[3 * at + 0] = s0;
-                shift[3 * at + 1] = s1;
-                shift[3 * at + 2] = s2;
+      const int total = __shfl_sync(0xffffffffu, incl_c, 31);
+      if (c > 0 && cp.min_image) {
+        const int s0 = nearest_image(pi.x, pj.x, cp.len[0], cp.n[0]);
+        const int s1 = nearest_image(pi.y, pj.y, cp.len[1], cp.n[1]);
+        const int s2 = nearest_image(pi.z, pj.z, cp.len[2], cp.n[2]);
+        double rx, ry, rz;
+        pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz);
+        const int at = base + incl_c - c;
+        sender[at] = j;
+        receiver[at] = i;
+        edge_vec[3 * at + 0] = static_cast<float>(rx);
+        edge_vec[3 * at + 1] = static_cast<float>(ry);
+        edge_vec[3 * at + 2] = static_cast<float>(rz);
+        if (shift) {
+          shift[3 * at + 0] = s0;
+          shift[3 * at + 1] = s1;
+          shift[3 * at + 2] = s2;
+        }
+      } else if (c > 0) {
+        int at = base + incl_c - c;
+        double rx, ry, rz;
+        for (int s0 = -cp.n[0]; s0 <= cp.n[0]; ++s0)
+          for (int s1 = -cp.n[1]; s1 <= cp.n[1]; ++s1)
+            for (int s2 = -cp.n[2]; s2 <= cp.n[2]; ++s2) {
+              if (j == i && s0 == 0 && s1 == 0 && s2 == 0) continue;
+              if (pair_test(pi, pj, s0, s1, s2, cp, &rx, &ry, &rz)) {
+                sender[at] = j;
+                receiver[at] = i;
+                edge_vec[3 * at + 0] = static_cast<float>(rx);
+                edge_vec[3 * at + 1] = static_cast<float>(ry);
+                edge_vec[3 * at + 2] = static_cast<float>(rz);
+                if (shift) {
+                  shift[3 * at + 0] = s0;
+                  shift[3 * at + 1] = s1;
+                  shift[3 * at + 2] = s2;
+                }
+                ++at;
               }
-              ++at;
             }
-          }
+      }
+      base += total;
     }
-    base += total;
+  }
+}
+
+// Nearest-image lists are symmetric with at most one image per pair, and the image of j <- i is
+// minus that of i <- j (rint and the clamp are odd functions). So the transposed order needs no
+// sort: the edges j sends, in receiver order, are the reverses of row j's edges in sender order,
+// t_row_ptr = row_ptr and t_perm[m] = id of the reverse of edge m (sender j found in row i).
+__global__ void k_reverse_edges(const int* __restrict__ row_ptr, const int* __restrict__ sender,
+                                const int* __restrict__ receiver, int n_edges, int* __restrict__ t_perm) {
+  for (int m = blockIdx.x * blockDim.x + threadIdx.x; m < n_edges; m += gridDim.x * blockDim.x) {
+    const int j = receiver[m];
+    const int i = sender[m];
+    int lo = row_ptr[i], hi = row_ptr[i + 1];   // first entry of row i with sender >= j
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (sender[mid] < j) lo = mid + 1; else hi = mid;
+    }
+    t_perm[m] = lo;
   }
 }
 
@@ -152,15 +193,17 @@ __global__ void k_iota(int* __restrict__ v, int n) {
   for (int k = blockIdx.x * blockDim.x + threadIdx.x; k < n; k += gridDim.x * blockDim.x) v[k] = k;
 }
 
-// ptr[r] = first k with keys[k] >= r (keys sorted), r = 0..n_nodes.
-__global__ void k_lower_bound_ptr(const int* __restrict__ keys, int n_keys, int n_nodes, int* __restrict__ ptr) {
-  for (int r = blockIdx.x * blockDim.x + threadIdx.x; r <= n_nodes; r += gridDim.x * blockDim.x) {
-    int lo = 0, hi = n_keys;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (keys[mid] < r) lo = mid + 1; else hi = mid;
-    }
-    ptr[r] = lo;
+// ptr[r] = first k with keys[k] >= r (keys sorted), r = 0..n_nodes: every entry is written once,
+// by the edge at which the key passes r (or by the last edge / thread 0 at the ends).
+__global__ void k_ptr_from_sorted(const int* __restrict__ keys, int n_keys, int n_nodes, int* __restrict__ ptr) {
+  if (n_keys == 0) {
+    for (int r = blockIdx.x * blockDim.x + threadIdx.x; r <= n_nodes; r += gridDim.x * blockDim.x) ptr[r] = 0;
+    return;
+  }
+  for (int k = blockIdx.x * blockDim.x + threadIdx.x; k <= n_keys; k += gridDim.x * blockDim.x) {
+    const int lo = k == 0 ? 0 : keys[k - 1] + 1;      // keys in (keys[k-1], keys[k]] start at k
+    const int hi = k == n_keys ? n_nodes : keys[k];
+    for (int r = lo; r <= hi; ++r) ptr[r] = k;
   }
 }
 
@@ -194,8 +237,11 @@ int key_bits(int n_nodes) {
   return b;
 }
 
+int n_chunks_of(int n_nodes) { return n_nodes > 0 ? (n_nodes + kChunk - 1) / kChunk : 1; }
+
 struct GraphWs {
-  int* counts;   // n_nodes + 1
+  int* counts;   // n_nodes * n_chunks (+1)
+  int* incl;     // n_nodes * n_chunks
   int* ka;
   int* kb;
   int* va;
@@ -208,8 +254,9 @@ struct GraphWs {
 
 size_t cub_temp_bytes(int n_nodes, int max_edges) {
   size_t scan_b = 0, sort_b = 0;
+  const long long n_cnt = static_cast<long long>(n_nodes > 0 ? n_nodes : 1) * n_chunks_of(n_nodes);
   cub::DeviceScan::InclusiveSum(nullptr, scan_b, static_cast<const int*>(nullptr),
-                                static_cast<int*>(nullptr), n_nodes > 0 ? n_nodes : 1);
+                                static_cast<int*>(nullptr), static_cast<int>(n_cnt));
   cub::DeviceRadixSort::SortPairs(nullptr, sort_b, static_cast<const int*>(nullptr),
                                   static_cast<int*>(nullptr), static_cast<const int*>(nullptr),
                                   static_cast<int*>(nullptr), max_edges > 0 ? max_edges : 1, 0,
@@ -221,8 +268,11 @@ GraphWs carve(void* ws, int n_nodes, int max_edges) {
   char* p = static_cast<char*>(ws);
   GraphWs g;
   const size_t eb = align256(sizeof(int) * static_cast<size_t>(max_edges > 0 ? max_edges : 1));
+  const size_t cb = align256(sizeof(int) * (static_cast<size_t>(n_nodes) * n_chunks_of(n_nodes) + 1));
   g.counts = reinterpret_cast<int*>(p);
-  p += align256(sizeof(int) * (static_cast<size_t>(n_nodes) + 1));
+  p += cb;
+  g.incl = reinterpret_cast<int*>(p);
+  p += cb;
   g.ka = reinterpret_cast<int*>(p); p += eb;
   g.kb = reinterpret_cast<int*>(p); p += eb;
   g.va = reinterpret_cast<int*>(p); p += eb;
@@ -251,7 +301,8 @@ etp_status transpose(int n_nodes, int n_edges, const int* sender, int* t_row_ptr
                                                     0, key_bits(n_nodes), s);
     if (e != cudaSuccess) return cuda_status(e, "transpose sort");
   }
-  k_lower_bound_ptr<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.kb, n_edges, n_nodes, t_row_ptr);
+  k_ptr_from_sorted<<<grid_for((n_edges > n_nodes ? n_edges : n_nodes) + 1, 256), 256, 0, s>>>(g.kb, n_edges,
+                                                                                          n_nodes, t_row_ptr);
   return cuda_status(cudaGetLastError(), "transpose");
 }
 
@@ -259,8 +310,8 @@ etp_status transpose(int n_nodes, int n_edges, const int* sender, int* t_row_ptr
 
 size_t graph_workspace_bytes(int n_nodes, int max_edges) {
   const size_t eb = align256(sizeof(int) * static_cast<size_t>(max_edges > 0 ? max_edges : 1));
-  return align256(sizeof(int) * (static_cast<size_t>(n_nodes) + 1)) + 5 * eb + 256 +
-         align256(cub_temp_bytes(n_nodes, max_edges));
+  const size_t cb = align256(sizeof(int) * (static_cast<size_t>(n_nodes) * n_chunks_of(n_nodes) + 1));
+  return 2 * cb + 5 * eb + 256 + align256(cub_temp_bytes(n_nodes, max_edges));
 }
 
 etp_status neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,
@@ -306,15 +357,18 @@ etp_status neighbors(const float* pos, int n_nodes, const double* cell, const in
   }
   GraphWs g = carve(ws, n_nodes, max_edges);
   cudaError_t e;
+  const int n_chunks = n_chunks_of(n_nodes);
+  const long long n_tasks = static_cast<long long>(n_nodes) * n_chunks;
+  const int task_blocks = grid_for(n_tasks * 32, 256);
   if (n_nodes > 0) {
-    const int warps = 4;
-    k_nbr_count<<<(n_nodes + warps - 1) / warps, 32 * warps, 0, s>>>(pos, n_nodes, cp, g.counts);
+    k_nbr_count<<<task_blocks, 256, 0, s>>>(pos, n_nodes, n_chunks, cp, g.counts);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour count");
     size_t tb = g.cub_bytes;
-    e = cub::DeviceScan::InclusiveSum(g.cub_tmp, tb, g.counts, row_ptr + 1, n_nodes, s);
+    e = cub::DeviceScan::InclusiveSum(g.cub_tmp, tb, g.counts, g.incl, static_cast<int>(n_tasks), s);
     if (e != cudaSuccess) return cuda_status(e, "neighbour scan");
   }
-  if ((e = cudaMemsetAsync(row_ptr, 0, sizeof(int), s)) != cudaSuccess) return cuda_status(e, "memset");
+  k_row_ptr_chunks<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.incl, n_nodes, n_chunks, row_ptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "row pointers");
   int total = 0;
   if ((e = cudaMemcpyAsync(&total, row_ptr + n_nodes, sizeof(int), cudaMemcpyDeviceToHost, s)) != cudaSuccess)
     return cuda_status(e, "read edge count");
@@ -325,10 +379,16 @@ etp_status neighbors(const float* pos, int n_nodes, const double* cell, const in
     return ETP_ERR_CAPACITY;
   }
   if (n_nodes > 0 && total > 0) {
-    const int warps = 4;
-    k_nbr_emit<<<(n_nodes + warps - 1) / warps, 32 * warps, 0, s>>>(pos, n_nodes, cp, row_ptr, sender,
-                                                                   edge_vec, shift);
+    k_nbr_emit<<<task_blocks, 256, 0, s>>>(pos, n_nodes, n_chunks, cp, g.counts, g.incl, sender, edge_vec, shift,
+                                           g.ka);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour emit");
+  }
+  if (cp.min_image) {
+    e = cudaMemcpyAsync(t_row_ptr, row_ptr, sizeof(int) * (static_cast<size_t>(n_nodes) + 1),
+                        cudaMemcpyDeviceToDevice, s);
+    if (e != cudaSuccess) return cuda_status(e, "transposed row pointers");
+    if (total > 0) k_reverse_edges<<<grid_for(total, 256), 256, 0, s>>>(row_ptr, sender, g.ka, total, t_perm);
+    return cuda_status(cudaGetLastError(), "reverse edges");
   }
   return transpose(n_nodes, total, sender, t_row_ptr, t_perm, g, s);
 }
@@ -364,7 +424,8 @@ etp_status build_csr(int n_nodes, int n_edges, const int* receiver, const int* s
     if (e != cudaSuccess) return cuda_status(e, "csr sort 2");
     k_gather_edges<<<grid_for(n_edges, 256), 256, 0, s>>>(pm, n_edges, sender_in, edge_vec_in, sender, edge_vec);
   }
-  k_lower_bound_ptr<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.kb, n_edges, n_nodes, row_ptr);
+  k_ptr_from_sorted<<<grid_for((n_edges > n_nodes ? n_edges : n_nodes) + 1, 256), 256, 0, s>>>(g.kb, n_edges,
+                                                                                          n_nodes, row_ptr);
   if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "build_csr");
   return transpose(n_nodes, n_edges, sender, t_row_ptr, t_perm, g, s);
 }

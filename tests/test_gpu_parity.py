@@ -78,6 +78,41 @@ def test_neighbors_bit_exact_full(wls, name):
     assert np.array_equal(_np(g.t_perm), ref["t_perm"])
 
 
+class _Cell:
+    """A small periodic system for the neighbour paths that the workloads do not reach."""
+
+    def __init__(self, cell, n, seed, r_cut=5.0):
+        rng = np.random.default_rng(seed)
+        frac = rng.random((n, 3))
+        self.cell = np.asarray(cell, dtype=np.float64)
+        self.pos = (frac @ self.cell).astype(np.float32)
+        self.pbc = (True, True, True)
+        self.r_cut = np.float32(r_cut)
+        self.n_nodes = n
+
+
+@pytest.mark.parametrize("case", ["orthorhombic_small", "triclinic", "slab"])
+def test_neighbors_bit_exact_image_scan(case):
+    """Cells where the nearest-image shortcut does not apply: a periodic length below 2 r_cut
+    (several images of one pair), a sheared cell, and a slab periodic in two axes only."""
+    if case == "orthorhombic_small":
+        sysm = _Cell(np.diag([7.1, 7.6, 8.3]), 40, seed=21)
+    elif case == "triclinic":
+        sysm = _Cell([[11.0, 0.0, 0.0], [3.1, 10.5, 0.0], [-1.7, 2.2, 12.0]], 60, seed=22)
+    else:
+        sysm = _Cell(np.diag([12.0, 12.5, 30.0]), 50, seed=23)
+        sysm.pbc = (True, True, False)
+    ref = full_graph(sysm)
+    g = etp.neighbors(torch.from_numpy(sysm.pos).to(DEV), float(sysm.r_cut), cell=sysm.cell, pbc=sysm.pbc)
+    assert g.n_edges == len(ref["sender"])
+    assert np.array_equal(_np(g.row_ptr), ref["row_ptr"])
+    assert np.array_equal(_np(g.sender), ref["sender"])
+    assert np.array_equal(_np(g.shift), ref["shift"])
+    assert np.array_equal(_np(g.edge_vec).view(np.uint32), ref["edge_vec"].view(np.uint32))
+    assert np.array_equal(_np(g.t_row_ptr), ref["t_row_ptr"])
+    assert np.array_equal(_np(g.t_perm), ref["t_perm"])
+
+
 @pytest.mark.parametrize("name", ["diamond8k", "melt32k"])
 def test_neighbors_bit_exact_sampled(wls, name):
     wl = wls(name)
