@@ -197,6 +197,34 @@ def conv_vjp(spec, row_ptr, sender, edge_vec, x, W, grad_out):
     return grad_x, grad_vec
 
 
+def conv_vjp_weights(spec, row_ptr, sender, edge_vec, x, grad_out):
+    """Exact gradient of L = <grad_out, conv_forward(...)> with respect to W (float64).
+
+    The forward is linear in W through w_{e,p,u} = sum_b R_b(d_e) W[b,p,u], so
+      dL/dW[b,p,u] = sum_e R_b(d_e) dL/dw_{e,p,u},
+      dL/dw_{e,p,u} = sum_m3 g[recv, l3, m3, u] sum_{m1,m2} C[m1,m2,m3] x[send, l1, m1, u] Y_{l2 m2}(e).
+    Returns [n_basis, n_paths, C].
+    """
+    row_ptr = np.asarray(row_ptr, dtype=np.int64)
+    n_nodes = len(row_ptr) - 1
+    sender = np.asarray(sender, dtype=np.int64)
+    n_e = len(sender)
+    receiver = np.repeat(np.arange(n_nodes), np.diff(row_ptr))
+    x = np.asarray(x, dtype=np.float64)
+    g = np.asarray(grad_out, dtype=np.float64)
+    _, _, ys, rad = _edge_geometry(spec, edge_vec)
+    c, n_p = spec.channels, len(spec.paths)
+    dw_edge = np.zeros((n_e, n_p, c))
+    for p, (bi, l2, bo) in enumerate(spec.paths):
+        l1, _, l3 = spec.path_ls(p)
+        cg = cg_real(l1, l2, l3)
+        xj = x[sender][:, spec.in_slice(bi)].reshape(n_e, 2 * l1 + 1, c)
+        gi = g[receiver][:, spec.out_slice(bo)].reshape(n_e, 2 * l3 + 1, c)
+        s = np.einsum("abc,eb,eau->ecu", cg, ys[l2], xj)
+        dw_edge[:, p, :] = (gi * s).sum(axis=1)
+    return (rad.T @ dw_edge.reshape(n_e, n_p * c)).reshape(spec.n_basis, n_p, c)
+
+
 def flop_counts(spec):
     """Algorithmic operation counts per edge of the plain definition (FMA = 2 flops).
 

@@ -5,7 +5,7 @@ from scipy.spatial import cKDTree
 
 import workloads
 from oracle.cg import cg_real
-from oracle.conv import ConvSpec, conv_forward, conv_vjp, flop_counts, parse_irreps
+from oracle.conv import ConvSpec, conv_forward, conv_vjp, conv_vjp_weights, flop_counts, parse_irreps
 from oracle.graph import csr, forces_from_edge_grads, neighbors
 from oracle.radial import radial
 from oracle.wigner import euler_angles, random_rotation, wigner_D_real
@@ -253,6 +253,46 @@ def test_vjp_against_finite_differences_and_complex_step(tiny):
     xc = x.astype(np.complex128)
     xc[3, 2] += 1e-30j
     assert abs(_loss(tiny, xc, vec).imag / 1e-30 - gx[3, 2]) < 1e-12
+
+
+def test_weight_gradient_is_the_adjoint_of_the_forward(tiny):
+    # the forward is linear in W: <dL/dW, V> = <g, F(x; W = V)> for every V, exactly
+    spec, nb = tiny["spec"], tiny["nb"]
+    dw = conv_vjp_weights(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], tiny["g"])
+    assert dw.shape == (spec.n_basis, len(spec.paths), spec.channels)
+    rng = np.random.default_rng(12)
+    for _ in range(3):
+        v = rng.standard_normal(dw.shape)
+        out = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], v)
+        lhs = float((dw * v).sum())
+        rhs = float((tiny["g"] * out).sum())
+        assert abs(lhs - rhs) < 1e-10 * max(1.0, abs(rhs))
+    # a single nonzero entry of V picks out one entry of dW
+    v = np.zeros(dw.shape)
+    v[3, 2, 5] = 1.0
+    out = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], v)
+    assert abs(dw[3, 2, 5] - float((tiny["g"] * out).sum())) < 1e-12 * max(1.0, abs(dw[3, 2, 5]))
+
+
+def test_weight_gradient_scalar_only_brute_force(tiny):
+    # lmax = 0, 0e only: dL/dW[b,0,u] = sum_e R_b(d_e) g[recv,u] x[send,u], brute force loops
+    spec = ConvSpec("8x0e", 0, "8x0e", 8, float(tiny["wl"].r_cut))
+    nb = tiny["nb"]
+    rng = np.random.default_rng(8)
+    n = tiny["wl"].n_nodes
+    x = rng.standard_normal((n, 8))
+    g = rng.standard_normal((n, 8))
+    dw = conv_vjp_weights(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], x, g)
+    ref = np.zeros((8, 1, 8))
+    rc = np.float64(np.float32(spec.r_cut))
+    for e in range(len(nb["sender"])):
+        i, j = nb["receiver"][e], nb["sender"][e]
+        d = float(np.linalg.norm(nb["edge_vec"][e].astype(np.float64)))
+        rb = radial(np.array([d]), 8, rc)[0]
+        for b in range(8):
+            for u in range(8):
+                ref[b, 0, u] += rb[b] * g[i, u] * x[j, u]
+    assert np.abs(dw - ref).max() < 1e-12
 
 
 def test_forces_sum_and_torque(tiny):
