@@ -41,6 +41,7 @@ SIGNATURES = {
     "etp_forward": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "etp_forward_noalloc": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "etp_backward": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "etp_backward_weights": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "etp_radial_weights": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
     "etp_forces": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "etp_graph_workspace_bytes": (_sz, [_i, _i]),
@@ -264,6 +265,20 @@ class EdgeConv:
             _stream(dev)), "etp_backward")
         return (grad_x if want_grad_x else None), (grad_vec if want_grad_vec else None)
 
+    def backward_weights(self, graph, x, grad_out, grad_W=None, workspace=None):
+        """dL/dW [n_basis, n_paths, C] for L = <grad_out, forward(graph, x, W)>."""
+        torch = _torch()
+        _need_cuda(x, grad_out)
+        x, grad_out = _f32(x), _f32(grad_out)
+        if grad_W is None:
+            grad_W = torch.empty((self.info["n_basis"], self.info["n_paths"], self.info["channels"]),
+                                 dtype=torch.float32, device=x.device)
+        ws, nb = self._workspace(graph.n_nodes, graph.n_edges, x.device, workspace)
+        _check(load_library().etp_backward_weights(
+            self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.sender), _ptr(graph.edge_vec),
+            _ptr(x), _ptr(grad_out), _ptr(grad_W), _ptr(ws), nb, _stream(x.device)), "etp_backward_weights")
+        return grad_W
+
     def radial_weights(self, edge_vec, W):
         torch = _torch()
         _need_cuda(edge_vec, W)
@@ -277,7 +292,7 @@ class EdgeConv:
 
 
 def edge_conv_function():
-    """torch.autograd.Function: out = conv(x, edge_vec); gradients for x and edge_vec (not W)."""
+    """torch.autograd.Function: out = conv(x, edge_vec, W); gradients for x, edge_vec and W."""
     torch = _torch()
 
     class _EdgeConvFn(torch.autograd.Function):
@@ -292,10 +307,13 @@ def edge_conv_function():
         @staticmethod
         def backward(ctx, grad_out):
             x, W = ctx.saved_tensors
+            go = grad_out.contiguous()
+            gx = gv = gW = None
+            if ctx.needs_input_grad[2] or ctx.needs_input_grad[3]:
+                gx, gv = ctx.conv.backward(ctx.graph, x.detach(), W.detach(), go, ctx.needs_input_grad[2],
+                                           ctx.needs_input_grad[3])
             if ctx.needs_input_grad[4]:
-                raise NotImplementedError("the weight gradient dL/dW is not implemented")
-            gx, gv = ctx.conv.backward(ctx.graph, x, W, grad_out.contiguous(), ctx.needs_input_grad[2],
-                                       ctx.needs_input_grad[3])
-            return None, None, gx, gv, None
+                gW = ctx.conv.backward_weights(ctx.graph, x.detach(), go).reshape(W.shape)
+            return None, None, gx, gv, gW
 
     return _EdgeConvFn

@@ -209,7 +209,8 @@ etp_status etp_get_info(etp_handle h, etp_info_t* info) {
 }
 
 // Workspace: [recv_map: n_edges ints][validation scratch: n_edges + 1 ints][tensor-core forward
-// or backward: pre-split weights + status word (+ per-unit edge-gradient partials)]
+// or backward: pre-split weights + status word (+ per-unit edge-gradient partials), or the weight
+// gradient's per-edge-range partial sums]
 static size_t ws_scratch_offset(int n_edges) { return align256(sizeof(int) * static_cast<size_t>(n_edges)); }
 static size_t ws_tc_offset(int n_edges) {
   return ws_scratch_offset(n_edges) + align256(sizeof(int) * (static_cast<size_t>(n_edges) + 1));
@@ -219,7 +220,9 @@ size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   if (!h || n_edges < 0 || n_nodes < 0) return 0;
   const size_t f = tc::forward_tc_workspace_bytes(h->c, n_nodes);
   const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
-  return ws_tc_offset(n_edges) + (f > b ? f : b);
+  const size_t w = weight_grad_workspace_bytes(h->c, n_edges);
+  const size_t m = f > b ? f : b;
+  return ws_tc_offset(n_edges) + (m > w ? m : w);
 }
 
 // The tensor-core forward is the default; ETP_FORWARD=generic selects the all-FP32 kernel.
@@ -334,6 +337,41 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
   }
   return launch_backward(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, t_row_ptr, t_perm, x,
                          W, grad_out, grad_x, grad_edge_vec, recv_map, s);
+}
+
+etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                                const int* sender, const float* edge_vec, const float* x,
+                                const float* grad_out, float* grad_W, void* workspace,
+                                size_t workspace_bytes, void* stream) {
+  if (!h) {
+    set_error("etp_backward_weights: NULL handle");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_nodes < 0 || n_edges < 0) {
+    set_error("etp_backward_weights: negative size");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(n_nodes) * h->c.dim >= (1LL << 31)) {
+    set_error("etp_backward_weights: n_nodes * dim must stay below 2^31");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  if (!row_ptr || !grad_W || (n_edges > 0 && (!sender || !edge_vec || !x || !grad_out))) {
+    set_error("etp_backward_weights: NULL array");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_edges > 0 && (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges))) {
+    set_error("etp_backward_weights: workspace missing or smaller than etp_workspace_bytes()");
+    return ETP_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (validate_requested() && n_edges > 0) {
+    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_scratch_offset(n_edges));
+    etp_status st = validate_graph(n_nodes, n_edges, row_ptr, sender, nullptr, nullptr, scratch, s);
+    if (st != ETP_OK) return st;
+  }
+  int* recv = static_cast<int*>(workspace);
+  void* part = workspace ? static_cast<char*>(workspace) + ws_tc_offset(n_edges) : nullptr;
+  return launch_weight_grad(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, grad_out, grad_W, recv, part, s);
 }
 
 etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, const float* W,

@@ -714,4 +714,13 @@ etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int*
 }
 
 }  // namespace tc
+
+etp_status launch_recv_of_edge(const int* row_ptr, int n_nodes, int n_edges, int* recv, cudaStream_t s) {
+  if (n_edges <= 0) return ETP_OK;
+  int blocks = (n_edges + 255) / 256;
+  if (blocks > 8 * tc::bnum_sms()) blocks = 8 * tc::bnum_sms();
+  tc::k_recv_of_edge<<<blocks, 256, 0, s>>>(row_ptr, n_nodes, n_edges, recv);
+  return cuda_status(cudaGetLastError(), "edge receivers");
+}
+
 }  // namespace etp

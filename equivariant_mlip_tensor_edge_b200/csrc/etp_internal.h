@@ -67,6 +67,15 @@ etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int*
                               cudaStream_t s);
 }  // namespace tc
 
+// receiver of every canonical edge, recv[e] (etp_bwd_tc.cu)
+etp_status launch_recv_of_edge(const int* row_ptr, int n_nodes, int n_edges, int* recv, cudaStream_t s);
+
+// ---- weight gradient dL/dW (etp_dw.cu); recv: n_edges ints of scratch
+size_t weight_grad_workspace_bytes(const Ctx& c, int n_edges);
+etp_status launch_weight_grad(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
+                              const float* edge_vec, const float* x, const float* grad_out, float* grad_W,
+                              int* recv, void* ws, cudaStream_t s);
+
 // ---- graph kernels (etp_graph.cu)
 size_t graph_workspace_bytes(int n_nodes, int max_edges);
 etp_status neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,

@@ -6,7 +6,8 @@ Emits, for every supported l_max (in = SH = out = L):
     contraction sum_m gY_m dY_m/dr needed by the backward pass;
   * the path list (l1, l2, l3), lexicographic, triangle rule, l1 + l2 + l3 even;
   * per path, the real-basis Clebsch-Gordan nonzeros as float immediates inside
-    straight-line forward and backward contraction code.
+    straight-line forward and backward contraction code, and the per-path factor
+    of the weight gradient, sum_{m1,m3} x[l1 m1] (sum_m2 C Y[l2 m2]) g[l3 m3].
 
 Independent of the float64 oracle by construction: Clebsch-Gordan values come
 from ``sympy.physics.wigner.clebsch_gordan`` and the harmonic polynomials from a
@@ -264,6 +265,64 @@ def emit_paths(out, lmax):
                     out.append(f"      q{m2} = fmaf({repr_f32(np.float32(v))}, x[{idx(l1, a - l1)}][k] * g[{idx(l3, b - l3)}][k], q{m2});")
                 out.append(f"      gY[{idx(l2, m2 - l2)}] = fmaf(wp[k], q{m2}, gY[{idx(l2, m2 - l2)}]);")
         out.append("    }")
+        out.append("  }")
+    out.append("}")
+
+    # weight gradient factor (one edge, K channels): gw_p[k] = sum_{m1,m3} x[l1 m1] M[m3][m1] g[l3 m3],
+    # evaluated as x . (M^T g) or g . (M x), whichever side is shorter; handed to gsink per path.
+    out.append("template <int K, class GS>")
+    out.append(f"__device__ __forceinline__ void tp_gw_{lmax}(const float* Y, const float (&x)[{D}][K],")
+    out.append(f"    const float (&g)[{D}][K], GS&& gsink) {{")
+    for p, ((l1, l2, l3), c) in enumerate(zip(paths, cgs)):
+        out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
+        mnz = []
+        for m3 in range(2 * l3 + 1):
+            for m1 in range(2 * l1 + 1):
+                terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
+                if not terms:
+                    continue
+                if l2 == 0:
+                    e = repr_f32(np.float32(terms[0][0]))
+                else:
+                    e = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                out.append(f"    const float M{m3}_{m1} = {e};")
+                mnz.append((m3, m1))
+        out.append("    float gw[K];")
+        out.append("    #pragma unroll")
+        out.append("    for (int k = 0; k < K; ++k) {")
+        via_v = (2 * l1 + 1) <= (2 * l3 + 1)
+        first = True
+        if via_v:
+            for m1 in range(2 * l1 + 1):
+                col = [(a, b) for (a, b) in mnz if b == m1]
+                if not col:
+                    continue
+                a, b = col[0]
+                out.append(f"      float v{m1} = M{a}_{b} * g[{idx(l3, a - l3)}][k];")
+                for a, b in col[1:]:
+                    out.append(f"      v{m1} = fmaf(M{a}_{b}, g[{idx(l3, a - l3)}][k], v{m1});")
+                if first:
+                    out.append(f"      float t = x[{idx(l1, m1 - l1)}][k] * v{m1};")
+                    first = False
+                else:
+                    out.append(f"      t = fmaf(x[{idx(l1, m1 - l1)}][k], v{m1}, t);")
+        else:
+            for m3 in range(2 * l3 + 1):
+                row = [(a, b) for (a, b) in mnz if a == m3]
+                if not row:
+                    continue
+                a, b = row[0]
+                out.append(f"      float s{m3} = M{a}_{b} * x[{idx(l1, b - l1)}][k];")
+                for a, b in row[1:]:
+                    out.append(f"      s{m3} = fmaf(M{a}_{b}, x[{idx(l1, b - l1)}][k], s{m3});")
+                if first:
+                    out.append(f"      float t = g[{idx(l3, m3 - l3)}][k] * s{m3};")
+                    first = False
+                else:
+                    out.append(f"      t = fmaf(g[{idx(l3, m3 - l3)}][k], s{m3}, t);")
+        out.append("      gw[k] = t;" if not first else "      gw[k] = 0.0f;")
+        out.append("    }")
+        out.append(f"    gsink(IC<{p}>{{}}, gw);")
         out.append("  }")
     out.append("}")
     return P, nnz, s3

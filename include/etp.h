@@ -98,7 +98,8 @@ etp_status etp_get_info(etp_handle h, etp_info_t* info);
 const char* etp_status_string(etp_status s);
 const char* etp_last_error(void);
 
-/* Bytes of device workspace etp_forward / etp_backward need for a graph of this size. */
+/* Bytes of device workspace etp_forward / etp_backward / etp_backward_weights need for a graph of
+ * this size. */
 size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges);
 
 /* Fused forward: out[n_nodes][dim_out] = convolution of x[n_nodes][dim_in] over the CSR graph.
@@ -140,6 +141,17 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
                         const int* t_perm, const float* x, const float* W, const float* grad_out,
                         float* grad_x, float* grad_edge_vec, void* workspace,
                         size_t workspace_bytes, void* stream);
+
+/* Weight gradient of the convolution for the cotangent grad_out (the training path):
+ *   grad_W[n_basis][n_paths][C] = dL/dW,  L = <grad_out, out>,
+ *   dL/dW[b][p][u] = sum_e R_b(d_e) sum_{m1,m3} x[send, l1, m1, u] (sum_m2 C Y_{l2 m2}) g[recv, l3, m3, u].
+ * Runs over the canonical (receiver-sorted) order, with the channels on the lanes; partial sums
+ * per range of edges are added in range order, so repeated calls give identical bits.
+ * grad_W is overwritten (zero for a graph without edges). Uses the etp_workspace_bytes workspace. */
+etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                                const int* sender, const float* edge_vec, const float* x,
+                                const float* grad_out, float* grad_W, void* workspace,
+                                size_t workspace_bytes, void* stream);
 
 /* Radial projection alone: w_out[n_edges][n_paths][C] = sum_b R_b(|r_e|) W[b][p][u]. */
 etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, const float* W,

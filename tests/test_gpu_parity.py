@@ -476,3 +476,90 @@ def test_backward_ragged_degrees_and_channels(lmax, c):
     assert np.all(gx[10] == 0.0)
     assert_blocks_close(gx, rgx, c, lmax, f"ragged grad_x lmax={lmax} C={c}")
     assert_close_rel(gv, rgv, f"ragged grad_edge_vec lmax={lmax} C={c}")
+
+
+# ------------------------------------------------------------------ weight gradient dL/dW
+
+def _weight_grad_ref(wl, spec, x, gout):
+    from oracle.conv import conv_vjp_weights
+    ref_g = full_graph(wl)
+    return conv_vjp_weights(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, gout)
+
+
+@pytest.mark.parametrize("name", ["tiny", "diamond1k"])
+def test_weight_grad_parity_full(wls, name):
+    wl = wls(name)
+    conv = _conv(wl)
+    spec = spec_of(wl)
+    x, W = _inputs(wl, conv)
+    gout = wl.cotangent()
+    g = _gpu_graph(wl)
+    xd, gd = torch.from_numpy(x).to(DEV), torch.from_numpy(gout).to(DEV)
+    dw = conv.backward_weights(g, xd, gd)
+    ref = _weight_grad_ref(wl, spec, x, gout)
+    assert_close_rel(_np(dw), ref, f"{name} dL/dW")
+    assert torch.equal(dw, conv.backward_weights(g, xd, gd)), "weight gradient is not bitwise deterministic"
+
+
+@pytest.mark.parametrize("name", ["diamond8k", "melt32k"])
+def test_weight_grad_adjoint_at_full_size(wls, name):
+    """At sizes the oracle cannot finish: the forward is linear in W, so <dL/dW, V> = <g, F(W = V)>
+    for a random V, with both sides from the GPU (the forward is checked against the oracle)."""
+    wl = wls(name)
+    conv = _conv(wl)
+    x, _ = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    xd = torch.from_numpy(x).to(DEV)
+    gd = torch.from_numpy(wl.cotangent()).to(DEV)
+    dw = conv.backward_weights(g, xd, gd).double()
+    rng = np.random.default_rng(17)
+    v = torch.from_numpy(rng.standard_normal(tuple(dw.shape)).astype(np.float32)).to(DEV)
+    out = conv.forward(g, xd, v).double()
+    lhs = float((dw * v.double()).sum())
+    rhs = float((gd.double() * out).sum())
+    scale = float((dw.abs() * v.double().abs()).sum())
+    assert abs(lhs - rhs) <= 1e-5 * scale, (lhs, rhs, scale)
+
+
+@pytest.mark.parametrize("lmax,c", [(1, 20), (2, 24), (3, 8), (3, 36)])
+def test_weight_grad_ragged_degrees_and_channels(lmax, c):
+    from oracle.conv import ConvSpec, conv_vjp_weights
+    irr = "+".join(f"{c}x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
+    n = 13
+    degrees = np.array([0, 1, 31, 32, 33, 127, 128, 129, 300, 5, 0, 64, 97])
+    recv, send, vec = _skewed_graph(n, degrees, seed=20 + lmax, hub=3, silent=10)
+    conv = etp.EdgeConv(irr, lmax, irr, 8, 5.0)
+    spec = ConvSpec(irr, lmax, irr, 8, 5.0)
+    rng = np.random.default_rng(300 + lmax)
+    x = rng.standard_normal((n, spec.dim_in)).astype(np.float32)
+    gout = rng.standard_normal((n, spec.dim_out)).astype(np.float32)
+    g = etp.build_csr(n, torch.from_numpy(recv).to(DEV), torch.from_numpy(send).to(DEV),
+                      torch.from_numpy(vec).to(DEV))
+    dw = _np(conv.backward_weights(g, torch.from_numpy(x).to(DEV), torch.from_numpy(gout).to(DEV)))
+    order = np.lexsort((send, recv))
+    rp = np.concatenate([[0], np.cumsum(degrees)])
+    ref = conv_vjp_weights(spec, rp, send[order], vec[order], x, gout)
+    assert_close_rel(dw, ref, f"ragged dL/dW lmax={lmax} C={c}")
+
+
+def test_weight_grad_empty_graph_and_autograd(wls):
+    wl = wls("tiny")
+    conv = _conv(wl)
+    x, W = _inputs(wl, conv)
+    # no edges: the gradient is zero
+    n = 5
+    empty = etp.build_csr(n, torch.zeros(0, dtype=torch.int32, device=DEV), torch.zeros(0, dtype=torch.int32, device=DEV),
+                          torch.zeros((0, 3), dtype=torch.float32, device=DEV))
+    xe = torch.randn(n, conv.info["dim_in"], device=DEV)
+    ge = torch.randn(n, conv.info["dim_out"], device=DEV)
+    dw0 = conv.backward_weights(empty, xe, ge)
+    assert torch.count_nonzero(dw0) == 0
+    # autograd: W.grad equals backward_weights
+    g = _gpu_graph(wl)
+    fn = etp.edge_conv_function()
+    xt = torch.from_numpy(x).to(DEV)
+    Wt = torch.from_numpy(W).to(DEV).requires_grad_(True)
+    out = fn.apply(conv, g, xt, g.edge_vec, Wt)
+    gout = torch.from_numpy(wl.cotangent()).to(DEV)
+    (out * gout).sum().backward()
+    assert torch.equal(Wt.grad, conv.backward_weights(g, xt, gout))
