@@ -80,8 +80,12 @@ def algorithmic_counts(info, n_nodes, n_edges):
     radial = 2.0 * info["n_basis"] * info["n_paths"] * c * n_edges
     fwd_bytes = 4.0 * (2 * n_nodes * dim + 4 * n_edges + n_nodes + 1)
     bwd_bytes = 4.0 * (3 * n_nodes * dim + 4 * n_edges + 3 * n_edges + 2 * (n_nodes + 1) + n_edges)
-    return dict(fwd_flop=fwd_flop, bwd_flop=bwd_flop, fwd_radial_flop=radial, bwd_radial_flop=2 * radial,
-                fwd_bytes=fwd_bytes, bwd_bytes=bwd_bytes)
+    # weight gradient (etp_backward_weights): the per-path factor costs what the forward contraction
+    # does, and the edge reduction sum_e R_b gw runs on the FP32 pipe too (2 n_basis P C per edge)
+    dw_flop = fwd_flop + radial
+    dw_bytes = 4.0 * (2 * n_nodes * dim + 4 * n_edges + n_edges + n_nodes + 1)
+    return dict(fwd_flop=fwd_flop, bwd_flop=bwd_flop, dw_flop=dw_flop, fwd_radial_flop=radial,
+                bwd_radial_flop=2 * radial, fwd_bytes=fwd_bytes, bwd_bytes=bwd_bytes, dw_bytes=dw_bytes)
 
 
 # ---------------------------------------------------------------- recorded DRAM traffic
@@ -90,12 +94,13 @@ CSRC = os.path.join(ROOT, "equivariant_mlip_tensor_edge_b200", "csrc")
 KERNEL_SOURCES = {
     "k_fwd_tc": ["etp_fwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_bwd_tc": ["etp_bwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
+    "k_dw": ["etp_dw.cu", "etp_device.h", "generated/etp_paths.h"],
 }
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised in
 # profiles/<kernel>_<workload>.md, keyed by a hash of the kernel's sources at capture time.
 RECORDED_TRAFFIC = {
-    ("k_fwd_tc", "diamond1k"): (3851520 + 0, "3dc4f01c49e106a4"),
-    ("k_bwd_tc", "diamond1k"): (6544640 + 256, "4fec9d22dbff828c"),
+    ("k_fwd_tc", "diamond1k"): (3852288 + 0, "7c719f2d835c7e28"),
+    ("k_bwd_tc", "diamond1k"): (6544384 + 0, "5b09b69388783517"),
 }
 
 
@@ -207,6 +212,7 @@ def run_gpu(args, rank, world, local_rank):
         gx=torch.empty((n, info["dim_in"]), dtype=torch.float32, device=dev),
         gv=torch.empty((cap, 3), dtype=torch.float32, device=dev),
         f=torch.empty((n, 3), dtype=torch.float32, device=dev),
+        dw=torch.empty((info["n_basis"], info["n_paths"], info["channels"]), dtype=torch.float32, device=dev),
     )
     lib = etp.load_library()
     import ctypes
@@ -242,10 +248,15 @@ def run_gpu(args, rank, world, local_rank):
 
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # > 126 MB L2
 
-    def timed(fn, k):
+    def timed(fn, k, host_ahead=False):
+        """Mean device time of fn over k calls, L2 flushed before each. host_ahead: a device-side
+        sleep after the flush lets the host enqueue fn entirely before the first event, so the
+        time is the kernels' alone, not the host's launch latency."""
         total = 0.0
         for _ in range(k):
             flush.fill_(1.0)
+            if host_ahead:
+                torch.cuda._sleep(400_000)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()
@@ -274,9 +285,11 @@ def run_gpu(args, rank, world, local_rank):
         dist.barrier()
     # per-kernel timings on the same stream (dominant kernels), same flush discipline
     reps = max(args.steps, 5)
-    ms_fwd = timed(lambda: conv_fwd(gr, x, W), reps)
-    ms_bwd = timed(lambda: conv_bwd(gr, x, W, gout), reps)
+    ms_fwd = timed(lambda: conv_fwd(gr, x, W), reps, host_ahead=True)
+    ms_bwd = timed(lambda: conv_bwd(gr, x, W, gout), reps, host_ahead=True)
     ms_graph = timed(lambda: graph_step(pos), reps)
+    ms_dw = timed(lambda: conv.backward_weights(gr, x, gout, grad_W=bufs["dw"], workspace=bufs["ws"]), reps,
+                  host_ahead=True)
     clocks = sampler.stop() if rank == 0 else None
 
     # end to end through the public API with host buffers (copies inside the timed region)
@@ -297,12 +310,12 @@ def run_gpu(args, rank, world, local_rank):
     d2h = out_h.numel() * 4 + f_h.numel() * 4
 
     e = gr.n_edges
-    t_local = torch.tensor([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph], dtype=torch.float64, device=dev)
+    t_local = torch.tensor([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw], dtype=torch.float64, device=dev)
     edges_local = torch.tensor([float(e)], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
         dist.all_reduce(edges_local, op=dist.ReduceOp.SUM)
-    ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph = t_local.tolist()
+    ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw = t_local.tolist()
     total_edges = edges_local.item()
     if rank != 0:
         return None
@@ -316,12 +329,13 @@ def run_gpu(args, rank, world, local_rank):
     def roof(kind, ms):
         flop = cnt[f"{kind}_flop"]
         ach = flop / (ms * 1e-3) / 1e12
-        kernel = "k_bwd_tc" if kind == "bwd" else "k_fwd_tc"
+        kernel = {"bwd": "k_bwd_tc", "fwd": "k_fwd_tc", "dw": "k_dw"}[kind]
         return {"bound": "alu", "achieved": round(ach, 3), "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
                 "frac": round(ach / fp32_peak, 4), "traffic": recorded_traffic(kernel, wl.name),
                 "kernel": kernel,
-                "timed": ("the whole etp_backward call (k_bprep, k_recv_of_edge, k_bwd_tc, k_sum_units)"
-                          if kind == "bwd" else "the whole etp_forward call (k_prep, k_fwd_tc)"),
+                "timed": {"bwd": "the whole etp_backward call (k_bprep, k_recv_of_edge, k_bwd_tc, k_sum_units)",
+                          "fwd": "the whole etp_forward call (k_prep, k_fwd_tc)",
+                          "dw": "the whole etp_backward_weights call (k_recv_of_edge, k_dw, k_dw_sum)"}[kind],
                 "peak_source": f"derived: 148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz ({peak_kind} sm_max_mhz)",
                 "ms_per_launch": round(ms, 5),
                 "hbm_frac_of_" + peak_kind: round(cnt[f"{kind}_bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
@@ -348,6 +362,8 @@ def run_gpu(args, rank, world, local_rank):
         "ms_fwd": round(ms_fwd, 5), "ms_bwd": round(ms_bwd, 5), "ms_graph": round(ms_graph, 5),
         "roofline": roof(dominant, ms_bwd if dominant == "bwd" else ms_fwd),
         "roofline_fwd": roof("fwd", ms_fwd),
+        "ms_weight_grad": round(ms_dw, 5),
+        "roofline_weight_grad": roof("dw", ms_dw),
         "e2e": {"value": round(total_edges / (ms_e2e * 1e-3), 1), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step(info, n) * args.steps,

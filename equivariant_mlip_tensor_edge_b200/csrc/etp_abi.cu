@@ -221,14 +221,24 @@ size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   const size_t f = tc::forward_tc_workspace_bytes(h->c, n_nodes);
   const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
   const size_t w = weight_grad_workspace_bytes(h->c, n_edges);
-  const size_t m = f > b ? f : b;
-  return ws_tc_offset(n_edges) + (m > w ? m : w);
+  const size_t cmw = cm::workspace_bytes(h->c);
+  size_t m = f > b ? f : b;
+  m = m > w ? m : w;
+  return ws_tc_offset(n_edges) + (m > cmw ? m : cmw);
 }
 
-// The tensor-core forward is the default; ETP_FORWARD=generic selects the all-FP32 kernel.
+// Forward kernels: the edge-major tensor-core kernel by default. ETP_FORWARD=channel selects the
+// channel-major kernel where it applies (l_max <= 2, C in {32, 64, 128}; faster on graphs with
+// irregular degrees, slower on the regular ones) and ETP_FORWARD=generic the all-FP32 one. Every
+// kernel is tested.
 static bool use_tc_forward() {
   const char* v = std::getenv("ETP_FORWARD");
   return !(v && std::strcmp(v, "generic") == 0);
+}
+
+static bool use_cm_forward(const Ctx& c) {
+  const char* v = std::getenv("ETP_FORWARD");
+  return cm::supported(c) && v && std::strcmp(v, "channel") == 0;
 }
 
 // Likewise for the backward: ETP_BACKWARD=generic selects the all-FP32 kernel.
@@ -294,6 +304,11 @@ etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_pt
       return ETP_ERR_INVALID_ARG;
     }
     void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
+    if (use_cm_forward(h->c)) {
+      st = cm::launch(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);
+      if (st == ETP_OK && validate_requested()) st = cm::status(h->c, tcws, s);
+      return st;
+    }
     st = tc::launch_forward_tc(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);
     if (st == ETP_OK && validate_requested()) st = tc::forward_tc_status(h->c, tcws, s);
     return st;

@@ -9,8 +9,8 @@
 // 8 x P sums of its channel in registers. The per-edge geometry (Y, R, indices) of 32 edges at a
 // time is computed one edge per lane and shared through shared memory. Receiver rows of the
 // cotangent change only at receiver boundaries (canonical order) and stay in registers.
-// Each warp writes its partial sums; a second kernel adds the edge ranges in order, so the
-// result does not depend on scheduling.
+// Each warp writes its partial sums; a second kernel adds the edge ranges in a fixed order, so
+// the result does not depend on scheduling.
 #include <cstdint>
 #include <string>
 
@@ -139,24 +139,24 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_dw(int n_edges, int C, 
   }
 }
 
-// dW[b][p][u] = sum over edge ranges, in range order
-__global__ void k_dw_sum(const float* __restrict__ part, int n_ranges, int n_out, float* __restrict__ dW) {
-  for (int o = blockIdx.x * blockDim.x + threadIdx.x; o < n_out; o += gridDim.x * blockDim.x) {
-    float s = 0.0f;
-    for (int r = 0; r < n_ranges; ++r) s += part[static_cast<size_t>(r) * n_out + o];
-    dW[o] = s;
+// dW[b][p][u] = sum over edge ranges: a block per 32 outputs, warp w adds the ranges w, w + 8, ...
+// in order, then warp 0 adds the 8 warp sums in order (a fixed summation tree: deterministic).
+__global__ void __launch_bounds__(256) k_dw_sum(const float* __restrict__ part, int n_ranges, int n_out,
+                                                float* __restrict__ dW) {
+  __shared__ float ws[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int o = blockIdx.x * 32 + lane;
+  float s = 0.0f;
+  if (o < n_out)
+    for (int r = w; r < n_ranges; r += 8) s += part[static_cast<size_t>(r) * n_out + o];
+  ws[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && o < n_out) {
+    float t = ws[0][lane];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) t += ws[k][lane];
+    dW[o] = t;
   }
-}
-
-int g_dsms = 0;
-int dnum_sms() {
-  if (g_dsms == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&g_dsms, cudaDevAttrMultiProcessorCount, dev);
-    if (g_dsms <= 0) g_dsms = 148;
-  }
-  return g_dsms;
 }
 
 // Edge ranges: about 16 warps per SM in total, ranges a multiple of 32 edges.
@@ -193,9 +193,7 @@ etp_status dw_launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr,
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return cuda_status(e, "weight gradient launch");
   }
-  int sblocks = (n_out + 255) / 256;
-  if (sblocks > 8 * dnum_sms()) sblocks = 8 * dnum_sms();
-  k_dw_sum<<<sblocks, 256, 0, s>>>(part, n_ranges, n_out, dW);
+  k_dw_sum<<<(n_out + 31) / 32, 256, 0, s>>>(part, n_ranges, n_out, dW);
   return cuda_status(cudaGetLastError(), "weight gradient sum launch");
 }
 

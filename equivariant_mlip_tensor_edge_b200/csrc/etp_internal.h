@@ -67,6 +67,15 @@ etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int*
                               cudaStream_t s);
 }  // namespace tc
 
+// ---- channel-major forward (etp_fwd_cm.cu): l_max <= 2 and C in {32, 64, 128}
+namespace cm {
+bool supported(const Ctx& c);
+size_t workspace_bytes(const Ctx& c);
+etp_status launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
+                  const float* edge_vec, const float* x, const float* W, float* out, void* ws, cudaStream_t s);
+etp_status status(const Ctx& c, const void* ws, cudaStream_t s);
+}  // namespace cm
+
 // receiver of every canonical edge, recv[e] (etp_bwd_tc.cu)
 etp_status launch_recv_of_edge(const int* row_ptr, int n_nodes, int n_edges, int* recv, cudaStream_t s);
 
