@@ -176,6 +176,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- ranks
+
+def combine_ranks(times_ms, edges, world, device):
+    """Whole-job numbers of a multi-rank run: every timing is the maximum over the ranks (the
+    slowest replica sets the step time) and the edges are summed (every replica's edges count
+    toward the job's throughput). A no-op for one rank."""
+    import torch
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    e = torch.tensor([float(edges)], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(e, op=dist.ReduceOp.SUM)
+    return t.tolist(), e.item()
+
+
 # ---------------------------------------------------------------- GPU arm
 
 def run_gpu(args, rank, world, local_rank):
@@ -310,13 +326,8 @@ def run_gpu(args, rank, world, local_rank):
     d2h = out_h.numel() * 4 + f_h.numel() * 4
 
     e = gr.n_edges
-    t_local = torch.tensor([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw], dtype=torch.float64, device=dev)
-    edges_local = torch.tensor([float(e)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_local, op=dist.ReduceOp.MAX)
-        dist.all_reduce(edges_local, op=dist.ReduceOp.SUM)
-    ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw = t_local.tolist()
-    total_edges = edges_local.item()
+    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw), total_edges = combine_ranks(
+        [ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw], e, world, dev)
     if rank != 0:
         return None
 
