@@ -123,11 +123,19 @@ def _edge_rows(row_ptr, receivers):
     return receivers, edges.astype(np.int64), local
 
 
-def conv_forward(spec, row_ptr, sender, edge_vec, x, W, receivers=None):
+def _mask_bits(path_mask, n_p):
+    """[E, n_p] 0/1 array from per-edge masks (bit p of path_mask[e] set: path p is on)."""
+    m = np.asarray(path_mask, dtype=np.uint64)
+    return ((m[:, None] >> np.arange(n_p, dtype=np.uint64)[None, :]) & np.uint64(1)).astype(np.float64)
+
+
+def conv_forward(spec, row_ptr, sender, edge_vec, x, W, receivers=None, path_mask=None):
     """out[i] for i in ``receivers`` (default: all). Returns [len(receivers), dim_out].
 
     x: [N, dim_in]; W: [n_basis, n_paths, C]. Inputs are upcast to float64
     (complex inputs stay complex, for complex-step checks).
+    path_mask: optional per-edge integers (canonical order); path p contributes for edge e only
+    when bit p of path_mask[e] is set (per-edge path selection, as in adaptive-depth models).
     """
     receivers, edges, local = _edge_rows(row_ptr, receivers)
     sender = np.asarray(sender, dtype=np.int64)[edges]
@@ -137,6 +145,8 @@ def conv_forward(spec, row_ptr, sender, edge_vec, x, W, receivers=None):
     vec, d, ys, rad = _edge_geometry(spec, np.asarray(edge_vec)[edges])
     n_e, c, n_p = len(edges), spec.channels, len(spec.paths)
     w = (rad @ W.reshape(spec.n_basis, n_p * c)).reshape(n_e, n_p, c)
+    if path_mask is not None:
+        w = w * _mask_bits(np.asarray(path_mask)[edges], n_p)[:, :, None]
     dtype = np.result_type(vec, xs_all, np.float64)
     out = np.zeros((len(receivers), spec.dim_out), dtype=dtype)
     for p, (bi, l2, bo) in enumerate(spec.paths):
@@ -150,7 +160,7 @@ def conv_forward(spec, row_ptr, sender, edge_vec, x, W, receivers=None):
     return out
 
 
-def conv_vjp(spec, row_ptr, sender, edge_vec, x, W, grad_out):
+def conv_vjp(spec, row_ptr, sender, edge_vec, x, W, grad_out, path_mask=None):
     """Exact VJP of ``conv_forward`` (all receivers) with respect to x and the edge vectors.
 
     Returns grad_x [N, dim_in] and grad_edge_vec [E, 3] (float64).
@@ -173,6 +183,8 @@ def conv_vjp(spec, row_ptr, sender, edge_vec, x, W, grad_out):
     vec, d, ys, rad = _edge_geometry(spec, edge_vec)
     c, n_p = spec.channels, len(spec.paths)
     w = (rad @ W.reshape(spec.n_basis, n_p * c)).reshape(n_e, n_p, c)
+    mbits = _mask_bits(path_mask, n_p) if path_mask is not None else np.ones((n_e, n_p))
+    w = w * mbits[:, :, None]
     grad_x = np.zeros((n_nodes, spec.dim_in))
     grad_w = np.zeros((n_e, n_p, c))
     grad_y = [np.zeros((n_e, 2 * l + 1)) for l in range(spec.sh_lmax + 1)]
@@ -189,6 +201,7 @@ def conv_vjp(spec, row_ptr, sender, edge_vec, x, W, grad_out):
         s = np.einsum("abc,eb,eau->ecu", cg, ys[l2], xj)
         grad_w[:, p, :] = (gi * s).sum(axis=1)
         grad_y[l2] += np.einsum("abc,eau,ecu->eb", cg, xj, gw)
+    grad_w = grad_w * mbits[:, :, None]   # a masked path's weight does not reach the output
     grad_r = grad_w.reshape(n_e, n_p * c) @ W.reshape(spec.n_basis, n_p * c).T
     grad_d = (grad_r * radial_deriv(d, spec.n_basis, np.float64(np.float32(spec.r_cut)))).sum(axis=1)
     grad_vec = grad_d[:, None] * vec / d[:, None]

@@ -255,6 +255,56 @@ def test_vjp_against_finite_differences_and_complex_step(tiny):
     assert abs(_loss(tiny, xc, vec).imag / 1e-30 - gx[3, 2]) < 1e-12
 
 
+def test_path_mask_partitions_the_forward(tiny):
+    # paths are independent terms: a mask and its complement add up to the unmasked output, a
+    # single-path mask equals the forward with the other paths' weights zeroed, all-ones is a no-op
+    spec, nb = tiny["spec"], tiny["nb"]
+    n_e, n_p = len(nb["sender"]), len(spec.paths)
+    rng = np.random.default_rng(14)
+    mask = rng.integers(0, 1 << n_p, size=n_e)
+    full = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], tiny["W"])
+    a = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], tiny["W"], path_mask=mask)
+    b = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], tiny["W"],
+                     path_mask=((1 << n_p) - 1) ^ mask)
+    assert np.abs(a + b - full).max() < 1e-12 * np.abs(full).max()
+    ones = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], tiny["W"],
+                        path_mask=np.full(n_e, (1 << n_p) - 1))
+    assert np.array_equal(ones, full)
+    p = 2
+    only = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], tiny["W"],
+                        path_mask=np.full(n_e, 1 << p))
+    w2 = np.zeros_like(tiny["W"])
+    w2[:, p, :] = tiny["W"][:, p, :]
+    ref = conv_forward(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], w2)
+    assert np.abs(only - ref).max() < 1e-13 * max(1.0, np.abs(ref).max())
+
+
+def test_masked_vjp_against_finite_differences(tiny):
+    spec, nb = tiny["spec"], tiny["nb"]
+    n_e, n_p = len(nb["sender"]), len(spec.paths)
+    mask = np.random.default_rng(15).integers(0, 1 << n_p, size=n_e)
+    gx, gv = conv_vjp(spec, tiny["row_ptr"], nb["sender"], nb["edge_vec"], tiny["x"], tiny["W"], tiny["g"],
+                      path_mask=mask)
+    vec = nb["edge_vec"].astype(np.float64)
+
+    def loss(v):
+        out = conv_forward(spec, tiny["row_ptr"], nb["sender"], v, tiny["x"], tiny["W"], path_mask=mask)
+        return float((tiny["g"] * out).sum().real) if not np.iscomplexobj(out) else (tiny["g"] * out).sum()
+
+    rng = np.random.default_rng(16)
+    for _ in range(4):
+        e, k = rng.integers(n_e), rng.integers(3)
+        vc = vec.astype(np.complex128)
+        vc[e, k] += 1e-30j
+        cs = loss(vc).imag / 1e-30
+        assert abs(cs - gv[e, k]) < 1e-12 * max(1.0, abs(cs))
+    # grad_x: the loss is linear in x
+    xc = tiny["x"].astype(np.complex128)
+    xc[5, 3] += 1e-30j
+    out = conv_forward(spec, tiny["row_ptr"], nb["sender"], vec, xc, tiny["W"], path_mask=mask)
+    assert abs((tiny["g"] * out).sum().imag / 1e-30 - gx[5, 3]) < 1e-12
+
+
 def test_weight_gradient_is_the_adjoint_of_the_forward(tiny):
     # the forward is linear in W: <dL/dW, V> = <g, F(x; W = V)> for every V, exactly
     spec, nb = tiny["spec"], tiny["nb"]
