@@ -42,6 +42,9 @@ SIGNATURES = {
     "etp_forward_noalloc": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "etp_backward": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "etp_backward_weights": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "etp_forward_masked": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "etp_backward_masked": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
+                                 _vp]),
     "etp_radial_weights": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
     "etp_forces": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "etp_graph_workspace_bytes": (_sz, [_i, _i]),
@@ -235,20 +238,29 @@ class EdgeConv:
             workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=device)
         return workspace, nb
 
-    def forward(self, graph, x, W, out=None, workspace=None):
+    def forward(self, graph, x, W, out=None, workspace=None, path_mask=None):
+        """path_mask: optional int32 CUDA tensor [n_edges] (canonical order), bit p = path p on."""
         torch = _torch()
         _need_cuda(x, W, graph.row_ptr)
         x, W = _f32(x), _f32(W)
         if out is None:
             out = torch.empty((graph.n_nodes, self.info["dim_out"]), dtype=torch.float32, device=x.device)
         ws, nb = self._workspace(graph.n_nodes, graph.n_edges, x.device, workspace)
-        _check(load_library().etp_forward(self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr),
-                                          _ptr(graph.sender), _ptr(graph.edge_vec), _ptr(x), _ptr(W), _ptr(out),
-                                          _ptr(ws), nb, _stream(x.device)), "etp_forward")
+        lib = load_library()
+        if path_mask is None:
+            _check(lib.etp_forward(self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr),
+                                   _ptr(graph.sender), _ptr(graph.edge_vec), _ptr(x), _ptr(W), _ptr(out),
+                                   _ptr(ws), nb, _stream(x.device)), "etp_forward")
+        else:
+            _need_cuda(path_mask)
+            m = _i32(path_mask)
+            _check(lib.etp_forward_masked(self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr),
+                                          _ptr(graph.sender), _ptr(graph.edge_vec), _ptr(x), _ptr(W), _ptr(m),
+                                          _ptr(out), _ptr(ws), nb, _stream(x.device)), "etp_forward_masked")
         return out
 
     def backward(self, graph, x, W, grad_out, want_grad_x=True, want_grad_vec=True, grad_x=None,
-                 grad_vec=None, workspace=None):
+                 grad_vec=None, workspace=None, path_mask=None):
         torch = _torch()
         _need_cuda(x, W, grad_out)
         x, W, grad_out = _f32(x), _f32(W), _f32(grad_out)
@@ -258,11 +270,20 @@ class EdgeConv:
         if want_grad_vec and grad_vec is None:
             grad_vec = torch.empty((max(graph.n_edges, 1), 3), dtype=torch.float32, device=dev)[:graph.n_edges]
         ws, nb = self._workspace(graph.n_nodes, graph.n_edges, dev, workspace)
-        _check(load_library().etp_backward(
-            self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.sender), _ptr(graph.edge_vec),
-            _ptr(graph.t_row_ptr), _ptr(graph.t_perm), _ptr(x), _ptr(W), _ptr(grad_out),
-            _ptr(grad_x) if want_grad_x else None, _ptr(grad_vec) if want_grad_vec else None, _ptr(ws), nb,
-            _stream(dev)), "etp_backward")
+        gx_p = _ptr(grad_x) if want_grad_x else None
+        gv_p = _ptr(grad_vec) if want_grad_vec else None
+        if path_mask is None:
+            _check(load_library().etp_backward(
+                self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.sender), _ptr(graph.edge_vec),
+                _ptr(graph.t_row_ptr), _ptr(graph.t_perm), _ptr(x), _ptr(W), _ptr(grad_out), gx_p, gv_p, _ptr(ws), nb,
+                _stream(dev)), "etp_backward")
+        else:
+            _need_cuda(path_mask)
+            m = _i32(path_mask)
+            _check(load_library().etp_backward_masked(
+                self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.sender), _ptr(graph.edge_vec),
+                _ptr(graph.t_row_ptr), _ptr(graph.t_perm), _ptr(x), _ptr(W), _ptr(m), _ptr(grad_out), gx_p, gv_p,
+                _ptr(ws), nb, _stream(dev)), "etp_backward_masked")
         return (grad_x if want_grad_x else None), (grad_vec if want_grad_vec else None)
 
     def backward_weights(self, graph, x, grad_out, grad_W=None, workspace=None):

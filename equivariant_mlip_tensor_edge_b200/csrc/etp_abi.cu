@@ -354,6 +354,71 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
                          W, grad_out, grad_x, grad_edge_vec, recv_map, s);
 }
 
+etp_status etp_forward_masked(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                              const int* sender, const float* edge_vec, const float* x, const float* W,
+                              const uint32_t* path_mask, float* out, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+  etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_forward_masked");
+  if (st != ETP_OK) return st;
+  if (!out || !aligned16(out) || (n_edges > 0 && !path_mask)) {
+    set_error("etp_forward_masked: out (16-byte aligned) and path_mask must be device pointers");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges)) {
+    set_error("etp_forward_masked: workspace missing or smaller than etp_workspace_bytes()");
+    return ETP_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (validate_requested()) {
+    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_scratch_offset(n_edges));
+    st = validate_graph(n_nodes, n_edges, row_ptr, sender, nullptr, nullptr, scratch, s);
+    if (st != ETP_OK) return st;
+  }
+  if (n_nodes == 0) return ETP_OK;
+  void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
+  st = tc::launch_forward_tc(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s,
+                             n_edges > 0 ? path_mask : nullptr);
+  if (st == ETP_OK && validate_requested()) st = tc::forward_tc_status(h->c, tcws, s);
+  return st;
+}
+
+etp_status etp_backward_masked(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                               const int* sender, const float* edge_vec, const int* t_row_ptr,
+                               const int* t_perm, const float* x, const float* W,
+                               const uint32_t* path_mask, const float* grad_out, float* grad_x,
+                               float* grad_edge_vec, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_backward_masked");
+  if (st != ETP_OK) return st;
+  if (!t_row_ptr || (n_edges > 0 && (!t_perm || !grad_out || !path_mask)) || (!grad_x && !grad_edge_vec)) {
+    set_error("etp_backward_masked: NULL array (grad_x and grad_edge_vec may not both be NULL)");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if ((grad_x && !aligned16(grad_x)) || (grad_out && !aligned16(grad_out))) {
+    set_error("etp_backward_masked: grad_x and grad_out must be 16-byte aligned");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges)) {
+    set_error("etp_backward_masked: workspace missing or smaller than etp_workspace_bytes()");
+    return ETP_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (validate_requested()) {
+    int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_scratch_offset(n_edges));
+    st = validate_graph(n_nodes, n_edges, row_ptr, sender, t_row_ptr, t_perm, scratch, s);
+    if (st != ETP_OK) return st;
+  }
+  if (n_nodes == 0) return ETP_OK;
+  if (n_edges == 0)   // nothing is sent: zero outputs from the kernel without edges
+    return launch_backward(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, t_row_ptr, t_perm, x, W, grad_out,
+                           grad_x, grad_edge_vec, static_cast<int*>(workspace), s);
+  void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
+  st = tc::launch_backward_tc(h->c, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W, grad_out, grad_x,
+                              grad_edge_vec, static_cast<int*>(workspace), tcws, s, path_mask);
+  if (st == ETP_OK && validate_requested()) st = tc::backward_tc_status(h->c, tcws, s);
+  return st;
+}
+
 etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
                                 const int* sender, const float* edge_vec, const float* x,
                                 const float* grad_out, float* grad_W, void* workspace,

@@ -68,7 +68,8 @@ struct BCfg {
   static constexpr int OFF_E = OFF_W + 2 * WBUF;               // [quad][tile][EW][32]
   static constexpr int OFF_J = OFF_E + kQuads * SMAX * EW * 32 * 4;   // receivers [quad][tile][32]
   static constexpr int OFF_I = OFF_J + kQuads * SMAX * 32 * 4;        // edge ids   [quad][tile][32]
-  static constexpr int OFF_X = OFF_I + kQuads * SMAX * 32 * 4;
+  static constexpr int OFF_K = OFF_I + kQuads * SMAX * 32 * 4;        // path masks [quad][tile][32]
+  static constexpr int OFF_X = OFF_K + kQuads * SMAX * 32 * 4;
   static constexpr int OFF_R = OFF_X + kQuads * kStages * STAGEB;
   static constexpr int END = OFF_R + kQuads * 32 * VS * 4;
   static constexpr int SMEM = END < 118 * 1024 ? 118 * 1024 : END;
@@ -92,6 +93,7 @@ struct BArgs {
   const float* x;
   const float* g;         // grad_out
   const float* wt;
+  const uint32_t* mask;   // per-edge path mask (bit p: path p on), or null
   float* grad_x;          // may be null
   float* gpart;           // [unit][E][3] partial edge gradients, or grad_edge_vec when n_units == 1; may be null
   int n_edges;
@@ -207,7 +209,9 @@ __global__ void k_sum_units(const float* __restrict__ part, int n_units, int n_e
   }
 }
 
-template <int L>
+// MASKED: as in the forward, a path whose bit is clear in an edge's mask contributes nothing for
+// that edge (w = w' = 0), and a path no edge of the item needs is skipped.
+template <int L, bool MASKED>
 __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
   using G = BCfg<L>;
   using Gn = Gen<L>;
@@ -228,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
   float* Ebuf = reinterpret_cast<float*>(smem + G::OFF_E);    // [quad][tile][EW][32]
   int* Jbuf = reinterpret_cast<int*>(smem + G::OFF_J);        // receivers
   int* Ibuf = reinterpret_cast<int*>(smem + G::OFF_I);        // canonical edge ids
+  uint32_t* Kbuf = reinterpret_cast<uint32_t*>(smem + G::OFF_K);
   unsigned char* Xbuf = smem + G::OFF_X;
   float* Red = reinterpret_cast<float*>(smem + G::OFF_R);
 
@@ -335,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
     float* Eq = Ebuf + q * (SMAX * EW * 32);
     int* Jq = Jbuf + q * (SMAX * 32);
     int* Iq = Ibuf + q * (SMAX * 32);
+    uint32_t* Kq = Kbuf + q * (SMAX * 32);
     float* Rw = Red + q * (32 * VS);
     unsigned char* Xw = Xbuf + q * kStages * G::STAGEB + lane * G::SLOTB;
     uint32_t titem = 0, n_setup = 0;
@@ -383,6 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
             }
             Jq[s * 32 + lane] = recv;
             Iq[s * 32 + lane] = e;
+            if constexpr (MASKED) Kq[s * 32 + lane] = e >= 0 ? a.mask[e] : 0u;
             float* E = Eq + s * EW * 32 + lane;
 #pragma unroll
             for (int c = 0; c < D; ++c) E[c * 32] = Y[c];
@@ -493,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
               const uint32_t tb = tmem + (static_cast<uint32_t>(32 * q) << 16) + slot * G::SLOTC;
               float wch[16], dch[16];
               // (array bounds spelled G::K: see the forward kernel)
+              [[maybe_unused]] const uint32_t mbits = MASKED ? Kq[s * 32 + lane] : ~0u;
               auto wf = [&](auto pc, float (&wp)[G::K], float (&wdp)[G::K]) {
                 constexpr int p = decltype(pc)::value;
                 if constexpr (p % G::PPC == 0) {
@@ -501,10 +509,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
                   tmem_wait_ld();
                 }
                 constexpr int o = (p % G::PPC) * G::K;
+                if constexpr (MASKED) {
+                  const bool on = (mbits >> p) & 1u;
 #pragma unroll
-                for (int k = 0; k < G::K; ++k) {
-                  wp[k] = wch[o + k];
-                  wdp[k] = dch[o + k];
+                  for (int k = 0; k < G::K; ++k) {
+                    wp[k] = on ? wch[o + k] : 0.0f;
+                    wdp[k] = on ? dch[o + k] : 0.0f;
+                  }
+                  return __any_sync(kFull, on);
+                } else {
+#pragma unroll
+                  for (int k = 0; k < G::K; ++k) {
+                    wp[k] = wch[o + k];
+                    wdp[k] = dch[o + k];
+                  }
                 }
               };
               Gn::template bwd<K>(Y, wf, xv, gv, gx, gY, accd);
@@ -612,7 +630,7 @@ size_t bws_bytes(int channels, int n_edges) {
 template <int L>
 etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const float* edge_vec,
                    const int* t_row_ptr, const int* t_perm, const float* x, const float* W, const float* g,
-                   float* grad_x, float* grad_vec, int* recv, void* ws, cudaStream_t s) {
+                   float* grad_x, float* grad_vec, int* recv, void* ws, cudaStream_t s, const uint32_t* mask) {
   using G = BCfg<L>;
   const int n_units = (c.channels + kUnitC - 1) / kUnitC;
   char* p = static_cast<char*>(ws);
@@ -629,7 +647,8 @@ etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, c
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "backward prep");
-  e = cudaFuncSetAttribute(k_bwd_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+  e = mask ? cudaFuncSetAttribute(k_bwd_tc<L, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM)
+           : cudaFuncSetAttribute(k_bwd_tc<L, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return cuda_status(e, "tc backward smem attribute");
   BArgs a;
   a.n_nodes = n_nodes;
@@ -645,6 +664,7 @@ etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, c
   a.x = x;
   a.g = g;
   a.wt = wt;
+  a.mask = mask;
   a.grad_x = grad_x;
   a.gpart = grad_vec ? part : nullptr;
   a.n_edges = n_edges;
@@ -654,7 +674,8 @@ etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, c
   const long long min_grid = (n_rg + G::MAXRG - 3) / (G::MAXRG - 2);
   if (grid < min_grid) grid = min_grid;
   if (grid > a.n_groups) grid = a.n_groups;
-  k_bwd_tc<L><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
+  if (mask) k_bwd_tc<L, true><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
+  else k_bwd_tc<L, false><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "tc backward launch");
   if (grad_vec && n_units > 1 && n_edges > 0) {
@@ -700,14 +721,14 @@ etp_status backward_tc_status(const Ctx& c, const void* ws, cudaStream_t s) {
 etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const float* edge_vec,
                               const int* t_row_ptr, const int* t_perm, const float* x, const float* W,
                               const float* grad_out, float* grad_x, float* grad_edge_vec, int* recv, void* ws,
-                              cudaStream_t s) {
+                              cudaStream_t s, const uint32_t* path_mask) {
   switch (c.lmax) {
     case 1: return blaunch<1>(c, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W, grad_out, grad_x,
-                              grad_edge_vec, recv, ws, s);
+                              grad_edge_vec, recv, ws, s, path_mask);
     case 2: return blaunch<2>(c, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W, grad_out, grad_x,
-                              grad_edge_vec, recv, ws, s);
+                              grad_edge_vec, recv, ws, s, path_mask);
     case 3: return blaunch<3>(c, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W, grad_out, grad_x,
-                              grad_edge_vec, recv, ws, s);
+                              grad_edge_vec, recv, ws, s, path_mask);
   }
   set_error("tc backward: unsupported lmax");
   return ETP_ERR_UNSUPPORTED;

@@ -62,7 +62,8 @@ struct Cfg {
   static constexpr int OFF_W = OFF_A + SMAX * 2 * 4096;
   static constexpr int OFF_Y = OFF_W + 2 * WBUF;
   static constexpr int OFF_J = OFF_Y + kQuads * SMAX * D * 32 * 4;
-  static constexpr int OFF_X = OFF_J + kQuads * SMAX * 32 * 4;
+  static constexpr int OFF_K = OFF_J + kQuads * SMAX * 32 * 4;   // [quad][tile][32] path masks
+  static constexpr int OFF_X = OFF_K + kQuads * SMAX * 32 * 4;
   static constexpr int END = OFF_X + kQuads * kStages * STAGEB;
   static constexpr int SMEM = END < 118 * 1024 ? 118 * 1024 : END;   // > half an SM: one CTA per SM
   static_assert(END <= 227 * 1024, "shared memory budget");
@@ -83,6 +84,7 @@ struct Args {
   const float* edge_vec;
   const float* x;
   const float* wt;    // pre-split weights, [unit][pass][hi/lo][NCOL x 8 canonical]
+  const uint32_t* mask;   // per-edge path mask (bit p: path p on), or null
   float* out;
   int* err;
 };
@@ -165,7 +167,9 @@ __global__ void k_prep(const float* __restrict__ W, int C, int n_units, float* _
   }
 }
 
-template <int L>
+// MASKED: a path whose bit is clear in an edge's mask contributes nothing for that edge, and a
+// path no edge of the item needs is skipped.
+template <int L, bool MASKED>
 __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   using G = Cfg<L>;
   using Gn = Gen<L>;
@@ -185,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   float* Wbuf = reinterpret_cast<float*>(smem + G::OFF_W);      // [2][pass][hl][NCOL x 8]
   float* Ybuf = reinterpret_cast<float*>(smem + G::OFF_Y);      // [quad][tile][D][32]
   int* Jbuf = reinterpret_cast<int*>(smem + G::OFF_J);          // [quad][tile][32]
+  uint32_t* Kbuf = reinterpret_cast<uint32_t*>(smem + G::OFF_K); // [quad][tile][32]
   unsigned char* Xbuf = smem + G::OFF_X;                        // [quad][stage][lane][SLOTB]
 
   const int warp = threadIdx.x >> 5;
@@ -300,6 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
     const int q = warp;
     float* Yq = Ybuf + q * (SMAX * D * 32);
     int* Jq = Jbuf + q * (SMAX * 32);
+    uint32_t* Kq = Kbuf + q * (SMAX * 32);
     unsigned char* Xw0 = Xbuf + q * kStages * G::STAGEB;
     unsigned char* Xw = Xw0 + lane * G::SLOTB;
     uint32_t titem = 0, n_setup = 0;
@@ -342,6 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
               radial_basis<false>(dd, a.inv_rc, R, dR);
             }
             Jq[s * 32 + lane] = jj;
+            if constexpr (MASKED) Kq[s * 32 + lane] = jj >= 0 ? a.mask[gi.beg[q] + le] : 0u;
 #pragma unroll
             for (int c = 0; c < D; ++c) Yq[(s * D + c) * 32 + lane] = Y[c];
             const int row = 32 * q + lane;
@@ -433,6 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
               float wch[32];
               // (array bounds spelled G::K: a generic lambda whose parameter is sized by a local
               // constexpr of the kernel template crashes the CUDA 12.9 front end)
+              [[maybe_unused]] const uint32_t mbits = MASKED ? Kq[s * 32 + lane] : ~0u;
               auto wf = [&](auto pc, float (&wp)[G::K]) {
                 constexpr int p = decltype(pc)::value;
                 if constexpr (p % G::PPC == 0) {
@@ -441,8 +449,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
                   tmem_wait_ld();
                 }
                 constexpr int o = (p % G::PPC) * G::K;
+                if constexpr (MASKED) {
+                  const bool on = (mbits >> p) & 1u;
 #pragma unroll
-                for (int k = 0; k < G::K; ++k) wp[k] = wch[o + k];
+                  for (int k = 0; k < G::K; ++k) wp[k] = on ? wch[o + k] : 0.0f;
+                  return __any_sync(kFull, on);
+                } else {
+#pragma unroll
+                  for (int k = 0; k < G::K; ++k) wp[k] = wch[o + k];
+                }
               };
               Gn::template fwd<K>(Y, wf, xv, acc);
             }
@@ -531,7 +546,7 @@ int* status_word(const Ctx& c, void* ws) {
 
 template <int L>
 etp_status launch(const Ctx& c, int n_nodes, const int* row_ptr, const int* sender, const float* edge_vec,
-                  const float* x, const float* W, float* out, void* ws, cudaStream_t s) {
+                  const float* x, const float* W, const uint32_t* a_mask, float* out, void* ws, cudaStream_t s) {
   using G = Cfg<L>;
   const int n_units = (c.channels + kUnitC - 1) / kUnitC;
   float* wt = static_cast<float*>(ws);
@@ -539,7 +554,8 @@ etp_status launch(const Ctx& c, int n_nodes, const int* row_ptr, const int* send
   k_prep<L><<<32, 256, 0, s>>>(W, c.channels, n_units, wt, err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "forward prep");
-  e = cudaFuncSetAttribute(k_fwd_tc<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
+  e = a_mask ? cudaFuncSetAttribute(k_fwd_tc<L, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM)
+             : cudaFuncSetAttribute(k_fwd_tc<L, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
   if (e != cudaSuccess) return cuda_status(e, "tc forward smem attribute");
   Args a;
   a.n_nodes = n_nodes;
@@ -553,6 +569,7 @@ etp_status launch(const Ctx& c, int n_nodes, const int* row_ptr, const int* send
   a.edge_vec = edge_vec;
   a.x = x;
   a.wt = wt;
+  a.mask = a_mask;
   a.out = out;
   a.err = err;
   // enough CTAs that no CTA spans more than MAXRG receiver groups (row-pointer cache size)
@@ -561,7 +578,8 @@ etp_status launch(const Ctx& c, int n_nodes, const int* row_ptr, const int* send
   const long long min_grid = (n_rg + G::MAXRG - 3) / (G::MAXRG - 2);
   if (grid < min_grid) grid = min_grid;
   if (grid > a.n_groups) grid = a.n_groups;
-  k_fwd_tc<L><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
+  if (a_mask) k_fwd_tc<L, true><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
+  else k_fwd_tc<L, false><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
   return cuda_status(cudaGetLastError(), "tc forward launch");
 }
 
@@ -593,12 +611,12 @@ etp_status forward_tc_status(const Ctx& c, const void* ws, cudaStream_t s) {
 
 etp_status launch_forward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                              const float* edge_vec, const float* x, const float* W, float* out, void* ws,
-                             cudaStream_t s) {
+                             cudaStream_t s, const uint32_t* path_mask) {
   (void)n_edges;
   switch (c.lmax) {
-    case 1: return launch<1>(c, n_nodes, row_ptr, sender, edge_vec, x, W, out, ws, s);
-    case 2: return launch<2>(c, n_nodes, row_ptr, sender, edge_vec, x, W, out, ws, s);
-    case 3: return launch<3>(c, n_nodes, row_ptr, sender, edge_vec, x, W, out, ws, s);
+    case 1: return launch<1>(c, n_nodes, row_ptr, sender, edge_vec, x, W, path_mask, out, ws, s);
+    case 2: return launch<2>(c, n_nodes, row_ptr, sender, edge_vec, x, W, path_mask, out, ws, s);
+    case 3: return launch<3>(c, n_nodes, row_ptr, sender, edge_vec, x, W, path_mask, out, ws, s);
   }
   set_error("tc forward: unsupported lmax");
   return ETP_ERR_UNSUPPORTED;

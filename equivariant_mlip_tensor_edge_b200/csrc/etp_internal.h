@@ -53,9 +53,10 @@ namespace tc {
 // ---- forward with the radial projection on tcgen05 tensor cores (etp_fwd_tc.cu)
 size_t forward_tc_workspace_bytes(const Ctx& c, int n_nodes);
 etp_status forward_tc_status(const Ctx& c, const void* ws, cudaStream_t s);
+// path_mask: per canonical edge, bit p set = path p contributes (null: every path)
 etp_status launch_forward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                              const float* edge_vec, const float* x, const float* W, float* out, void* ws,
-                             cudaStream_t s);
+                             cudaStream_t s, const uint32_t* path_mask = nullptr);
 
 // ---- backward with the radial projections on tcgen05 tensor cores (etp_bwd_tc.cu)
 size_t backward_tc_workspace_bytes(const Ctx& c, int n_edges);
@@ -64,7 +65,7 @@ etp_status backward_tc_status(const Ctx& c, const void* ws, cudaStream_t s);
 etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const float* edge_vec,
                               const int* t_row_ptr, const int* t_perm, const float* x, const float* W,
                               const float* grad_out, float* grad_x, float* grad_edge_vec, int* recv, void* ws,
-                              cudaStream_t s);
+                              cudaStream_t s, const uint32_t* path_mask = nullptr);
 }  // namespace tc
 
 // ---- channel-major forward (etp_fwd_cm.cu): l_max <= 2 and C in {32, 64, 128}

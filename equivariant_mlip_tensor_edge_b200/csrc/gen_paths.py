@@ -174,7 +174,8 @@ def emit_paths(out, lmax):
     out.append(f"    const float (&x)[{D}][K], float (&acc)[{D}][K]) {{")
     for p, ((l1, l2, l3), c) in enumerate(zip(paths, cgs)):
         out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
-        out.append(f"    float wp[K]; wfetch(IC<{p}>{{}}, wp);")
+        out.append(f"    float wp[K];")
+        out.append(f"    if (fetch(wfetch, IC<{p}>{{}}, wp)) {{")
         # M[m3][m1] = sum_m2 C[m1,m2,m3] Y[l2,m2]
         mnz = []
         for m3 in range(2 * l3 + 1):
@@ -209,6 +210,7 @@ def emit_paths(out, lmax):
                     out.append(f"      s{m3} = fmaf(M{a}_{b}, x[{idx(l1, b - l1)}][k], s{m3});")
                 out.append(f"      acc[{idx(l3, m3 - l3)}][k] = fmaf(wp[k], s{m3}, acc[{idx(l3, m3 - l3)}][k]);")
         out.append("    }")
+        out.append("    }")
         out.append("  }")
     out.append("}")
 
@@ -222,7 +224,8 @@ def emit_paths(out, lmax):
     out.append(f"    float* gY, float& accd) {{")
     for p, ((l1, l2, l3), c) in enumerate(zip(paths, cgs)):
         out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
-        out.append(f"    float wp[K], wdp[K]; wfetch(IC<{p}>{{}}, wp, wdp);")
+        out.append(f"    float wp[K], wdp[K];")
+        out.append(f"    if (fetch(wfetch, IC<{p}>{{}}, wp, wdp)) {{")
         mnz = []
         for m3 in range(2 * l3 + 1):
             for m1 in range(2 * l1 + 1):
@@ -264,6 +267,7 @@ def emit_paths(out, lmax):
                 for v, a, b in terms[1:]:
                     out.append(f"      q{m2} = fmaf({repr_f32(np.float32(v))}, x[{idx(l1, a - l1)}][k] * g[{idx(l3, b - l3)}][k], q{m2});")
                 out.append(f"      gY[{idx(l2, m2 - l2)}] = fmaf(wp[k], q{m2}, gY[{idx(l2, m2 - l2)}]);")
+        out.append("    }")
         out.append("    }")
         out.append("  }")
     out.append("}")
@@ -468,12 +472,24 @@ def generate():
     out = ["// GENERATED by gen_paths.py -- do not edit.",
            "// Real-basis Clebsch-Gordan contractions and real spherical harmonics, unrolled per path.",
            "#pragma once",
+           "#include <type_traits>",
            "namespace etp_gen {",
            "// compile-time path index handed to the weight-fetch callback",
            "template <int N> struct IC {",
            "  static constexpr int value = N;",
            "  __host__ __device__ constexpr operator int() const { return N; }",
            "};",
+           "// wfetch(IC<p>, w...) fills the path's weights; a callback that returns bool can skip the",
+           "// path (false: no contribution), one that returns nothing always computes it",
+           "template <class F, class... A>",
+           "__device__ __forceinline__ bool fetch(F&& f, A&&... a) {",
+           "  if constexpr (std::is_void_v<decltype(f(a...))>) {",
+           "    f(a...);",
+           "    return true;",
+           "  } else {",
+           "    return f(a...);",
+           "  }",
+           "}",
            "template <int L> struct PathSet;",
            "template <int L, int G> struct CmLayout;"]
     for lmax in LMAX_SUPPORTED:

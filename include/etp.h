@@ -148,6 +148,23 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
  * Runs over the canonical (receiver-sorted) order, with the channels on the lanes; partial sums
  * per range of edges are added in range order, so repeated calls give identical bits.
  * grad_W is overwritten (zero for a graph without edges). Uses the etp_workspace_bytes workspace. */
+/* Per-edge path selection (adaptive computation: an edge may use only some of the paths).
+ * path_mask[n_edges] (device, canonical edge order): bit p set = path p contributes for that edge;
+ * a clear bit is the same as w_{e,p,u} = 0 for every u. Paths that no edge of a 32-edge tile needs
+ * are skipped, so masks that switch paths off for whole neighbourhoods also save time. Otherwise as
+ * etp_forward / etp_backward (always the tensor-core kernels; the backward is the VJP of the masked
+ * forward). */
+etp_status etp_forward_masked(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                              const int* sender, const float* edge_vec, const float* x, const float* W,
+                              const unsigned int* path_mask, float* out, void* workspace,
+                              size_t workspace_bytes, void* stream);
+etp_status etp_backward_masked(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
+                               const int* sender, const float* edge_vec, const int* t_row_ptr,
+                               const int* t_perm, const float* x, const float* W,
+                               const unsigned int* path_mask, const float* grad_out, float* grad_x,
+                               float* grad_edge_vec, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
 etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
                                 const int* sender, const float* edge_vec, const float* x,
                                 const float* grad_out, float* grad_W, void* workspace,

@@ -599,3 +599,48 @@ def test_forward_channel_major_ragged(lmax, c, monkeypatch):
     monkeypatch.delenv("ETP_FORWARD")
     edge = _np(conv.forward(g, xd, Wd))
     assert_blocks_close(o, edge.astype(np.float64), c, lmax, f"channel-major vs edge-major lmax={lmax} C={c}")
+
+
+# ------------------------------------------------------------------ per-edge path masks
+
+@pytest.mark.parametrize("name", ["tiny", "diamond1k"])
+def test_path_mask_forward_backward_parity(wls, name, monkeypatch):
+    monkeypatch.setenv("ETP_VALIDATE", "1")
+    wl = wls(name)
+    conv = _conv(wl)
+    spec = spec_of(wl)
+    x, W = _inputs(wl, conv)
+    gout = wl.cotangent()
+    g = _gpu_graph(wl)
+    ref_g = full_graph(wl)
+    n_p = conv.n_paths
+    rng = np.random.default_rng(31)
+    mask = rng.integers(0, 1 << n_p, size=g.n_edges).astype(np.int64)
+    mask[: g.n_edges // 3] = (1 << n_p) - 1          # some edges keep every path
+    md = torch.from_numpy(mask.astype(np.int32)).to(DEV)
+    xd, Wd, gd = torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV), torch.from_numpy(gout).to(DEV)
+    out = conv.forward(g, xd, Wd, path_mask=md)
+    ref = conv_forward(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, path_mask=mask)
+    assert_blocks_close(_np(out), ref, wl.channels, wl.lmax, f"{name} masked forward")
+    gx, gv = conv.backward(g, xd, Wd, gd, path_mask=md)
+    rgx, rgv = conv_vjp(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, gout, path_mask=mask)
+    assert_blocks_close(_np(gx), rgx, wl.channels, wl.lmax, f"{name} masked grad_x")
+    assert_close_rel(_np(gv), rgv, f"{name} masked grad_edge_vec")
+
+
+def test_path_mask_all_ones_and_zero(wls):
+    wl = wls("diamond1k")
+    conv = _conv(wl)
+    x, W = _inputs(wl, conv)
+    g = _gpu_graph(wl)
+    xd, Wd = torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)
+    gd = torch.from_numpy(wl.cotangent()).to(DEV)
+    ones = torch.full((g.n_edges,), (1 << conv.n_paths) - 1, dtype=torch.int32, device=DEV)
+    zero = torch.zeros(g.n_edges, dtype=torch.int32, device=DEV)
+    assert torch.equal(conv.forward(g, xd, Wd, path_mask=ones), conv.forward(g, xd, Wd))
+    assert torch.count_nonzero(conv.forward(g, xd, Wd, path_mask=zero)) == 0
+    gx1, gv1 = conv.backward(g, xd, Wd, gd, path_mask=ones)
+    gx0, gv0 = conv.backward(g, xd, Wd, gd)
+    assert torch.equal(gx1, gx0) and torch.equal(gv1, gv0)
+    gxz, gvz = conv.backward(g, xd, Wd, gd, path_mask=zero)
+    assert torch.count_nonzero(gxz) == 0 and torch.count_nonzero(gvz) == 0
