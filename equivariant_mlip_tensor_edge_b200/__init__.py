@@ -46,6 +46,7 @@ SIGNATURES = {
     "etp_backward_masked": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz,
                                  _vp]),
     "etp_radial_weights": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
+    "etp_node_ladder": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp]),
     "etp_forces": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "etp_graph_workspace_bytes": (_sz, [_i, _i]),
     "etp_neighbors": (_i, [_vp, _i, _dp, _ip, _f, _i, _ip, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -310,6 +311,25 @@ class EdgeConv:
         _check(load_library().etp_radial_weights(self._h, e, _ptr(edge_vec), _ptr(W), _ptr(out),
                                                  _stream(edge_vec.device)), "etp_radial_weights")
         return out
+
+
+def node_ladder(A, Ws, lmax, out=None):
+    """Node-local product ladder: out = B_1 + ... + B_nu with B_1 = A and B_{q+1} = P(B_q, A; Ws[q-1]).
+
+    A: [N, C (lmax+1)^2] float32 CUDA tensor (node-row layout); Ws: [nu - 1, n_paths, C] (nu - 1 may
+    be 0). Returns out like A.
+    """
+    torch = _torch()
+    _need_cuda(A, Ws)
+    A, Ws = _f32(A), _f32(Ws)
+    n, dim = A.shape
+    c = dim // ((lmax + 1) ** 2)
+    nu = Ws.shape[0] + 1
+    if out is None:
+        out = torch.empty_like(A)
+    _check(load_library().etp_node_ladder(int(lmax), c, n, nu, _ptr(A), _ptr(Ws) if nu > 1 else None, _ptr(out),
+                                          _stream(A.device)), "etp_node_ladder")
+    return out
 
 
 def edge_conv_function():

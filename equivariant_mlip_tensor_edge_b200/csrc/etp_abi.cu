@@ -454,6 +454,36 @@ etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const in
   return launch_weight_grad(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, grad_out, grad_W, recv, part, s);
 }
 
+etp_status etp_node_ladder(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,
+                           float* out, void* stream) {
+  if (lmax < 1 || lmax > kMaxL) {
+    set_error("etp_node_ladder: lmax must be 1, 2 or 3");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  if (channels < 4 || channels > 256 || channels % 4 != 0) {
+    set_error("etp_node_ladder: channels must be a multiple of 4 in [4, 256]");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  if (n_nodes < 0 || nu < 1 || nu > 8) {
+    set_error("etp_node_ladder: n_nodes >= 0 and 1 <= nu <= 8");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(n_nodes) * (lmax + 1) * (lmax + 1) * channels >= (1LL << 31)) {
+    set_error("etp_node_ladder: n_nodes * dim must stay below 2^31");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  if (n_nodes > 0 && (!A || !out || (nu > 1 && !W))) {
+    set_error("etp_node_ladder: NULL array");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if ((A && !aligned16(A)) || (out && !aligned16(out)) || (W && !aligned16(W))) {
+    set_error("etp_node_ladder: A, W and out must be 16-byte aligned");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_nodes == 0) return ETP_OK;
+  return launch_node_ladder(lmax, channels, n_nodes, nu, A, W, out, static_cast<cudaStream_t>(stream));
+}
+
 etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, const float* W,
                               float* w_out, void* stream) {
   if (!h || n_edges < 0 || (n_edges > 0 && (!edge_vec || !W || !w_out))) {

@@ -86,6 +86,10 @@ etp_status launch_weight_grad(const Ctx& c, int n_nodes, int n_edges, const int*
                               const float* edge_vec, const float* x, const float* grad_out, float* grad_W,
                               int* recv, void* ws, cudaStream_t s);
 
+// ---- node-local product ladder (etp_product.cu)
+etp_status launch_node_ladder(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,
+                              float* out, cudaStream_t s);
+
 // ---- graph kernels (etp_graph.cu)
 size_t graph_workspace_bytes(int n_nodes, int max_edges);
 etp_status neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,

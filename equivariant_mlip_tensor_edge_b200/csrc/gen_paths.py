@@ -7,7 +7,8 @@ Emits, for every supported l_max (in = SH = out = L):
   * the path list (l1, l2, l3), lexicographic, triangle rule, l1 + l2 + l3 even;
   * per path, the real-basis Clebsch-Gordan nonzeros as float immediates inside
     straight-line forward and backward contraction code, and the per-path factor
-    of the weight gradient, sum_{m1,m3} x[l1 m1] (sum_m2 C Y[l2 m2]) g[l3 m3].
+    of the weight gradient, sum_{m1,m3} x[l1 m1] (sum_m2 C Y[l2 m2]) g[l3 m3];
+  * the node-local path-reduced product of two feature rows (tp_node_L).
 
 Independent of the float64 oracle by construction: Clebsch-Gordan values come
 from ``sympy.physics.wigner.clebsch_gordan`` and the harmonic polynomials from a
@@ -332,6 +333,40 @@ def emit_paths(out, lmax):
     return P, nnz, s3
 
 
+# ---------------------------------------------------------------- node-local product
+def emit_node(out, lmax):
+    """acc[l3 m3][k] += w_p[k] sum_{m1,m2} C[m1,m2,m3] b[l1 m1][k] a[l2 m2][k] for every path: the
+    path-reduced product of two node features, one channel per k (FlashCart Fig. 3b)."""
+    paths = paths_for(lmax)
+    D = (lmax + 1) ** 2
+    ent = path_m_entries(lmax)
+    out.append("template <int K, class WF>")
+    out.append(f"__device__ __forceinline__ void tp_node_{lmax}(const float (&b)[{D}][K], const float (&a)[{D}][K],")
+    out.append(f"    WF&& wfetch, float (&acc)[{D}][K]) {{")
+    for p, (l1, l2, l3) in enumerate(paths):
+        out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
+        out.append("    float wp[K];")
+        out.append(f"    wfetch(IC<{p}>{{}}, wp);")
+        out.append("    #pragma unroll")
+        out.append("    for (int k = 0; k < K; ++k) {")
+        for m3 in range(2 * l3 + 1):
+            row = [(m1, terms) for (a3, m1, terms) in ent[p] if a3 == m3]
+            if not row:
+                continue
+            first = True
+            for m1, terms in row:
+                mexpr = " + ".join(f"{repr_f32(np.float32(v))}*a[{i}][k]" for v, i in terms)
+                if first:
+                    out.append(f"      float s{m3} = ({mexpr}) * b[{idx(l1, m1 - l1)}][k];")
+                    first = False
+                else:
+                    out.append(f"      s{m3} = fmaf({mexpr}, b[{idx(l1, m1 - l1)}][k], s{m3});")
+            out.append(f"      acc[{idx(l3, m3 - l3)}][k] = fmaf(wp[k], s{m3}, acc[{idx(l3, m3 - l3)}][k]);")
+        out.append("    }")
+        out.append("  }")
+    out.append("}")
+
+
 # ---------------------------------------------------------------- channel-major forward
 # Lanes hold channels; the paths are dealt to G warps that share a 32-channel slice (G = 128 / C
 # for C in {32, 64, 128}), so each warp evaluates a subset of the paths for every edge. The
@@ -497,6 +532,8 @@ def generate():
         emit_paths(out, lmax)
     for lmax in CM_LMAX:
         emit_cm(out, lmax)
+    for lmax in LMAX_SUPPORTED:
+        emit_node(out, lmax)
     out.append("}  // namespace etp_gen")
     return "\n".join(out) + "\n"
 

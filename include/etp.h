@@ -148,6 +148,17 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
  * Runs over the canonical (receiver-sorted) order, with the channels on the lanes; partial sums
  * per range of edges are added in range order, so repeated calls give identical bits.
  * grad_W is overwritten (zero for a graph without edges). Uses the etp_workspace_bytes workspace. */
+/* Node-local product ladder of correlation order nu (FlashCart Fig. 3b and Fig. E1, path-reduced):
+ *   B_1 = A,  B_{q+1}[l3, m3, u] = sum_{p=(l1,l2,l3)} W[q-1][p][u] sum_{m1,m2} C B_q[l1, m1, u] A[l2, m2, u],
+ *   out = B_1 + ... + B_nu,
+ * with the real Clebsch-Gordan coefficients and the path set of the convolution for in = SH = out
+ * = lmax (4, 11, 23 paths for lmax 1, 2, 3), no edges and no radial part. A, out: [n_nodes][dim]
+ * node rows (layout as for the convolution, dim = channels (lmax + 1)^2); W: [nu - 1][n_paths]
+ * [channels] (unused when nu == 1). channels: a multiple of 4 in [4, 256]; 1 <= nu <= 8. Device
+ * pointers, 16-byte aligned; asynchronous on stream; no workspace. */
+etp_status etp_node_ladder(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,
+                           float* out, void* stream);
+
 /* Per-edge path selection (adaptive computation: an edge may use only some of the paths).
  * path_mask[n_edges] (device, canonical edge order): bit p set = path p contributes for that edge;
  * a clear bit is the same as w_{e,p,u} = 0 for every u. Paths that no edge of a 32-edge tile needs

@@ -644,3 +644,21 @@ def test_path_mask_all_ones_and_zero(wls):
     assert torch.equal(gx1, gx0) and torch.equal(gv1, gv0)
     gxz, gvz = conv.backward(g, xd, Wd, gd, path_mask=zero)
     assert torch.count_nonzero(gxz) == 0 and torch.count_nonzero(gvz) == 0
+
+
+# ------------------------------------------------------------------ node-local product ladder
+
+@pytest.mark.parametrize("lmax,c,n,nu", [(1, 128, 4096, 3), (2, 128, 4096, 3), (3, 128, 4096, 2), (2, 64, 37, 5),
+                                        (3, 8, 37, 4), (1, 4, 5, 1)])
+def test_node_ladder_parity(lmax, c, n, nu):
+    """The node-local product ladder against the oracle: the pages' 4096-node x 128-channel case and
+    small ragged ones, correlation orders 1..5."""
+    from oracle.product import node_ladder, product_paths
+    rng = np.random.default_rng(600 + 10 * lmax + nu)
+    dim = (lmax + 1) ** 2 * c
+    n_p = len(product_paths(lmax))
+    A = rng.standard_normal((n, dim)).astype(np.float32)
+    Ws = (rng.standard_normal((nu - 1, n_p, c)) / np.sqrt(n_p)).astype(np.float32)
+    out = etp.node_ladder(torch.from_numpy(A).to(DEV), torch.from_numpy(Ws).to(DEV), lmax)
+    ref = node_ladder(lmax, c, A, Ws)
+    assert_blocks_close(_np(out), ref, c, lmax, f"node ladder lmax={lmax} C={c} nu={nu}")
