@@ -95,12 +95,14 @@ KERNEL_SOURCES = {
     "k_fwd_tc": ["etp_fwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_bwd_tc": ["etp_bwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_dw": ["etp_dw.cu", "etp_device.h", "generated/etp_paths.h"],
+    "k_node_ladder": ["etp_product.cu", "etp_device.h", "generated/etp_paths.h"],
 }
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised in
 # profiles/<kernel>_<workload>.md, keyed by a hash of the kernel's sources at capture time.
 RECORDED_TRAFFIC = {
-    ("k_fwd_tc", "diamond1k"): (3852288 + 0, "7c719f2d835c7e28"),
-    ("k_bwd_tc", "diamond1k"): (6544384 + 0, "5b09b69388783517"),
+    ("k_fwd_tc", "diamond1k"): (3857664 + 0, "2ef350fce27bf8a2"),
+    ("k_bwd_tc", "diamond1k"): (6545152 + 256, "fa34cf52cc7c6eaa"),
+    ("k_node_ladder", "ladder4096_l2"): (18898432 + 0, "6f03787ca5847418"),
 }
 
 
@@ -306,6 +308,16 @@ def run_gpu(args, rank, world, local_rank):
     ms_graph = timed(lambda: graph_step(pos), reps)
     ms_dw = timed(lambda: conv.backward_weights(gr, x, gout, grad_W=bufs["dw"], workspace=bufs["ws"]), reps,
                   host_ahead=True)
+    # node-local product ladder: 4096 nodes x 128 channels, correlation order 3, the workload's rank
+    lad = dict(n=4096, c=128, nu=3, lmax=wl.lmax)
+    gen = torch.Generator().manual_seed(1234)
+    lad_dim = (lad["lmax"] + 1) ** 2 * lad["c"]
+    lad_A = torch.randn((lad["n"], lad_dim), generator=gen).to(dev)
+    lad_W = (torch.randn((lad["nu"] - 1, info["n_paths"], lad["c"]), generator=gen) / info["n_paths"] ** 0.5).to(dev)
+    lad_out = torch.empty_like(lad_A)
+    for _ in range(3):
+        etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out)
+    ms_ladder = timed(lambda: etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out), reps, host_ahead=True)
     clocks = sampler.stop() if rank == 0 else None
 
     # end to end through the public API with host buffers (copies inside the timed region)
@@ -326,8 +338,8 @@ def run_gpu(args, rank, world, local_rank):
     d2h = out_h.numel() * 4 + f_h.numel() * 4
 
     e = gr.n_edges
-    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw), total_edges = combine_ranks(
-        [ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw], e, world, dev)
+    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder), total_edges = combine_ranks(
+        [ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder], e, world, dev)
     if rank != 0:
         return None
 
@@ -350,6 +362,25 @@ def run_gpu(args, rank, world, local_rank):
                 "peak_source": f"derived: 148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz ({peak_kind} sm_max_mhz)",
                 "ms_per_launch": round(ms, 5),
                 "hbm_frac_of_" + peak_kind: round(cnt[f"{kind}_bytes"] / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
+
+    def ladder_roof(ms):
+        """The ladder's bound is the slower of its compulsory HBM bytes (A read, out written, W) and
+        its FP32 work (3 nnz + 2 sum_p(2 l3 + 1) flop per node, channel and step)."""
+        steps = lad["nu"] - 1
+        flop = float(3 * info["cg_nnz"] + 2 * info["sum_2l3p1"]) * lad["c"] * lad["n"] * steps
+        byts = 4.0 * (2 * lad["n"] * lad_dim + steps * info["n_paths"] * lad["c"])
+        t_alu = flop / (fp32_peak * 1e12)
+        t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+        if t_hbm >= t_alu:
+            ach, peak, unit, bound = byts / (ms * 1e-3) / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
+        else:
+            ach, peak, unit, bound = flop / (ms * 1e-3) / 1e12, fp32_peak, "TFLOP/s", "alu"
+        return {"workload": f"{lad['n']} nodes x {lad['c']} channels, lmax {lad['lmax']}, order {lad['nu']}",
+                "kernel": "k_node_ladder", "ms_per_launch": round(ms, 5), "bound": bound,
+                "achieved": round(ach, 3), "peak": round(peak, 2), "unit": unit, "frac": round(ach / peak, 4),
+                "peak_source": peak_kind, "traffic": recorded_traffic("k_node_ladder", f"ladder4096_l{lad['lmax']}"),
+                "alu_frac": round(flop / (ms * 1e-3) / 1e12 / fp32_peak, 4),
+                "hbm_frac_of_" + peak_kind: round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
 
     line = {
         "metric": METRIC,
@@ -375,6 +406,7 @@ def run_gpu(args, rank, world, local_rank):
         "roofline_fwd": roof("fwd", ms_fwd),
         "ms_weight_grad": round(ms_dw, 5),
         "roofline_weight_grad": roof("dw", ms_dw),
+        "node_ladder": ladder_roof(ms_ladder),
         "e2e": {"value": round(total_edges / (ms_e2e * 1e-3), 1), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step(info, n) * args.steps,

@@ -16,7 +16,9 @@
 namespace etp {
 namespace {
 
-template <int L> struct NodeK { static constexpr int K = L >= 3 ? 2 : 4; };
+// Channels per thread: 2 (one 8-byte access per component row; measured faster than 1 or 4 at
+// 4096 nodes x 128 channels for every rank and order 2..5 but one, where it is within 5%).
+constexpr int kNodeK = 2;
 
 #define ETP_NODE_BIND(LL)                                                                              \
   template <int K, class WF>                                                                           \
@@ -48,28 +50,47 @@ __device__ __forceinline__ void store_k(float* p, const float (&v)[K]) {
   else *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
 }
 
+template <int D, int K>
+__device__ __forceinline__ void load_item(const float* A, int C, int node, int ch, float (&v)[D][K]) {
+  const float* ar = A + static_cast<size_t>(node) * D * C + ch;
+#pragma unroll
+  for (int c = 0; c < D; ++c) load_k<K>(ar + c * C, v[c]);
+}
+
 // W: [nu - 1][P][C]
 template <int L>
 __global__ void __launch_bounds__(256) k_node_ladder(int n_nodes, int C, int nu, const float* __restrict__ A,
                                                      const float* __restrict__ W, float* __restrict__ out) {
-  constexpr int D = Gen<L>::D, P = Gen<L>::P, K = NodeK<L>::K;
+  constexpr int D = Gen<L>::D, P = Gen<L>::P, K = kNodeK;
   const int groups = C / K;
-  const long long total = static_cast<long long>(n_nodes) * groups;
-  for (long long t = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; t < total;
-       t += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int node = static_cast<int>(t / groups);
-    const int ch = static_cast<int>(t - static_cast<long long>(node) * groups) * K;
-    const float* ar = A + static_cast<size_t>(node) * D * C + ch;
+  // item t = node * groups + channel group; the grid-stride walk advances (node, group) by the
+  // stride's quotient and remainder instead of dividing every item (the launch keeps
+  // n_nodes * groups below 2^31)
+  const int stride = gridDim.x * blockDim.x;
+  const int d_node = stride / groups, d_grp = stride - d_node * groups;
+  const int t0 = blockIdx.x * blockDim.x + threadIdx.x;
+  int node = t0 / groups, grp = t0 - node * groups;
+  // the grid holds only what is resident, so a thread takes several (node, channel-pair) items: the
+  // next item's rows are requested before the current item's products, which hides their latency
+  float an[D][K];
+  if (node < n_nodes) load_item<D, K>(A, C, node, grp * K, an);
+  while (node < n_nodes) {
+    const int ch = grp * K;
+    int next_node = node + d_node, next_grp = grp + d_grp;
+    if (next_grp >= groups) {
+      next_grp -= groups;
+      ++next_node;
+    }
     float a[D][K], b[D][K], o[D][K];
 #pragma unroll
-    for (int c = 0; c < D; ++c) {
-      load_k<K>(ar + c * C, a[c]);
+    for (int c = 0; c < D; ++c)
 #pragma unroll
       for (int k = 0; k < K; ++k) {
-        b[c][k] = a[c][k];
-        o[c][k] = a[c][k];
+        a[c][k] = an[c][k];
+        b[c][k] = an[c][k];
+        o[c][k] = an[c][k];
       }
-    }
+    if (next_node < n_nodes) load_item<D, K>(A, C, next_node, next_grp * K, an);
     for (int q = 0; q + 1 < nu; ++q) {
       const float* wq = W + static_cast<size_t>(q) * P * C + ch;
       float acc[D][K];
@@ -77,11 +98,11 @@ __global__ void __launch_bounds__(256) k_node_ladder(int n_nodes, int C, int nu,
       for (int c = 0; c < D; ++c)
 #pragma unroll
         for (int k = 0; k < K; ++k) acc[c][k] = 0.0f;
-      // (array bound spelled NodeK<L>::K: a generic lambda whose parameter is sized by a local
-      // constexpr of the kernel template crashes the CUDA 12.9 front end)
-      tp_node(IntLN<L>{}, b, a, [&](auto pc, float (&wp)[NodeK<L>::K]) {
+      // (array bound spelled kNodeK: a generic lambda whose parameter is sized by a local constexpr
+      // of the kernel template crashes the CUDA 12.9 front end)
+      tp_node(IntLN<L>{}, b, a, [&](auto pc, float (&wp)[kNodeK]) {
         constexpr int p = decltype(pc)::value;
-        load_k<NodeK<L>::K>(wq + p * C, wp);
+        load_k<kNodeK>(wq + p * C, wp);
       }, acc);
 #pragma unroll
       for (int c = 0; c < D; ++c)
@@ -94,6 +115,8 @@ __global__ void __launch_bounds__(256) k_node_ladder(int n_nodes, int C, int nu,
     float* orow = out + static_cast<size_t>(node) * D * C + ch;
 #pragma unroll
     for (int c = 0; c < D; ++c) store_k<K>(orow + c * C, o[c]);
+    node = next_node;
+    grp = next_grp;
   }
 }
 
@@ -111,10 +134,14 @@ int nnum_sms() {
 template <int L>
 etp_status ladder_launch(int channels, int n_nodes, int nu, const float* A, const float* W, float* out,
                          cudaStream_t s) {
-  constexpr int K = NodeK<L>::K;
-  const long long total = static_cast<long long>(n_nodes) * (channels / K);
+  static int per_sm = 0;
+  if (per_sm == 0) {
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_node_ladder<L>, 256, 0);
+    if (per_sm <= 0) per_sm = 1;
+  }
+  const long long total = static_cast<long long>(n_nodes) * (channels / kNodeK);
   long long blocks = (total + 255) / 256;
-  if (blocks > 32LL * nnum_sms()) blocks = 32LL * nnum_sms();
+  if (blocks > static_cast<long long>(per_sm) * nnum_sms()) blocks = static_cast<long long>(per_sm) * nnum_sms();
   if (blocks < 1) blocks = 1;
   k_node_ladder<L><<<static_cast<int>(blocks), 256, 0, s>>>(n_nodes, channels, nu, A, W, out);
   return cuda_status(cudaGetLastError(), "node ladder launch");
