@@ -84,21 +84,25 @@ def _cg_complex_tensor(l1, l2, l3):
 def cg_real(l1, l2, l3):
     """Real-basis CG tensor C[m1, m2, m3] (indices offset by l), float64.
 
-    C_real[a,b,c] = sum conj(Q1[a,m1]) conj(Q2[b,m2]) Q3[c,m3] C_complex[m1,m2,m3],
-    so that z_c = sum_ab C_real[a,b,c] x_a y_b couples real-basis vectors the
-    way the complex CG couples complex ones. For l1+l2+l3 even the result is
-    real (the only case the parity-restricted irreps use); odd sums give a
-    purely imaginary tensor and are rejected here.
+    With T[a,b,c] = sum conj(Q1[a,m1]) conj(Q2[b,m2]) Q3[c,m3] C_complex[m1,m2,m3], the vector
+    z_c = sum_ab T[a,b,c] x_a y_b couples real-basis vectors the way the complex CG couples
+    complex ones. For l1+l2+l3 even T is real and is returned as it is (the only case that
+    irreps with the harmonics' parity use). For l1+l2+l3 odd T is purely imaginary, T = i T',
+    and the coupling of real vectors is the real tensor T' (the imaginary part), an
+    antisymmetric coupling such as the cross product for 1 x 1 -> 1; its overall sign is a
+    convention that a path weight absorbs.
     """
     if not (abs(l1 - l2) <= l3 <= l1 + l2):
         raise ValueError("triangle rule violated")
-    if (l1 + l2 + l3) % 2:
-        raise ValueError("odd l1+l2+l3 is not used by SH-parity irreps")
     cc = _cg_complex_tensor(l1, l2, l3)
     q1, q2, q3 = real_basis(l1), real_basis(l2), real_basis(l3)
     r = np.einsum("ai,bj,ck,ijk->abc", q1.conj(), q2.conj(), q3, cc)
-    assert np.abs(r.imag).max() < 1e-13, (l1, l2, l3)
-    out = r.real.copy()
+    if (l1 + l2 + l3) % 2 == 0:
+        assert np.abs(r.imag).max() < 1e-13, (l1, l2, l3)
+        out = r.real.copy()
+    else:
+        assert np.abs(r.real).max() < 1e-13, (l1, l2, l3)
+        out = r.imag.copy()
     out[np.abs(out) < 1e-14] = 0.0
     out.setflags(write=False)
     return out

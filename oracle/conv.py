@@ -15,10 +15,16 @@ rows hold rank blocks at offsets off(l), channels contiguous):
 
 "uvu": the output channel equals the input channel; the harmonics have
 multiplicity one. Paths are all (block_in, l2, block_out) with the triangle
-rule and parity p1 (-1)^l2 = p3, in lexicographic (block_in, l2, block_out)
-order ("Fast and Accurate Foundation Models...", section VII: irreps parity
-restricted to that of the harmonics). W has layout [n_basis, n_paths, C].
-Node rows: blocks in irreps order, each block [m][u] (m = -l..l, u contiguous).
+rule, parity p1 (-1)^l2 = p3 and equal multiplicities of the two blocks (the
+channel pairing needs them), in lexicographic (block_in, l2, block_out) order
+("Fast and Accurate Foundation Models...", section VII: irreps parity
+restricted to that of the harmonics is the fast case; NequIP-style per-l
+channel counts of "High-performance training and inference...", Table 1, and
+paths with l1 + l2 + l3 odd are the general one). W has layout
+[n_basis, weight_numel]: path p owns the mul_p columns starting at
+woff_p = sum of the earlier paths' multiplicities ([n_basis, n_paths, C] when
+every block has C channels). Node rows: blocks in irreps order, each block
+[m][u] (m = -l..l, u contiguous).
 
 Vectorised with numpy over edges, one path at a time; the receiver sum is a
 plain scatter-add (np.add.at). No blocking, fusion or reordering beyond that.
@@ -55,21 +61,25 @@ class ConvSpec:
     blocks_in: list = field(init=False)
     blocks_out: list = field(init=False)
     paths: list = field(init=False)
-    channels: int = field(init=False)
+    channels: int = field(init=False)      # the common multiplicity, or None when blocks differ
+    path_mul: list = field(init=False)
+    woff: list = field(init=False)
+    weight_numel: int = field(init=False)  # columns of W (per basis function)
 
     def __post_init__(self):
         self.blocks_in = parse_irreps(self.irreps_in)
         self.blocks_out = parse_irreps(self.irreps_out)
         muls = {b[0] for b in self.blocks_in + self.blocks_out}
-        if len(muls) != 1:
-            raise ValueError("uvu needs one multiplicity for every block")
-        self.channels = muls.pop()
+        self.channels = muls.pop() if len(muls) == 1 else None
         self.paths = []
-        for bi, (_, l1, p1) in enumerate(self.blocks_in):
+        for bi, (m1, l1, p1) in enumerate(self.blocks_in):
             for l2 in range(self.sh_lmax + 1):
-                for bo, (_, l3, p3) in enumerate(self.blocks_out):
-                    if abs(l1 - l2) <= l3 <= l1 + l2 and p1 * (-1) ** l2 == p3:
+                for bo, (m3, l3, p3) in enumerate(self.blocks_out):
+                    if abs(l1 - l2) <= l3 <= l1 + l2 and p1 * (-1) ** l2 == p3 and m1 == m3:
                         self.paths.append((bi, l2, bo))
+        self.path_mul = [self.blocks_in[bi][0] for bi, _, _ in self.paths]
+        self.woff = [int(v) for v in np.cumsum([0] + self.path_mul)[:-1]]
+        self.weight_numel = int(sum(self.path_mul))
 
     @staticmethod
     def _offsets(blocks):
@@ -89,11 +99,15 @@ class ConvSpec:
 
     def in_slice(self, b):
         off = self._offsets(self.blocks_in)[0][b]
-        return slice(off, off + self.channels * (2 * self.blocks_in[b][1] + 1))
+        return slice(off, off + self.blocks_in[b][0] * (2 * self.blocks_in[b][1] + 1))
 
     def out_slice(self, b):
         off = self._offsets(self.blocks_out)[0][b]
-        return slice(off, off + self.channels * (2 * self.blocks_out[b][1] + 1))
+        return slice(off, off + self.blocks_out[b][0] * (2 * self.blocks_out[b][1] + 1))
+
+    def w_slice(self, p):
+        """Columns of W (and of the per-edge weights w) that belong to path p."""
+        return slice(self.woff[p], self.woff[p] + self.path_mul[p])
 
     def path_ls(self, p):
         bi, l2, bo = self.paths[p]
@@ -132,7 +146,7 @@ def _mask_bits(path_mask, n_p):
 def conv_forward(spec, row_ptr, sender, edge_vec, x, W, receivers=None, path_mask=None):
     """out[i] for i in ``receivers`` (default: all). Returns [len(receivers), dim_out].
 
-    x: [N, dim_in]; W: [n_basis, n_paths, C]. Inputs are upcast to float64
+    x: [N, dim_in]; W: [n_basis, weight_numel] (or [n_basis, n_paths, C]). Inputs are upcast to float64
     (complex inputs stay complex, for complex-step checks).
     path_mask: optional per-edge integers (canonical order); path p contributes for edge e only
     when bit p of path_mask[e] is set (per-edge path selection, as in adaptive-depth models).
@@ -143,17 +157,20 @@ def conv_forward(spec, row_ptr, sender, edge_vec, x, W, receivers=None, path_mas
     xs_all = xs_all.astype(np.float64) if xs_all.dtype == np.float32 else xs_all
     W = np.asarray(W, dtype=np.float64)
     vec, d, ys, rad = _edge_geometry(spec, np.asarray(edge_vec)[edges])
-    n_e, c, n_p = len(edges), spec.channels, len(spec.paths)
-    w = (rad @ W.reshape(spec.n_basis, n_p * c)).reshape(n_e, n_p, c)
-    if path_mask is not None:
-        w = w * _mask_bits(np.asarray(path_mask)[edges], n_p)[:, :, None]
+    n_e, n_p = len(edges), len(spec.paths)
+    w = rad @ W.reshape(spec.n_basis, spec.weight_numel)          # [E, weight_numel]
+    mbits = _mask_bits(np.asarray(path_mask)[edges], n_p) if path_mask is not None else None
     dtype = np.result_type(vec, xs_all, np.float64)
     out = np.zeros((len(receivers), spec.dim_out), dtype=dtype)
     for p, (bi, l2, bo) in enumerate(spec.paths):
         l1, _, l3 = spec.path_ls(p)
+        c = spec.path_mul[p]
         cg = cg_real(l1, l2, l3)
+        wp = w[:, spec.w_slice(p)]
+        if mbits is not None:
+            wp = wp * mbits[:, p, None]
         xj = xs_all[sender][:, spec.in_slice(bi)].reshape(n_e, 2 * l1 + 1, c)
-        msg = np.einsum("abc,eb,eau->ecu", cg, ys[l2], xj) * w[:, p, None, :]
+        msg = np.einsum("abc,eb,eau->ecu", cg, ys[l2], xj) * wp[:, None, :]
         blk = np.zeros((len(receivers), 2 * l3 + 1, c), dtype=dtype)
         np.add.at(blk, local, msg)
         out[:, spec.out_slice(bo)] += blk.reshape(len(receivers), -1)
@@ -181,28 +198,30 @@ def conv_vjp(spec, row_ptr, sender, edge_vec, x, W, grad_out, path_mask=None):
     g = np.asarray(grad_out, dtype=np.float64)
     W = np.asarray(W, dtype=np.float64)
     vec, d, ys, rad = _edge_geometry(spec, edge_vec)
-    c, n_p = spec.channels, len(spec.paths)
-    w = (rad @ W.reshape(spec.n_basis, n_p * c)).reshape(n_e, n_p, c)
+    n_p = len(spec.paths)
+    Wf = W.reshape(spec.n_basis, spec.weight_numel)
+    w = rad @ Wf                                                   # [E, weight_numel]
     mbits = _mask_bits(path_mask, n_p) if path_mask is not None else np.ones((n_e, n_p))
-    w = w * mbits[:, :, None]
     grad_x = np.zeros((n_nodes, spec.dim_in))
-    grad_w = np.zeros((n_e, n_p, c))
+    grad_w = np.zeros((n_e, spec.weight_numel))
     grad_y = [np.zeros((n_e, 2 * l + 1)) for l in range(spec.sh_lmax + 1)]
     for p, (bi, l2, bo) in enumerate(spec.paths):
         l1, _, l3 = spec.path_ls(p)
+        c = spec.path_mul[p]
         cg = cg_real(l1, l2, l3)
+        wp = w[:, spec.w_slice(p)] * mbits[:, p, None]
         xj = x[sender][:, spec.in_slice(bi)].reshape(n_e, 2 * l1 + 1, c)
         gi = g[receiver][:, spec.out_slice(bo)].reshape(n_e, 2 * l3 + 1, c)
-        gw = gi * w[:, p, None, :]
+        gw = gi * wp[:, None, :]
         gx_e = np.einsum("abc,eb,ecu->eau", cg, ys[l2], gw)
         blk = np.zeros((n_nodes, 2 * l1 + 1, c))
         np.add.at(blk, sender, gx_e)
         grad_x[:, spec.in_slice(bi)] += blk.reshape(n_nodes, -1)
         s = np.einsum("abc,eb,eau->ecu", cg, ys[l2], xj)
-        grad_w[:, p, :] = (gi * s).sum(axis=1)
+        # a masked path's weight does not reach the output
+        grad_w[:, spec.w_slice(p)] = (gi * s).sum(axis=1) * mbits[:, p, None]
         grad_y[l2] += np.einsum("abc,eau,ecu->eb", cg, xj, gw)
-    grad_w = grad_w * mbits[:, :, None]   # a masked path's weight does not reach the output
-    grad_r = grad_w.reshape(n_e, n_p * c) @ W.reshape(spec.n_basis, n_p * c).T
+    grad_r = grad_w @ Wf.T
     grad_d = (grad_r * radial_deriv(d, spec.n_basis, np.float64(np.float32(spec.r_cut)))).sum(axis=1)
     grad_vec = grad_d[:, None] * vec / d[:, None]
     for l in range(spec.sh_lmax + 1):
@@ -216,7 +235,7 @@ def conv_vjp_weights(spec, row_ptr, sender, edge_vec, x, grad_out):
     The forward is linear in W through w_{e,p,u} = sum_b R_b(d_e) W[b,p,u], so
       dL/dW[b,p,u] = sum_e R_b(d_e) dL/dw_{e,p,u},
       dL/dw_{e,p,u} = sum_m3 g[recv, l3, m3, u] sum_{m1,m2} C[m1,m2,m3] x[send, l1, m1, u] Y_{l2 m2}(e).
-    Returns [n_basis, n_paths, C].
+    Returns [n_basis, n_paths, C] when every block has C channels, else [n_basis, weight_numel].
     """
     row_ptr = np.asarray(row_ptr, dtype=np.int64)
     n_nodes = len(row_ptr) - 1
@@ -226,37 +245,41 @@ def conv_vjp_weights(spec, row_ptr, sender, edge_vec, x, grad_out):
     x = np.asarray(x, dtype=np.float64)
     g = np.asarray(grad_out, dtype=np.float64)
     _, _, ys, rad = _edge_geometry(spec, edge_vec)
-    c, n_p = spec.channels, len(spec.paths)
-    dw_edge = np.zeros((n_e, n_p, c))
+    n_p = len(spec.paths)
+    dw_edge = np.zeros((n_e, spec.weight_numel))
     for p, (bi, l2, bo) in enumerate(spec.paths):
         l1, _, l3 = spec.path_ls(p)
+        c = spec.path_mul[p]
         cg = cg_real(l1, l2, l3)
         xj = x[sender][:, spec.in_slice(bi)].reshape(n_e, 2 * l1 + 1, c)
         gi = g[receiver][:, spec.out_slice(bo)].reshape(n_e, 2 * l3 + 1, c)
         s = np.einsum("abc,eb,eau->ecu", cg, ys[l2], xj)
-        dw_edge[:, p, :] = (gi * s).sum(axis=1)
-    return (rad.T @ dw_edge.reshape(n_e, n_p * c)).reshape(spec.n_basis, n_p, c)
+        dw_edge[:, spec.w_slice(p)] = (gi * s).sum(axis=1)
+    dw = rad.T @ dw_edge
+    return dw.reshape(spec.n_basis, n_p, spec.channels) if spec.channels is not None else dw
 
 
 def flop_counts(spec):
     """Algorithmic operation counts per edge of the plain definition (FMA = 2 flops).
 
-    fwd_tp     : 2 (nnz + sum_p (2 l3 + 1)) C    -- CG contraction with c_k = C_k Y, then w * s
-    radial_proj: 2 n_basis n_paths C             -- w = R W
-    bwd_tp     : 2 (3 nnz + 2 sum_p (2 l3 + 1)) C -- grad_x, grad_w and grad_Y contractions
+    fwd_tp     : sum_p 2 (nnz_p + 2 l3 + 1) mul_p    -- CG contraction with c_k = C_k Y, then w * s
+    radial_proj: 2 n_basis weight_numel              -- w = R W
+    bwd_tp     : sum_p 2 (3 nnz_p + 2 (2 l3 + 1)) mul_p -- grad_x, grad_w and grad_Y contractions
+    (with one multiplicity C for every block: 2 (nnz + sum_p(2 l3 + 1)) C and so on).
     Also returns nnz (real-CG nonzeros over the path set) and sum_2l3p1.
     """
-    nnz = 0
-    s3 = 0
+    nnz = s3 = fwd = bwd = 0
     for p in range(len(spec.paths)):
         l1, l2, l3 = spec.path_ls(p)
-        nnz += int(np.count_nonzero(cg_real(l1, l2, l3)))
+        nz = int(np.count_nonzero(cg_real(l1, l2, l3)))
+        nnz += nz
         s3 += 2 * l3 + 1
-    c, n_p = spec.channels, len(spec.paths)
+        fwd += 2 * (nz + 2 * l3 + 1) * spec.path_mul[p]
+        bwd += 2 * (3 * nz + 2 * (2 * l3 + 1)) * spec.path_mul[p]
     return {
         "nnz": nnz,
         "sum_2l3p1": s3,
-        "fwd_tp": 2 * (nnz + s3) * c,
-        "radial_proj": 2 * spec.n_basis * n_p * c,
-        "bwd_tp": 2 * (3 * nnz + 2 * s3) * c,
+        "fwd_tp": fwd,
+        "radial_proj": 2 * spec.n_basis * spec.weight_numel,
+        "bwd_tp": bwd,
     }
