@@ -318,6 +318,25 @@ def run_gpu(args, rank, world, local_rank):
     for _ in range(3):
         etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out)
     ms_ladder = timed(lambda: etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out), reps, host_ahead=True)
+    # general irreps: NequIP-L channel counts on the same graph (table-driven kernels)
+    gen_irreps = "128x0e+64x1o+32x2e+32x3o"
+    gconv = etp.EdgeConv(gen_irreps, 3, gen_irreps, wl.n_basis, float(wl.r_cut))
+    gi = gconv.info
+    g_x = torch.randn((n, gi["dim_in"]), generator=gen).to(dev)
+    g_W = (torch.randn((gi["n_basis"], gi["weight_numel"] // gi["n_basis"]), generator=gen)
+           / gi["n_paths"] ** 0.5).to(dev)
+    g_g = torch.randn((n, gi["dim_out"]), generator=gen).to(dev)
+    g_ws = torch.empty(max(gconv.workspace_bytes(n, cap), 1), dtype=torch.uint8, device=dev)
+    g_out = torch.empty((n, gi["dim_out"]), device=dev)
+    g_gx = torch.empty((n, gi["dim_in"]), device=dev)
+    g_gv = torch.empty((cap, 3), device=dev)
+    gen_fwd = lambda: gconv.forward(gr, g_x, g_W, out=g_out, workspace=g_ws)
+    gen_bwd = lambda: gconv.backward(gr, g_x, g_W, g_g, grad_x=g_gx, grad_vec=g_gv[:gr.n_edges], workspace=g_ws)
+    for _ in range(3):
+        gen_fwd()
+        gen_bwd()
+    ms_gen_fwd = timed(gen_fwd, reps, host_ahead=True)
+    ms_gen_bwd = timed(gen_bwd, reps, host_ahead=True)
     clocks = sampler.stop() if rank == 0 else None
 
     # end to end through the public API with host buffers (copies inside the timed region)
@@ -338,8 +357,9 @@ def run_gpu(args, rank, world, local_rank):
     d2h = out_h.numel() * 4 + f_h.numel() * 4
 
     e = gr.n_edges
-    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder), total_edges = combine_ranks(
-        [ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder], e, world, dev)
+    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd), total_edges = \
+        combine_ranks([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd], e, world,
+                      dev)
     if rank != 0:
         return None
 
@@ -382,6 +402,14 @@ def run_gpu(args, rank, world, local_rank):
                 "alu_frac": round(flop / (ms * 1e-3) / 1e12 / fp32_peak, 4),
                 "hbm_frac_of_" + peak_kind: round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
 
+    def general_roof(ms, kind):
+        flop = float(gi[f"flop_{kind}"]) * e
+        ach = flop / (ms * 1e-3) / 1e12
+        return {"workload": f"{gen_irreps}, harmonics to l = 3, {wl.name} graph ({e} edges)",
+                "kernel": f"k_gen_{kind}", "ms_per_launch": round(ms, 5), "bound": "alu", "achieved": round(ach, 3),
+                "peak": round(fp32_peak, 2), "unit": "TFLOP/s", "frac": round(ach / fp32_peak, 4),
+                "edges_per_s": round(e / (ms * 1e-3), 1), "traffic": None}
+
     line = {
         "metric": METRIC,
         "value": round(total_edges / (ms_step * 1e-3), 1),
@@ -407,6 +435,8 @@ def run_gpu(args, rank, world, local_rank):
         "ms_weight_grad": round(ms_dw, 5),
         "roofline_weight_grad": roof("dw", ms_dw),
         "node_ladder": ladder_roof(ms_ladder),
+        "general_irreps_fwd": general_roof(ms_gen_fwd, "fwd"),
+        "general_irreps_bwd": general_roof(ms_gen_bwd, "bwd"),
         "e2e": {"value": round(total_edges / (ms_e2e * 1e-3), 1), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step(info, n) * args.steps,

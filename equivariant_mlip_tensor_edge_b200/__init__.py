@@ -28,7 +28,8 @@ class EtpInfo(ctypes.Structure):
     _fields_ = [("lmax", ctypes.c_int), ("channels", ctypes.c_int), ("dim_in", ctypes.c_int),
                 ("dim_out", ctypes.c_int), ("n_paths", ctypes.c_int), ("n_basis", ctypes.c_int),
                 ("weight_numel", ctypes.c_int), ("cg_nnz", ctypes.c_int), ("sum_2l3p1", ctypes.c_int),
-                ("r_cut", ctypes.c_float)]
+                ("r_cut", ctypes.c_float), ("general", ctypes.c_int), ("flop_fwd", ctypes.c_int),
+                ("flop_bwd", ctypes.c_int)]
 
 
 SIGNATURES = {

@@ -102,6 +102,102 @@ bool fill_from_table(Ctx* c, const std::vector<int>& ls) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// The uniform kernels' configuration: C x (0e + 1o + ... + Le) in and out, sh_lmax = L, 1 <= L <= 3,
+// C a multiple of 4 in [4, 256].
+bool uniform_config(const std::vector<Block>& bin, int sh_lmax, const std::vector<Block>& bout) {
+  const int L = static_cast<int>(bin.size()) - 1;
+  if (L < 1 || L > kMaxL || bin.size() != bout.size() || sh_lmax != L) return false;
+  const int C = bin[0].mul;
+  for (int l = 0; l <= L; ++l) {
+    const int par = (l % 2) ? -1 : 1;
+    const Block& a = bin[l];
+    const Block& b = bout[l];
+    if (a.l != l || b.l != l || a.parity != par || b.parity != par || a.mul != C || b.mul != C) return false;
+  }
+  return C % kBatch == 0 && C >= kBatch && C <= 256;
+}
+
+// General irreps: paths (block_in, l2, block_out), lexicographic, with the triangle rule, parity
+// p1 (-1)^l2 = p3 and equal multiplicities (uvu pairs channel u with channel u).
+bool general_config(const std::vector<Block>& bin, int sh_lmax, const std::vector<Block>& bout, float r_cut,
+                    Ctx* c, std::string* why) {
+  if (sh_lmax > etp_gen::kGenLmax) {
+    *why = "sh_lmax above 4";
+    return false;
+  }
+  GenParams& g = c->gen;
+  int lmax = sh_lmax;
+  std::vector<int> in_off, out_off;
+  int off = 0;
+  for (const Block& b : bin) {
+    if (b.l > etp_gen::kGenLmax || b.mul < 1 || b.mul > 1024) {
+      *why = "blocks need 0 <= l <= 4 and 1 <= multiplicity <= 1024";
+      return false;
+    }
+    in_off.push_back(off);
+    off += b.mul * (2 * b.l + 1);
+    lmax = b.l > lmax ? b.l : lmax;
+  }
+  g.dim_in = off;
+  off = 0;
+  for (const Block& b : bout) {
+    if (b.l > etp_gen::kGenLmax || b.mul < 1 || b.mul > 1024) {
+      *why = "blocks need 0 <= l <= 4 and 1 <= multiplicity <= 1024";
+      return false;
+    }
+    out_off.push_back(off);
+    off += b.mul * (2 * b.l + 1);
+    lmax = b.l > lmax ? b.l : lmax;
+  }
+  g.dim_out = off;
+  if (g.dim_in > kGenMaxDim || g.dim_out > kGenMaxDim) {
+    *why = "node rows longer than 4096 floats";
+    return false;
+  }
+  int n = 0, cols = 0, nnz = 0, s3 = 0;
+  for (size_t a = 0; a < bin.size(); ++a)
+    for (int l2 = 0; l2 <= sh_lmax; ++l2)
+      for (size_t b = 0; b < bout.size(); ++b) {
+        const Block& A = bin[a];
+        const Block& B = bout[b];
+        const int sh_par = (l2 % 2) ? -1 : 1;
+        if (!(std::abs(A.l - l2) <= B.l && B.l <= A.l + l2 && A.parity * sh_par == B.parity && A.mul == B.mul))
+          continue;
+        if (n == kGenMaxPaths) {
+          *why = "more than 160 paths";
+          return false;
+        }
+        const int tri = etp_gen::kGenTriId[(A.l * 5 + l2) * 5 + B.l];
+        g.p[n] = GenPath{in_off[a], out_off[b], cols, A.mul, tri};
+        cols += A.mul;
+        nnz += etp_gen::kGenTriNnz[tri];
+        s3 += 2 * B.l + 1;
+        c->flop_fwd += 2 * (etp_gen::kGenTriNnz[tri] + 2 * B.l + 1) * A.mul;
+        c->flop_bwd += 2 * (3 * etp_gen::kGenTriNnz[tri] + 2 * (2 * B.l + 1)) * A.mul;
+        ++n;
+      }
+  if (n == 0) {
+    *why = "no path couples the two irreps";
+    return false;
+  }
+  g.n_paths = n;
+  g.cols = cols;
+  g.sh_lmax = sh_lmax;
+  g.inv_rc = 1.0f / r_cut;
+  int mul = bin[0].mul;
+  for (const Block& b : bin) mul = b.mul == mul ? mul : 0;
+  for (const Block& b : bout) mul = b.mul == mul ? mul : 0;
+  c->general = true;
+  c->lmax = lmax;
+  c->channels = mul;
+  c->dim = g.dim_in;
+  c->n_paths = n;
+  c->cg_nnz = nnz;
+  c->sum_2l3p1 = s3;
+  c->r_cut = r_cut;
+  return true;
+}
+
 }  // namespace
 }  // namespace etp
 
@@ -144,25 +240,23 @@ etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out
     set_error("etp_create: only n_basis == 8 is implemented");
     return ETP_ERR_UNSUPPORTED;
   }
-  const int L = static_cast<int>(bin.size()) - 1;
-  if (L < 1 || L > kMaxL || bin.size() != bout.size() || sh_lmax != L) {
-    set_error("etp_create: need irreps_in == irreps_out == C x (0e..Le), sh_lmax == L, 1 <= L <= 3");
-    return ETP_ERR_UNSUPPORTED;
-  }
-  const int C = bin[0].mul;
-  for (int l = 0; l <= L; ++l) {
-    const int par = (l % 2) ? -1 : 1;
-    const Block& a = bin[l];
-    const Block& b = bout[l];
-    if (a.l != l || b.l != l || a.parity != par || b.parity != par || a.mul != C || b.mul != C) {
-      set_error("etp_create: blocks must be l = 0..L in order, parity (-1)^l, one multiplicity");
+  if (!uniform_config(bin, sh_lmax, bout)) {
+    etp_ctx* h = new (std::nothrow) etp_ctx;
+    if (!h) {
+      set_error("etp_create: out of host memory");
+      return ETP_ERR_INVALID_ARG;
+    }
+    std::string why;
+    if (!general_config(bin, sh_lmax, bout, r_cut, &h->c, &why)) {
+      delete h;
+      set_error("etp_create: unsupported irreps (" + why + ")");
       return ETP_ERR_UNSUPPORTED;
     }
+    *out = h;
+    return ETP_OK;
   }
-  if (C % kBatch != 0 || C < kBatch || C > 256) {
-    set_error("etp_create: channel count must be a multiple of 4 in [4, 256]");
-    return ETP_ERR_UNSUPPORTED;
-  }
+  const int L = static_cast<int>(bin.size()) - 1;
+  const int C = bin[0].mul;
   Ctx c;
   c.lmax = L;
   c.channels = C;
@@ -179,6 +273,8 @@ etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out
     set_error("etp_create: out of host memory");
     return ETP_ERR_INVALID_ARG;
   }
+  c.flop_fwd = 2 * (c.cg_nnz + c.sum_2l3p1) * C;
+  c.flop_bwd = 2 * (3 * c.cg_nnz + 2 * c.sum_2l3p1) * C;
   h->c = c;
   *out = h;
   return ETP_OK;
@@ -198,13 +294,16 @@ etp_status etp_get_info(etp_handle h, etp_info_t* info) {
   info->lmax = c.lmax;
   info->channels = c.channels;
   info->dim_in = c.dim;
-  info->dim_out = c.dim;
+  info->dim_out = c.general ? c.gen.dim_out : c.dim;
   info->n_paths = c.n_paths;
   info->n_basis = kNumBasis;
-  info->weight_numel = kNumBasis * c.n_paths * c.channels;
+  info->weight_numel = kNumBasis * (c.general ? c.gen.cols : c.n_paths * c.channels);
   info->cg_nnz = c.cg_nnz;
   info->sum_2l3p1 = c.sum_2l3p1;
   info->r_cut = c.r_cut;
+  info->general = c.general ? 1 : 0;
+  info->flop_fwd = c.flop_fwd;
+  info->flop_bwd = c.flop_bwd;
   return ETP_OK;
 }
 
@@ -218,6 +317,7 @@ static size_t ws_tc_offset(int n_edges) {
 
 size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   if (!h || n_edges < 0 || n_nodes < 0) return 0;
+  if (h->c.general) return ws_tc_offset(n_edges);   // receiver of each edge + validation scratch
   const size_t f = tc::forward_tc_workspace_bytes(h->c, n_nodes);
   const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
   const size_t w = weight_grad_workspace_bytes(h->c, n_edges);
@@ -258,7 +358,8 @@ static etp_status check_common(etp_handle h, int n_nodes, int n_edges, const int
     set_error(std::string(who) + ": negative size");
     return ETP_ERR_INVALID_ARG;
   }
-  if (static_cast<long long>(n_nodes) * h->c.dim >= (1LL << 31)) {
+  const int dmax = h->c.general && h->c.gen.dim_out > h->c.dim ? h->c.gen.dim_out : h->c.dim;
+  if (static_cast<long long>(n_nodes) * dmax >= (1LL << 31)) {
     set_error(std::string(who) + ": n_nodes * dim must stay below 2^31");
     return ETP_ERR_UNSUPPORTED;
   }
@@ -298,6 +399,8 @@ etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_pt
     if (st != ETP_OK) return st;
   }
   if (n_nodes == 0) return ETP_OK;
+  if (h->c.general)
+    return launch_general_forward(h->c.gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, s);
   if (use_tc_forward()) {
     if (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges)) {
       set_error("etp_forward: workspace missing or smaller than etp_workspace_bytes()");
@@ -343,6 +446,9 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
     if (st != ETP_OK) return st;
   }
   if (n_nodes == 0) return ETP_OK;
+  if (h->c.general)
+    return launch_general_backward(h->c.gen, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W,
+                                   grad_out, grad_x, grad_edge_vec, recv_map, s);
   if (n_edges > 0 && use_tc_backward()) {
     void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
     st = tc::launch_backward_tc(h->c, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W, grad_out,
@@ -360,6 +466,10 @@ etp_status etp_forward_masked(etp_handle h, int n_nodes, int n_edges, const int*
                               size_t workspace_bytes, void* stream) {
   etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_forward_masked");
   if (st != ETP_OK) return st;
+  if (h->c.general) {
+    set_error("etp_forward_masked: not implemented for general irreps handles");
+    return ETP_ERR_UNSUPPORTED;
+  }
   if (!out || !aligned16(out) || (n_edges > 0 && !path_mask)) {
     set_error("etp_forward_masked: out (16-byte aligned) and path_mask must be device pointers");
     return ETP_ERR_INVALID_ARG;
@@ -390,6 +500,10 @@ etp_status etp_backward_masked(etp_handle h, int n_nodes, int n_edges, const int
                                void* stream) {
   etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_backward_masked");
   if (st != ETP_OK) return st;
+  if (h->c.general) {
+    set_error("etp_backward_masked: not implemented for general irreps handles");
+    return ETP_ERR_UNSUPPORTED;
+  }
   if (!t_row_ptr || (n_edges > 0 && (!t_perm || !grad_out || !path_mask)) || (!grad_x && !grad_edge_vec)) {
     set_error("etp_backward_masked: NULL array (grad_x and grad_edge_vec may not both be NULL)");
     return ETP_ERR_INVALID_ARG;
@@ -426,6 +540,10 @@ etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const in
   if (!h) {
     set_error("etp_backward_weights: NULL handle");
     return ETP_ERR_INVALID_ARG;
+  }
+  if (h->c.general) {
+    set_error("etp_backward_weights: not implemented for general irreps handles");
+    return ETP_ERR_UNSUPPORTED;
   }
   if (n_nodes < 0 || n_edges < 0) {
     set_error("etp_backward_weights: negative size");
@@ -489,6 +607,10 @@ etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, 
   if (!h || n_edges < 0 || (n_edges > 0 && (!edge_vec || !W || !w_out))) {
     set_error("etp_radial_weights: bad argument");
     return ETP_ERR_INVALID_ARG;
+  }
+  if (h->c.general) {
+    set_error("etp_radial_weights: not implemented for general irreps handles");
+    return ETP_ERR_UNSUPPORTED;
   }
   if (n_edges == 0) return ETP_OK;
   return launch_radial_weights(h->c, n_edges, edge_vec, W, w_out, static_cast<cudaStream_t>(stream));

@@ -14,14 +14,36 @@ constexpr int kNumBasis = 8;     // radial basis functions (fixed at compile tim
 constexpr int kBatch = 4;        // channels per register batch (one float4 per component)
 constexpr int kMaxL = 3;
 
+// General irreps (any multiplicities and parities, rank <= 4): the path table the kernels read
+// from their parameter block. Path p couples input block component rows starting at in_off with
+// the harmonics of rank l2 into the output block at out_off, over mul channels, with weight
+// columns woff .. woff + mul - 1; tri is the coupling index of (l1, l2, l3).
+constexpr int kGenMaxPaths = 160;
+struct GenPath {
+  int in_off, out_off, woff, mul, tri;
+};
+struct GenParams {
+  int n_paths = 0;
+  int dim_in = 0;
+  int dim_out = 0;
+  int cols = 0;        // weight columns per basis function (sum of the paths' multiplicities)
+  int sh_lmax = 0;
+  float inv_rc = 0.f;
+  GenPath p[kGenMaxPaths];
+};
+
 struct Ctx {
   int lmax = 0;
-  int channels = 0;
-  int dim = 0;
+  int channels = 0;    // the common multiplicity (0 for a general handle whose blocks differ)
+  int dim = 0;         // dim_in (= dim_out for the uniform kernels)
   int n_paths = 0;
   int cg_nnz = 0;
   int sum_2l3p1 = 0;
   float r_cut = 0.f;
+  int flop_fwd = 0;       // FP32 flop per edge of the forward / backward contraction
+  int flop_bwd = 0;
+  bool general = false;   // true: the table-driven kernels of etp_general.cu serve this handle
+  GenParams gen;
 };
 
 // Configuration behind a handle (NULL for a NULL handle).
@@ -85,6 +107,16 @@ size_t weight_grad_workspace_bytes(const Ctx& c, int n_edges);
 etp_status launch_weight_grad(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                               const float* edge_vec, const float* x, const float* grad_out, float* grad_W,
                               int* recv, void* ws, cudaStream_t s);
+
+// ---- general irreps (etp_general.cu); recv: n_edges ints of scratch
+constexpr int kGenMaxDim = 4096;   // floats per node row (the kernels keep one row per warp in shared memory)
+etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
+                                  const int* sender, const float* edge_vec, const float* x, const float* W,
+                                  float* out, cudaStream_t s);
+etp_status launch_general_backward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
+                                   const float* edge_vec, const int* t_row_ptr, const int* t_perm,
+                                   const float* x, const float* W, const float* grad_out, float* grad_x,
+                                   float* grad_edge_vec, int* recv, cudaStream_t s);
 
 // ---- node-local product ladder (etp_product.cu)
 etp_status launch_node_ladder(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,

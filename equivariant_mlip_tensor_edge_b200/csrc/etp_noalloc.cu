@@ -74,6 +74,14 @@ extern "C" etp_status etp_forward_noalloc(etp_handle h, int n_nodes, int n_edges
     set_error("etp_forward_noalloc: x, W and out must be 16-byte aligned");
     return ETP_ERR_INVALID_ARG;
   }
+  if (c->general) {   // the general kernels need no scratch at all
+    if (static_cast<long long>(n_nodes) * c->gen.dim_out >= (1LL << 31)) {
+      set_error("etp_forward_noalloc: n_nodes * dim must stay below 2^31");
+      return ETP_ERR_UNSUPPORTED;
+    }
+    return etp::launch_general_forward(c->gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out,
+                                       static_cast<cudaStream_t>(stream));
+  }
   const size_t need = etp::tc::forward_tc_workspace_bytes(*c, n_nodes);
   if (need > etp::kScratchBytes) {
     set_error("etp_forward_noalloc: this handle needs " + std::to_string(need) +

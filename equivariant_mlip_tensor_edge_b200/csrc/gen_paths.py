@@ -8,7 +8,11 @@ Emits, for every supported l_max (in = SH = out = L):
   * per path, the real-basis Clebsch-Gordan nonzeros as float immediates inside
     straight-line forward and backward contraction code, and the per-path factor
     of the weight gradient, sum_{m1,m3} x[l1 m1] (sum_m2 C Y[l2 m2]) g[l3 m3];
-  * the node-local path-reduced product of two feature rows (tp_node_L).
+  * the node-local path-reduced product of two feature rows (tp_node_L);
+  * for general irreps (any multiplicities and parities, rank <= 4), one forward and one
+    backward contraction per coupling (l1, l2, l3), even and odd l1 + l2 + l3, over one
+    channel with the block stride as an argument, dispatched by a coupling index; and the
+    harmonics up to l = 4.
 
 Independent of the float64 oracle by construction: Clebsch-Gordan values come
 from ``sympy.physics.wigner.clebsch_gordan`` and the harmonic polynomials from a
@@ -60,6 +64,28 @@ def real_cg(l1, l2, l3):
     r = np.einsum("ai,bj,ck,ijk->abc", u1.conj(), u2.conj(), u3, c)
     assert np.abs(r.imag).max() < 1e-12
     r = r.real
+    r[np.abs(r) < 1e-12] = 0.0
+    return r
+
+
+def real_cg_any(l1, l2, l3):
+    """Real coupling for any triangle triple: the real tensor for l1 + l2 + l3 even; for odd sums
+    the change of basis gives i times a real tensor, and that real tensor is the coupling."""
+    c = np.zeros((2 * l1 + 1, 2 * l2 + 1, 2 * l3 + 1), dtype=complex)
+    for m1 in range(-l1, l1 + 1):
+        for m2 in range(-l2, l2 + 1):
+            m3 = m1 + m2
+            if abs(m3) <= l3:
+                c[m1 + l1, m2 + l2, m3 + l3] = float(sym_n(clebsch_gordan(l1, l2, l3, m1, m2, m3), 30))
+    u1, u2, u3 = complex_to_real(l1), complex_to_real(l2), complex_to_real(l3)
+    r = np.einsum("ai,bj,ck,ijk->abc", u1.conj(), u2.conj(), u3, c)
+    if (l1 + l2 + l3) % 2 == 0:
+        assert np.abs(r.imag).max() < 1e-12
+        r = r.real
+    else:
+        assert np.abs(r.real).max() < 1e-12
+        r = r.imag
+    r = r.copy()
     r[np.abs(r) < 1e-12] = 0.0
     return r
 
@@ -503,6 +529,98 @@ def emit_cm(out, lmax):
             out.append("}")
 
 
+# ---------------------------------------------------------------- general irreps
+
+GEN_LMAX = 4
+
+
+def gen_triples():
+    return [(a, b, c) for a in range(GEN_LMAX + 1) for b in range(GEN_LMAX + 1)
+            for c in range(abs(a - b), min(GEN_LMAX, a + b) + 1)]
+
+
+def emit_general(out):
+    """Per coupling t = (l1, l2, l3): gfwd_t adds w sum C Y x into acc[m3 * stride] and gbwd_t
+    accumulates grad_x, dL/dY and dL/dw for one channel. x, g and acc point at the channel's
+    element of component 0 of their block; components are `stride` floats apart."""
+    tri = gen_triples()
+    out.append(f"constexpr int kGenLmax = {GEN_LMAX};")
+    out.append(f"constexpr int kGenTriples = {len(tri)};")
+    ids = [[[-1] * (GEN_LMAX + 1) for _ in range(GEN_LMAX + 1)] for _ in range(GEN_LMAX + 1)]
+    for t, (a, b, c) in enumerate(tri):
+        ids[a][b][c] = t
+    flat = [ids[a][b][c] for a in range(GEN_LMAX + 1) for b in range(GEN_LMAX + 1) for c in range(GEN_LMAX + 1)]
+    out.append("// coupling index of (l1, l2, l3) at [(l1 * 5 + l2) * 5 + l3], -1 outside the triangle rule")
+    out.append("constexpr int kGenTriId[] = {" + ", ".join(map(str, flat)) + "};")
+    nnz = [int(np.count_nonzero(real_cg_any(*t))) for t in tri]
+    out.append("constexpr int kGenTriNnz[] = {" + ", ".join(map(str, nnz)) + "};")
+    for t, (l1, l2, l3) in enumerate(tri):
+        c = real_cg_any(l1, l2, l3)
+        groups = []   # (m3, m1, [(coef, y index)])
+        for m3 in range(2 * l3 + 1):
+            for m1 in range(2 * l1 + 1):
+                terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
+                if terms:
+                    groups.append((m3, m1, terms))
+        # forward
+        out.append(f"// ({l1},{l2},{l3})")
+        out.append(f"__device__ __forceinline__ void gfwd_{t}(const float* __restrict__ x, int stride, const float* Y,")
+        out.append("                                       float w, float* acc) {")
+        for m1 in range(2 * l1 + 1):
+            out.append(f"  const float x{m1} = x[{m1} * stride];")
+        for m3 in range(2 * l3 + 1):
+            row = [(m1, terms) for (a3, m1, terms) in groups if a3 == m3]
+            if not row:
+                continue
+            first = True
+            for m1, terms in row:
+                mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                if first:
+                    out.append(f"  float s{m3} = ({mexpr}) * x{m1};")
+                    first = False
+                else:
+                    out.append(f"  s{m3} = fmaf({mexpr}, x{m1}, s{m3});")
+            out.append(f"  acc[{m3} * stride] = fmaf(w, s{m3}, acc[{m3} * stride]);")
+        out.append("}")
+        # backward
+        out.append(f"__device__ __forceinline__ void gbwd_{t}(const float* __restrict__ x, const float* __restrict__ g,")
+        out.append("                                       int stride, const float* Y, float w, float* gx, float* gY,")
+        out.append("                                       float& gw) {")
+        for m1 in range(2 * l1 + 1):
+            out.append(f"  const float x{m1} = x[{m1} * stride];")
+            out.append(f"  float a{m1} = 0.0f;")
+        for m3 in range(2 * l3 + 1):
+            out.append(f"  const float g{m3} = g[{m3} * stride];")
+        for m3, m1, terms in groups:
+            mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+            out.append(f"  {{ const float mv = {mexpr};")
+            out.append(f"    a{m1} = fmaf(mv, g{m3}, a{m1});")
+            out.append(f"    const float xg = x{m1} * g{m3};")
+            out.append("    gw = fmaf(mv, xg, gw);")
+            for v, i in terms:
+                out.append(f"    gY[{i}] = fmaf({repr_f32(np.float32(v))} * w, xg, gY[{i}]);")
+            out.append("  }")
+        for m1 in range(2 * l1 + 1):
+            out.append(f"  gx[{m1} * stride] = fmaf(w, a{m1}, gx[{m1} * stride]);")
+        out.append("}")
+    out.append("__device__ __forceinline__ void gen_fwd(int t, const float* x, int stride, const float* Y, float w,")
+    out.append("                                        float* acc) {")
+    out.append("  switch (t) {")
+    for t in range(len(tri)):
+        out.append(f"    case {t}: gfwd_{t}(x, stride, Y, w, acc); break;")
+    out.append("    default: break;")
+    out.append("  }")
+    out.append("}")
+    out.append("__device__ __forceinline__ void gen_bwd(int t, const float* x, const float* g, int stride, const float* Y,")
+    out.append("                                        float w, float* gx, float* gY, float& gw) {")
+    out.append("  switch (t) {")
+    for t in range(len(tri)):
+        out.append(f"    case {t}: gbwd_{t}(x, g, stride, Y, w, gx, gY, gw); break;")
+    out.append("    default: break;")
+    out.append("  }")
+    out.append("}")
+
+
 def generate():
     out = ["// GENERATED by gen_paths.py -- do not edit.",
            "// Real-basis Clebsch-Gordan contractions and real spherical harmonics, unrolled per path.",
@@ -534,6 +652,8 @@ def generate():
         emit_cm(out, lmax)
     for lmax in LMAX_SUPPORTED:
         emit_node(out, lmax)
+    emit_sh(out, GEN_LMAX)
+    emit_general(out)
     out.append("}  // namespace etp_gen")
     return "\n".join(out) + "\n"
 

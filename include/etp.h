@@ -77,14 +77,30 @@ typedef struct {
   int cg_nnz;        /* real-CG nonzeros summed over the path set */
   int sum_2l3p1;     /* sum over paths of 2 l3 + 1 */
   float r_cut;
+  int general;       /* 1: general irreps handle (table-driven kernels), 0: uniform kernels */
+  int flop_fwd;      /* FP32 flop per edge of the forward contraction: sum_p 2 (nnz_p + 2 l3 + 1) mul_p */
+  int flop_bwd;      /* the same for the backward: sum_p 2 (3 nnz_p + 2 (2 l3 + 1)) mul_p */
 } etp_info_t;
 
 /* Create a convolution handle. Host-only, synchronous, allocates host memory only.
- * irreps_in / irreps_out: "CxL1p+CxL2p+..." strings, e.g. "64x0e+64x1o+64x2e".
- * Supported: every block has the same multiplicity C (C % 4 == 0, 4 <= C <= 256), blocks are
- * l = 0..L in order with parity (-1)^l, irreps_out == irreps_in, sh_lmax == L, L in {1,2,3},
- * n_basis == 8, r_cut > 0. Malformed strings -> ETP_ERR_IRREPS; anything else outside the
- * supported set -> ETP_ERR_UNSUPPORTED. The path list is the enumeration described above. */
+ * irreps_in / irreps_out: "mulxLp+mulxLp+..." strings, e.g. "64x0e+64x1o+64x2e".
+ * Two kinds of handle, chosen here:
+ *  - uniform (the tensor-core kernels): every block has the same multiplicity C (C % 4 == 0,
+ *    4 <= C <= 256), blocks are l = 0..L in order with parity (-1)^l, irreps_out == irreps_in,
+ *    sh_lmax == L, L in {1,2,3};
+ *  - general (table-driven FP32 kernels, info.general = 1): any blocks with 0 <= l <= 4 and
+ *    1 <= mul <= 1024 in any order and either parity, sh_lmax <= 4, node rows of at most 4096
+ *    floats, 1 to 160 paths. Paths join blocks of EQUAL multiplicity only (uvu: channel u to
+ *    channel u), so irreps like NequIP's 128x0e+64x1o+32x2e+32x3o couple 2e with 3o but not 1o
+ *    with 2e. Paths with l1 + l2 + l3 odd use the real antisymmetric coupling (the imaginary
+ *    part of the complex-to-real transformed Clebsch-Gordan tensor; the cross product for
+ *    1 x 1 -> 1). W is [n_basis][cols] with path p's mul_p columns after the earlier paths'
+ *    (the same as [n_basis][n_paths][C] when all blocks have C channels); node rows hold the
+ *    blocks in string order, block b as [m][u] with mul_b channels. General handles support
+ *    etp_forward, etp_forward_noalloc (no scratch needed) and etp_backward; the masked, weight
+ *    gradient and radial-weight calls return ETP_ERR_UNSUPPORTED for them.
+ * Both need n_basis == 8 and r_cut > 0. Malformed strings -> ETP_ERR_IRREPS; anything else
+ * outside these sets -> ETP_ERR_UNSUPPORTED. The path list is the enumeration described above. */
 etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_basis,
                       float r_cut, etp_handle* out);
 

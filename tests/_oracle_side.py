@@ -85,3 +85,19 @@ def assert_close_rel(gpu, ref, what, tol=TOL):
 
 __all__ = ["TOL", "spec_of", "full_graph", "given_graph", "rows_subgraph", "sampled_rows", "sender_edges",
            "forward_ref", "block_errors", "assert_blocks_close", "assert_close_rel", "conv_vjp"]
+
+
+def assert_irrep_blocks_close(gpu, ref, spec, side, what, tol=TOL):
+    """Per irrep block of a general spec (side: 'in' or 'out'), the same bound as above."""
+    blocks = spec.blocks_in if side == "in" else spec.blocks_out
+    sl_of = spec.in_slice if side == "in" else spec.out_slice
+    gpu = np.asarray(gpu, np.float64)
+    for b, (mul, l, par) in enumerate(blocks):
+        sl = sl_of(b)
+        err = float(np.abs(gpu[:, sl] - ref[:, sl]).max()) if ref.size else 0.0
+        scale = float(np.abs(ref[:, sl]).max()) if ref.size else 0.0
+        assert err <= tol * scale, f"{what}: block {mul}x{l}{'e' if par > 0 else 'o'} max|err|={err:.3e} > " \
+                                   f"{tol:g} * max|ref|={scale:.3e}"
+
+
+__all__.append("assert_irrep_blocks_close")

@@ -47,12 +47,18 @@ def test_create_status_codes():
     assert _create("64x0e+64x1q", 1, "64x0e+64x1o") == 2        # malformed
     assert _create("64x0e++64x1o", 1, "64x0e+64x1o") == 2
     assert _create(None, 1, "64x0e+64x1o") == 2
-    assert _create("64x0e+64x1e", 1, "64x0e+64x1e") == 3        # parity not (-1)^l
-    assert _create("64x0e+32x1o", 1, "64x0e+32x1o") == 3        # mixed multiplicity
-    assert _create("6x0e+6x1o", 1, "6x0e+6x1o") == 3            # C % 4 != 0
+    # general handles (table-driven kernels)
+    assert _create("64x0e+64x1e", 1, "64x0e+64x1e") == 0        # parity not (-1)^l
+    assert _create("64x0e+32x1o", 1, "64x0e+32x1o") == 0        # mixed multiplicity
+    assert _create("6x0e+6x1o", 1, "6x0e+6x1o") == 0            # C % 4 != 0
+    assert _create("8x0e+8x1o", 2, "8x0e+8x1o") == 0            # sh_lmax != L
+    assert _create("8x0e+8x1o+8x2e+8x3o+8x4e", 4, "8x0e+8x1o+8x2e+8x3o+8x4e") == 0
+    # outside both
     assert _create("8x0e+8x1o", 1, "8x0e+8x1o", nb=6) == 3      # n_basis != 8
-    assert _create("8x0e+8x1o", 2, "8x0e+8x1o") == 3            # sh_lmax != L
-    assert _create("8x0e+8x1o+8x2e+8x3o+8x4e", 4, "8x0e+8x1o+8x2e+8x3o+8x4e") == 3
+    assert _create("8x0e+8x5o", 1, "8x0e+8x5o") == 3            # l > 4
+    assert _create("8x0e+8x1o", 5, "8x0e+8x1o") == 3            # sh_lmax > 4
+    assert _create("8x0e", 0, "4x0e") == 3                      # no path (multiplicities differ)
+    assert _create("1024x0e+1024x1o+1024x2e", 2, "1024x0e+1024x1o+1024x2e") == 3   # rows above 4096 floats
     assert _create("8x0e+8x1o", 1, "8x0e+8x1o", rc=-1.0) == 1
 
 
@@ -67,14 +73,36 @@ def test_info_matches_independent_path_enumeration(lmax, c):
     assert conv.info["sum_2l3p1"] == fc["sum_2l3p1"]
     assert conv.info["dim_in"] == spec.dim_in == conv.info["dim_out"]
     assert conv.info["weight_numel"] == 8 * len(spec.paths) * c
+    assert conv.info["flop_fwd"] == fc["fwd_tp"] and conv.info["flop_bwd"] == fc["bwd_tp"]
     assert conv.workspace_bytes(100, 1000) >= 2 * 4 * 1000
+
+
+@pytest.mark.parametrize("irin,sh,irout", [
+    ("4x0e+3x1o+3x1e+4x2e+2x2o+3x3o+4x4e", 4, "4x0e+3x1o+3x1e+4x2e+2x2o+3x3o+4x4e"),
+    ("128x0e+64x1o+32x2e+32x3o", 3, "128x0e+64x1o+32x2e+32x3o"),
+    ("16x0e+16x1o", 2, "16x0e+16x1o+16x1e+16x2e"),
+    ("6x0e+6x1o+6x2e", 2, "6x0e+6x1o+6x2e"),
+])
+def test_general_info_matches_independent_path_enumeration(irin, sh, irout):
+    conv = etp.EdgeConv(irin, sh, irout, 8, 5.0)
+    spec = ConvSpec(irin, sh, irout, 8, 5.0)
+    fc = flop_counts(spec)
+    assert conv.info["general"] == 1
+    assert conv.info["n_paths"] == len(spec.paths)
+    assert conv.info["cg_nnz"] == fc["nnz"]
+    assert conv.info["sum_2l3p1"] == fc["sum_2l3p1"]
+    assert conv.info["dim_in"] == spec.dim_in and conv.info["dim_out"] == spec.dim_out
+    assert conv.info["weight_numel"] == 8 * spec.weight_numel
+    assert conv.info["channels"] == (spec.channels or 0)
+    assert conv.info["flop_fwd"] == fc["fwd_tp"] and conv.info["flop_bwd"] == fc["bwd_tp"]
+    assert etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x1o", 8, 5.0).info["general"] == 0
 
 
 def test_status_strings_and_errors(lib):
     for s in range(7):
         assert lib.etp_status_string(s)
     with pytest.raises(etp.EtpError) as ei:
-        etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x2o", 8, 5.0)
+        etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x5o", 8, 5.0)
     assert ei.value.status == 3
     assert "etp_create" in str(ei.value)
 

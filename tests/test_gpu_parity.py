@@ -15,8 +15,9 @@ import workloads
 from oracle.conv import conv_forward, conv_vjp
 from oracle.graph import forces_from_edge_grads
 from oracle.radial import radial
-from tests._oracle_side import (assert_blocks_close, assert_close_rel, forward_ref, full_graph, given_graph,
-                                rows_subgraph, sampled_rows, sender_edges, spec_of)
+from oracle.conv import ConvSpec
+from tests._oracle_side import (assert_blocks_close, assert_close_rel, assert_irrep_blocks_close, forward_ref,
+                                full_graph, given_graph, rows_subgraph, sampled_rows, sender_edges, spec_of)
 
 torch = pytest.importorskip("torch")
 etp = pytest.importorskip("equivariant_mlip_tensor_edge_b200")
@@ -662,3 +663,96 @@ def test_node_ladder_parity(lmax, c, n, nu):
     out = etp.node_ladder(torch.from_numpy(A).to(DEV), torch.from_numpy(Ws).to(DEV), lmax)
     ref = node_ladder(lmax, c, A, Ws)
     assert_blocks_close(_np(out), ref, c, lmax, f"node ladder lmax={lmax} C={c} nu={nu}")
+
+
+# ------------------------------------------------------------------ general irreps
+
+GENERAL = [
+    ("128x0e+64x1o+32x2e+32x3o", 3, "128x0e+64x1o+32x2e+32x3o"),        # NequIP-L channel counts
+    ("4x0e+3x1o+3x1e+4x2e+2x2o+3x3o+4x4e", 4, "4x0e+3x1o+3x1e+4x2e+2x2o+3x3o+4x4e"),
+    ("16x0e+16x1o+16x1e+16x2e+16x2o", 2, "16x0e+16x1o+16x1e+16x2e+16x2o"),   # odd l1 + l2 + l3 paths
+    ("32x0e+32x1o+32x2e+32x3o+32x4e", 4, "32x0e+32x1o+32x2e+32x3o+32x4e"),   # rank 4
+    ("16x0e+16x1o", 2, "16x0e+16x1o+16x1e+16x2e"),                         # irreps_out != irreps_in
+    ("6x0e+6x1o+6x2e", 2, "6x0e+6x1o+6x2e"),                               # C not a multiple of 4
+]
+
+
+def _general_inputs(spec, n, seed):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((n, spec.dim_in)).astype(np.float32)
+    W = (rng.standard_normal((8, spec.weight_numel)) / np.sqrt(len(spec.paths))).astype(np.float32)
+    gout = rng.standard_normal((n, spec.dim_out)).astype(np.float32)
+    return x, W, gout
+
+
+@pytest.mark.parametrize("irin,sh,irout", GENERAL)
+def test_general_irreps_parity_full(wls, irin, sh, irout):
+    """Forward and backward of general irreps handles against the oracle on the whole small cell."""
+    wl = wls("tiny")
+    conv = etp.EdgeConv(irin, sh, irout, 8, float(wl.r_cut))
+    assert conv.info["general"] == 1
+    spec = ConvSpec(irin, sh, irout, 8, float(wl.r_cut))
+    x, W, gout = _general_inputs(spec, wl.n_nodes, len(irin) + sh)
+    g = _gpu_graph(wl)
+    ref_g = full_graph(wl)
+    xd, Wd, gd = (torch.from_numpy(a).to(DEV) for a in (x, W, gout))
+    out = conv.forward(g, xd, Wd)
+    ref = conv_forward(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W)
+    assert_irrep_blocks_close(_np(out), ref, spec, "out", f"{irin} forward")
+    gx, gv = conv.backward(g, xd, Wd, gd)
+    rgx, rgv = conv_vjp(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, gout)
+    assert_irrep_blocks_close(_np(gx), rgx, spec, "in", f"{irin} grad_x")
+    assert_close_rel(_np(gv), rgv, f"{irin} grad_edge_vec")
+    # the no-workspace entry point runs the same kernel
+    out2 = torch.empty_like(out)
+    st = etp.load_library().etp_forward_noalloc(conv._h, g.n_nodes, g.n_edges, etp._ptr(g.row_ptr),
+                                                etp._ptr(g.sender), etp._ptr(g.edge_vec), etp._ptr(xd),
+                                                etp._ptr(Wd), etp._ptr(out2), etp._stream(xd.device))
+    assert st == 0 and torch.equal(out2, out)
+    # deterministic
+    assert torch.equal(conv.forward(g, xd, Wd), out)
+
+
+def test_general_irreps_parity_sampled_full_size(wls):
+    """NequIP-L channel counts (128x0e+64x1o+32x2e+32x3o, harmonics to l = 3) on the 1000-atom
+    diamond cell: sampled receivers (forward) and senders (backward), computed one by one."""
+    wl = wls("diamond1k")
+    irr = "128x0e+64x1o+32x2e+32x3o"
+    conv = etp.EdgeConv(irr, 3, irr, 8, float(wl.r_cut))
+    spec = ConvSpec(irr, 3, irr, 8, float(wl.r_cut))
+    x, W, gout = _general_inputs(spec, wl.n_nodes, 77)
+    g = _gpu_graph(wl)
+    xd, Wd, gd = (torch.from_numpy(a).to(DEV) for a in (x, W, gout))
+    out = _np(conv.forward(g, xd, Wd))
+    rng = np.random.default_rng(17)
+    sample = np.sort(rng.choice(wl.n_nodes, size=N_SAMPLE // 2, replace=False))
+    ref, _ = forward_ref(wl, spec, x, W, sample=sample)
+    assert_irrep_blocks_close(out[sample], ref, spec, "out", "NequIP-L forward (sampled)")
+    gx, gv = conv.backward(g, xd, Wd, gd)
+    gx, gv = _np(gx), _np(gv)
+    rows = sampled_rows(wl, sample)
+    recv, send, shift, vec = sender_edges(rows)
+    rp, snd, v = rows_subgraph(wl.n_nodes, recv, send, vec)
+    rgx, rgv = conv_vjp(spec, rp, snd, v, x, W, gout)
+    assert_irrep_blocks_close(gx[sample], rgx[sample], spec, "in", "NequIP-L grad_x (sampled)")
+    keys = _edge_keys(_gpu_receivers(g), _np(g.sender), _np(g.shift), wl.n_nodes)
+    want = _edge_keys(recv, send, shift, wl.n_nodes)
+    pos = np.searchsorted(keys, want)
+    assert np.array_equal(keys[pos], want)
+    assert_close_rel(gv[pos], rgv, "NequIP-L grad_edge_vec (sampled)")
+
+
+def test_general_irreps_unsupported_calls_refuse(wls):
+    wl = wls("tiny")
+    conv = etp.EdgeConv("8x0e+8x1e", 1, "8x0e+8x1e", 8, float(wl.r_cut))
+    spec = ConvSpec("8x0e+8x1e", 1, "8x0e+8x1e", 8, float(wl.r_cut))
+    x, W, gout = _general_inputs(spec, wl.n_nodes, 5)
+    g = _gpu_graph(wl)
+    xd, Wd, gd = (torch.from_numpy(a).to(DEV) for a in (x, W, gout))
+    with pytest.raises(etp.EtpError) as ei:
+        conv.backward_weights(g, xd, gd)
+    assert ei.value.status == 3
+    mask = torch.ones(g.n_edges, dtype=torch.int32, device=DEV)
+    with pytest.raises(etp.EtpError) as ei:
+        conv.forward(g, xd, Wd, path_mask=mask)
+    assert ei.value.status == 3
