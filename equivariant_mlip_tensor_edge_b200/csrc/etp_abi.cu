@@ -125,6 +125,10 @@ bool general_config(const std::vector<Block>& bin, int sh_lmax, const std::vecto
     *why = "sh_lmax above 4";
     return false;
   }
+  if (bin.size() > static_cast<size_t>(kGenMaxBlocks) || bout.size() > static_cast<size_t>(kGenMaxBlocks)) {
+    *why = "more than 16 blocks";
+    return false;
+  }
   GenParams& g = c->gen;
   int lmax = sh_lmax;
   std::vector<int> in_off, out_off;
@@ -164,7 +168,7 @@ bool general_config(const std::vector<Block>& bin, int sh_lmax, const std::vecto
         if (!(std::abs(A.l - l2) <= B.l && B.l <= A.l + l2 && A.parity * sh_par == B.parity && A.mul == B.mul))
           continue;
         if (n == kGenMaxPaths) {
-          *why = "more than 160 paths";
+          *why = "more than 128 paths";
           return false;
         }
         const int tri = etp_gen::kGenTriId[(A.l * 5 + l2) * 5 + B.l];
@@ -182,6 +186,30 @@ bool general_config(const std::vector<Block>& bin, int sh_lmax, const std::vecto
   }
   g.n_paths = n;
   g.cols = cols;
+  // work groups: the output blocks (forward) and input blocks (backward) that some path touches
+  for (int side = 0; side < 2; ++side) {
+    const std::vector<Block>& blocks = side ? bin : bout;
+    const std::vector<int>& offs = side ? in_off : out_off;
+    GenGroup* grp = side ? g.in_grp : g.out_grp;
+    unsigned char* order = side ? g.order_in : g.order_out;
+    int ng = 0, k = 0, mx = 0;
+    for (size_t b = 0; b < blocks.size(); ++b) {
+      const int beg = k;
+      for (int q = 0; q < n; ++q)
+        if ((side ? g.p[q].in_off : g.p[q].out_off) == offs[b]) order[k++] = static_cast<unsigned char>(q);
+      if (k == beg) continue;
+      const int size = blocks[b].mul * (2 * blocks[b].l + 1);
+      grp[ng++] = GenGroup{offs[b], size, beg, k};
+      mx = size > mx ? size : mx;
+    }
+    if (side) {
+      g.n_in_groups = ng;
+      g.max_in_size = mx;
+    } else {
+      g.n_out_groups = ng;
+      g.max_out_size = mx;
+    }
+  }
   g.sh_lmax = sh_lmax;
   g.inv_rc = 1.0f / r_cut;
   int mul = bin[0].mul;
@@ -317,7 +345,8 @@ static size_t ws_tc_offset(int n_edges) {
 
 size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   if (!h || n_edges < 0 || n_nodes < 0) return 0;
-  if (h->c.general) return ws_tc_offset(n_edges);   // receiver of each edge + validation scratch
+  if (h->c.general)   // receiver of each edge + validation scratch + edge-gradient partials
+    return ws_tc_offset(n_edges) + general_backward_partials_bytes(h->c.gen, n_edges);
   const size_t f = tc::forward_tc_workspace_bytes(h->c, n_nodes);
   const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
   const size_t w = weight_grad_workspace_bytes(h->c, n_edges);
@@ -448,7 +477,9 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
   if (n_nodes == 0) return ETP_OK;
   if (h->c.general)
     return launch_general_backward(h->c.gen, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W,
-                                   grad_out, grad_x, grad_edge_vec, recv_map, s);
+                                   grad_out, grad_x, grad_edge_vec, recv_map,
+                                   reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_tc_offset(n_edges)),
+                                   s);
   if (n_edges > 0 && use_tc_backward()) {
     void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
     st = tc::launch_backward_tc(h->c, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W, grad_out,

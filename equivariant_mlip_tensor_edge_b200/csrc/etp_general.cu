@@ -6,11 +6,14 @@
 // warp-uniform coupling index. Lanes hold channels: a path with mul channels runs its channel
 // u on lane u % 32, so every node-row access of a warp is one coalesced row segment.
 //
-//   forward : a warp per receiver, its output row accumulated in shared memory (each element
-//             belongs to one lane), edges in CSR order, paths in order: deterministic.
-//   backward: a warp per sender over the transposed order; grad_x accumulated like the forward
-//             output; per edge, dL/dY and dL/dR_b summed over the lanes in a fixed butterfly
-//             and turned into dL/dr_e by lane 0 (chain through the harmonics' gradient and dR/dd).
+//   forward : a warp per (receiver, output block): the block's row segment accumulated in shared
+//             memory (each element belongs to one lane), edges in CSR order, paths in order:
+//             deterministic. The geometry of 32 edges at a time (harmonics, radial basis) is
+//             computed one edge per lane and shared through shared memory.
+//   backward: a warp per (sender, input block) over the transposed order; grad_x accumulated like
+//             the forward output; per edge, dL/dY and dL/dR_b summed over the lanes in a fixed
+//             butterfly and turned into the block's share of dL/dr_e by lane 0 (chain through the
+//             harmonics' gradient and dR/dd); the shares are added over the blocks in order.
 #include <cstdint>
 #include <string>
 
@@ -53,6 +56,26 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Per-edge geometry staged in shared memory, one edge per lane, read back by every lane.
+constexpr int kGeoF = kY + kNumBasis;                      // forward: Y, R (odd stride: no bank conflicts)
+constexpr int kGeoB = kY + 2 * kNumBasis + 4;              // backward: Y, R, dR, n, 1/d
+
+__device__ __forceinline__ void edge_geometry(const float* __restrict__ edge_vec, int e, int sh_lmax, float inv_rc,
+                                              float (&Y)[kY], float (&R)[kNumBasis], float (&dR)[kNumBasis],
+                                              float (&n)[3], float& inv_d, bool deriv) {
+  const float vx = edge_vec[3 * e], vy = edge_vec[3 * e + 1], vz = edge_vec[3 * e + 2];
+  const float d = sqrtf(vx * vx + vy * vy + vz * vz);
+  inv_d = d > 0.0f ? 1.0f / d : 0.0f;
+  n[0] = vx * inv_d;
+  n[1] = vy * inv_d;
+  n[2] = vz * inv_d;
+  gen_sh(sh_lmax, n[0], n[1], n[2], Y);
+  if (deriv) radial_basis<true>(d, inv_rc, R, dR);
+  else radial_basis<false>(d, inv_rc, R, dR);
+}
+
+// Work unit: (receiver i, output block q). The warp sums, over i's edges and the paths into q,
+// the block's row segment in shared memory (element (m3, u) belongs to lane u % 32).
 __global__ void __launch_bounds__(32 * kGenWarps) k_gen_fwd(const __grid_constant__ GenParams g, int n_nodes,
                                                             const int* __restrict__ row_ptr,
                                                             const int* __restrict__ sender,
@@ -60,40 +83,81 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_fwd(const __grid_constan
                                                             const float* __restrict__ x,
                                                             const float* __restrict__ W,
                                                             float* __restrict__ out) {
-  extern __shared__ float sacc[];
+  extern __shared__ float smem[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  float* acc = sacc + wib * g.dim_out;
+  float* acc = smem + wib * (g.max_out_size + 32 * kGeoF + 32);
+  float* geo = acc + g.max_out_size;
+  int* sj = reinterpret_cast<int*>(geo + 32 * kGeoF);
+  const int n_items = n_nodes * g.n_out_groups;
   const int stride = gridDim.x * kGenWarps;
-  for (int i = blockIdx.x * kGenWarps + wib; i < n_nodes; i += stride) {
-    for (int v = lane; v < g.dim_out; v += 32) acc[v] = 0.0f;
-    __syncwarp();
+  for (int it = blockIdx.x * kGenWarps + wib; it < n_items; it += stride) {
+    const int i = it / g.n_out_groups;
+    const GenGroup& G = g.out_grp[it - i * g.n_out_groups];
+    for (int v = lane; v < G.size; v += 32) acc[v] = 0.0f;
     const int e1 = row_ptr[i + 1];
-    for (int e = row_ptr[i]; e < e1; ++e) {
-      const float vx = edge_vec[3 * e], vy = edge_vec[3 * e + 1], vz = edge_vec[3 * e + 2];
-      const float d = sqrtf(vx * vx + vy * vy + vz * vz);
-      const float inv_d = d > 0.0f ? 1.0f / d : 0.0f;
-      float Y[kY], R[kNumBasis], dR[kNumBasis];
-      gen_sh(g.sh_lmax, vx * inv_d, vy * inv_d, vz * inv_d, Y);
-      radial_basis<false>(d, g.inv_rc, R, dR);
-      const float* xj = x + static_cast<size_t>(sender[e]) * g.dim_in;
-      for (int p = 0; p < g.n_paths; ++p) {
-        const GenPath& P = g.p[p];
-        for (int u = lane; u < P.mul; u += 32) {
-          float w = 0.0f;
+    for (int c0 = row_ptr[i]; c0 < e1; c0 += 32) {
+      __syncwarp();   // the previous chunk's geometry has been read
+      if (c0 + lane < e1) {
+        float Y[kY], R[kNumBasis], dR[kNumBasis], nv[3], inv_d;
+        edge_geometry(edge_vec, c0 + lane, g.sh_lmax, g.inv_rc, Y, R, dR, nv, inv_d, false);
 #pragma unroll
-          for (int b = 0; b < kNumBasis; ++b) w = fmaf(R[b], __ldg(W + static_cast<size_t>(b) * g.cols + P.woff + u), w);
-          etp_gen::gen_fwd(P.tri, xj + P.in_off + u, P.mul, Y, w, acc + P.out_off + u);
+        for (int c = 0; c < kY; ++c) geo[lane * kGeoF + c] = Y[c];
+#pragma unroll
+        for (int b = 0; b < kNumBasis; ++b) geo[lane * kGeoF + kY + b] = R[b];
+        sj[lane] = sender[c0 + lane];
+      }
+      __syncwarp();
+      const int cnt = e1 - c0 < 32 ? e1 - c0 : 32;
+      for (int k = 0; k < cnt; ++k) {
+        const float* Y = geo + k * kGeoF;   // harmonics of edge k, read where the coupling uses them
+        float R[kNumBasis];
+#pragma unroll
+        for (int b = 0; b < kNumBasis; ++b) R[b] = geo[k * kGeoF + kY + b];
+        const float* xj = x + static_cast<size_t>(sj[k]) * g.dim_in;
+        for (int pi = G.beg; pi < G.end; ++pi) {
+          const GenPath& P = g.p[g.order_out[pi]];
+          for (int u = lane; u < P.mul; u += 32) {
+            float w = 0.0f;
+#pragma unroll
+            for (int b = 0; b < kNumBasis; ++b)
+              w = fmaf(R[b], __ldg(W + static_cast<size_t>(b) * g.cols + P.woff + u), w);
+            etp_gen::gen_fwd(P.tri, xj + P.in_off + u, P.mul, Y, w, acc + (P.out_off - G.off) + u);
+          }
         }
       }
     }
     __syncwarp();
-    float* orow = out + static_cast<size_t>(i) * g.dim_out;
-    for (int v = lane; v < g.dim_out; v += 32) orow[v] = acc[v];
-    __syncwarp();
+    float* orow = out + static_cast<size_t>(i) * g.dim_out + G.off;
+    for (int v = lane; v < G.size; v += 32) orow[v] = acc[v];
   }
 }
 
-__global__ void __launch_bounds__(32 * kGenWarps) k_gen_bwd(const __grid_constant__ GenParams g, int n_nodes,
+// Sum of v[k] over the warp for k = 0..31, scattered: lane L returns the sum of v[L]. Recursive
+// halving (16 + 8 + 4 + 2 + 1 shuffles), a fixed order.
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int k = 0; k < o; ++k) {
+      const float send = up ? v[k] : v[k + o];
+      const float keep = up ? v[k + o] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+constexpr int kRed = 33;   // per-edge reduced values: dL/dY (up to 25) and dL/dR (8), padded row
+
+// Work unit: (sender j, input block q) over the transposed order. grad_x of the block's row
+// segment as in the forward. Per edge the lanes'
+// dL/dY and dL/dR_b are summed by one scatter-reduction into a shared row; once per 32 edges,
+// lane k turns edge k's row into the group's share of dL/dr_e (chain through the harmonics'
+// gradient and dR/dd) at vec_out + 3 e: grad_edge_vec itself when there is one group, else the
+// group's partial array, summed over the groups in order afterwards.
+__global__ void __launch_bounds__(32 * kGenWarps, 3) k_gen_bwd(const __grid_constant__ GenParams g, int n_nodes,
+                                                            int n_edges,
                                                             const int* __restrict__ t_row_ptr,
                                                             const int* __restrict__ t_perm,
                                                             const int* __restrict__ recv,
@@ -102,72 +166,159 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_bwd(const __grid_constan
                                                             const float* __restrict__ W,
                                                             const float* __restrict__ gout,
                                                             float* __restrict__ grad_x,
-                                                            float* __restrict__ grad_vec) {
-  extern __shared__ float sgx[];
+                                                            float* __restrict__ vec_out) {
+  extern __shared__ float smem[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  float* gx = sgx + wib * g.dim_in;
+  float* gx = smem + wib * (g.max_in_size + 32 * kGeoB + 32 * kRed + 64);
+  float* geo = gx + g.max_in_size;
+  float* red = geo + 32 * kGeoB;
+  int* si = reinterpret_cast<int*>(red + 32 * kRed);
+  int* se = si + 32;
+  const bool wide = g.sh_lmax > 3;   // 25 + 8 values: one more than the scatter-reduction holds
+  const int n_items = n_nodes * g.n_in_groups;
   const int stride = gridDim.x * kGenWarps;
-  for (int j = blockIdx.x * kGenWarps + wib; j < n_nodes; j += stride) {
-    for (int v = lane; v < g.dim_in; v += 32) gx[v] = 0.0f;
-    __syncwarp();
+  for (int it = blockIdx.x * kGenWarps + wib; it < n_items; it += stride) {
+    const int j = it / g.n_in_groups;
+    const int q = it - j * g.n_in_groups;
+    const GenGroup& G = g.in_grp[q];
+    float* vq = vec_out ? vec_out + (g.n_in_groups > 1 ? static_cast<size_t>(q) * 3 * n_edges : 0) : nullptr;
+    for (int v = lane; v < G.size; v += 32) gx[v] = 0.0f;
     const float* xj = x + static_cast<size_t>(j) * g.dim_in;
     const int t1 = t_row_ptr[j + 1];
-    for (int t = t_row_ptr[j]; t < t1; ++t) {
-      const int e = t_perm[t];
-      const int i = recv[e];
-      const float vx = edge_vec[3 * e], vy = edge_vec[3 * e + 1], vz = edge_vec[3 * e + 2];
-      const float d = sqrtf(vx * vx + vy * vy + vz * vz);
-      const float inv_d = d > 0.0f ? 1.0f / d : 0.0f;
-      const float nx = vx * inv_d, ny = vy * inv_d, nz = vz * inv_d;
-      float Y[kY], R[kNumBasis], dR[kNumBasis];
-      gen_sh(g.sh_lmax, nx, ny, nz, Y);
-      radial_basis<true>(d, g.inv_rc, R, dR);
-      float gY[kY], gR[kNumBasis];
+    for (int c0 = t_row_ptr[j]; c0 < t1; c0 += 32) {
+      __syncwarp();
+      if (c0 + lane < t1) {
+        const int e = t_perm[c0 + lane];
+        float Y[kY], R[kNumBasis], dR[kNumBasis], nv[3], inv_d;
+        edge_geometry(edge_vec, e, g.sh_lmax, g.inv_rc, Y, R, dR, nv, inv_d, true);
+        float* o = geo + lane * kGeoB;
 #pragma unroll
-      for (int k = 0; k < kY; ++k) gY[k] = 0.0f;
+        for (int c = 0; c < kY; ++c) o[c] = Y[c];
 #pragma unroll
-      for (int b = 0; b < kNumBasis; ++b) gR[b] = 0.0f;
-      const float* gi = gout + static_cast<size_t>(i) * g.dim_out;
-      for (int p = 0; p < g.n_paths; ++p) {
-        const GenPath& P = g.p[p];
-        for (int u = lane; u < P.mul; u += 32) {
-          float wb[kNumBasis];
-          float w = 0.0f;
+        for (int b = 0; b < kNumBasis; ++b) {
+          o[kY + b] = R[b];
+          o[kY + kNumBasis + b] = dR[b];
+        }
+        o[kY + 2 * kNumBasis + 0] = nv[0];
+        o[kY + 2 * kNumBasis + 1] = nv[1];
+        o[kY + 2 * kNumBasis + 2] = nv[2];
+        o[kY + 2 * kNumBasis + 3] = inv_d;
+        si[lane] = recv[e];
+        se[lane] = e;
+      }
+      __syncwarp();
+      const int cnt = t1 - c0 < 32 ? t1 - c0 : 32;
+      for (int k = 0; k < cnt; ++k) {
+        const float* o = geo + k * kGeoB;
+        const float* Y = o;   // harmonics of edge k, read where the coupling uses them
+        float R[kNumBasis];
 #pragma unroll
-          for (int b = 0; b < kNumBasis; ++b) {
-            wb[b] = __ldg(W + static_cast<size_t>(b) * g.cols + P.woff + u);
-            w = fmaf(R[b], wb[b], w);
+        for (int b = 0; b < kNumBasis; ++b) R[b] = o[kY + b];
+        float gY[kY], gR[kNumBasis];
+#pragma unroll
+        for (int c = 0; c < kY; ++c) gY[c] = 0.0f;
+#pragma unroll
+        for (int b = 0; b < kNumBasis; ++b) gR[b] = 0.0f;
+        const float* gi = gout + static_cast<size_t>(si[k]) * g.dim_out;
+        for (int pi = G.beg; pi < G.end; ++pi) {
+          const GenPath& P = g.p[g.order_in[pi]];
+          for (int u = lane; u < P.mul; u += 32) {
+            float wb[kNumBasis];
+            float w = 0.0f;
+#pragma unroll
+            for (int b = 0; b < kNumBasis; ++b) {
+              wb[b] = __ldg(W + static_cast<size_t>(b) * g.cols + P.woff + u);
+              w = fmaf(R[b], wb[b], w);
+            }
+            float gw = 0.0f;
+            etp_gen::gen_bwd(P.tri, xj + P.in_off + u, gi + P.out_off + u, P.mul, Y, w, gx + (P.in_off - G.off) + u,
+                             gY, gw);
+#pragma unroll
+            for (int b = 0; b < kNumBasis; ++b) gR[b] = fmaf(wb[b], gw, gR[b]);
           }
-          float gw = 0.0f;
-          etp_gen::gen_bwd(P.tri, xj + P.in_off + u, gi + P.out_off + u, P.mul, Y, w, gx + P.in_off + u, gY, gw);
+        }
+        if (vq) {
+          // row layout: harmonics to l = 3 -> [gY 0..15][gR 0..7]; to l = 4 -> [gY 0..24][gR 0..7]
+          float v[32];
+          if (!wide) {
 #pragma unroll
-          for (int b = 0; b < kNumBasis; ++b) gR[b] = fmaf(wb[b], gw, gR[b]);
+            for (int c = 0; c < 16; ++c) v[c] = gY[c];
+#pragma unroll
+            for (int b = 0; b < kNumBasis; ++b) v[16 + b] = gR[b];
+#pragma unroll
+            for (int c = 24; c < 32; ++c) v[c] = 0.0f;
+          } else {
+#pragma unroll
+            for (int c = 0; c < kY; ++c) v[c] = gY[c];
+#pragma unroll
+            for (int b = 0; b < 7; ++b) v[kY + b] = gR[b];
+          }
+          const float r = reduce_scatter32(v, lane);
+          red[k * kRed + lane] = r;
+          if (wide) {
+            const float r7 = warp_sum(gR[7]);
+            if (lane == 0) red[k * kRed + 32] = r7;
+          }
         }
       }
-      if (grad_vec) {
+      if (vq) {
+        __syncwarp();
+        if (lane < cnt) {
+          const float* rr = red + lane * kRed;
+          const float* o = geo + lane * kGeoB;
+          float gY[kY], gR[kNumBasis];
+          if (!wide) {
 #pragma unroll
-        for (int k = 0; k < kY; ++k) gY[k] = warp_sum(gY[k]);
+            for (int c = 0; c < kY; ++c) gY[c] = c < 16 ? rr[c] : 0.0f;
 #pragma unroll
-        for (int b = 0; b < kNumBasis; ++b) gR[b] = warp_sum(gR[b]);
-        if (lane == 0) {
+            for (int b = 0; b < kNumBasis; ++b) gR[b] = rr[16 + b];
+          } else {
+#pragma unroll
+            for (int c = 0; c < kY; ++c) gY[c] = rr[c];
+#pragma unroll
+            for (int b = 0; b < kNumBasis; ++b) gR[b] = rr[kY + b];
+          }
           float gd = 0.0f;
 #pragma unroll
-          for (int b = 0; b < kNumBasis; ++b) gd = fmaf(gR[b], dR[b], gd);
+          for (int b = 0; b < kNumBasis; ++b) gd = fmaf(gR[b], o[kY + kNumBasis + b], gd);
+          const float nx = o[kY + 2 * kNumBasis], ny = o[kY + 2 * kNumBasis + 1], nz = o[kY + 2 * kNumBasis + 2];
+          const float inv_d = o[kY + 2 * kNumBasis + 3];
           float Gx, Gy, Gz, S;
           gen_sh_grad(g.sh_lmax, nx, ny, nz, gY, Gx, Gy, Gz, S);
           // dL/dr = gd n + (G - S n) / d
-          grad_vec[3 * e + 0] = fmaf(gd, nx, (Gx - S * nx) * inv_d);
-          grad_vec[3 * e + 1] = fmaf(gd, ny, (Gy - S * ny) * inv_d);
-          grad_vec[3 * e + 2] = fmaf(gd, nz, (Gz - S * nz) * inv_d);
+          const int e = se[lane];
+          vq[3 * e + 0] = fmaf(gd, nx, (Gx - S * nx) * inv_d);
+          vq[3 * e + 1] = fmaf(gd, ny, (Gy - S * ny) * inv_d);
+          vq[3 * e + 2] = fmaf(gd, nz, (Gz - S * nz) * inv_d);
         }
       }
     }
     __syncwarp();
     if (grad_x) {
-      float* row = grad_x + static_cast<size_t>(j) * g.dim_in;
-      for (int v = lane; v < g.dim_in; v += 32) row[v] = gx[v];
+      float* row = grad_x + static_cast<size_t>(j) * g.dim_in + G.off;
+      for (int v = lane; v < G.size; v += 32) row[v] = gx[v];
     }
-    __syncwarp();
+  }
+}
+
+// grad_edge_vec = sum of the input blocks' partials, in block order.
+__global__ void k_gen_sum_parts(const float* __restrict__ part, int n_groups, int n, float* __restrict__ out) {
+  for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < n; v += gridDim.x * blockDim.x) {
+    float s = part[v];
+    for (int q = 1; q < n_groups; ++q) s += part[static_cast<size_t>(q) * n + v];
+    out[v] = s;
+  }
+}
+
+// Input blocks that no path reads get zero grad_x rows.
+__global__ void k_gen_zero_unread(const __grid_constant__ GenParams g, int n_nodes, float* __restrict__ grad_x) {
+  const long long total = static_cast<long long>(n_nodes) * g.dim_in;
+  for (long long v = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; v < total;
+       v += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(v % g.dim_in);
+    bool read = false;
+    for (int q = 0; q < g.n_in_groups; ++q) read |= c >= g.in_grp[q].off && c < g.in_grp[q].off + g.in_grp[q].size;
+    if (!read) grad_x[v] = 0.0f;
   }
 }
 
@@ -187,33 +338,62 @@ int gen_blocks(int n_nodes) {
 
 }  // namespace
 
+size_t general_backward_partials_bytes(const GenParams& g, int n_edges) {
+  return g.n_in_groups > 1 ? align256(sizeof(float) * 3 * static_cast<size_t>(n_edges) * g.n_in_groups) : 0;
+}
+
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                   const int* sender, const float* edge_vec, const float* x, const float* W,
                                   float* out, cudaStream_t s) {
   (void)n_edges;
   if (n_nodes == 0) return ETP_OK;
-  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.dim_out);
+  int covered = 0;
+  for (int q = 0; q < g.n_out_groups; ++q) covered += g.out_grp[q].size;
+  if (covered < g.dim_out) {
+    // output blocks that no path writes are zero
+    cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * static_cast<size_t>(n_nodes) * g.dim_out, s);
+    if (e != cudaSuccess) return cuda_status(e, "general forward memset");
+  }
+  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.max_out_size + 32 * kGeoF + 32);
   cudaError_t e = cudaFuncSetAttribute(k_gen_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_status(e, "general forward smem attribute");
-  k_gen_fwd<<<gen_blocks(n_nodes), 32 * kGenWarps, smem, s>>>(g, n_nodes, row_ptr, sender, edge_vec, x, W, out);
+  k_gen_fwd<<<gen_blocks(n_nodes * g.n_out_groups), 32 * kGenWarps, smem, s>>>(g, n_nodes, row_ptr, sender, edge_vec,
+                                                                                x, W, out);
   return cuda_status(cudaGetLastError(), "general forward launch");
 }
 
 etp_status launch_general_backward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                    const float* edge_vec, const int* t_row_ptr, const int* t_perm,
                                    const float* x, const float* W, const float* grad_out, float* grad_x,
-                                   float* grad_edge_vec, int* recv, cudaStream_t s) {
+                                   float* grad_edge_vec, int* recv, float* part, cudaStream_t s) {
   if (n_nodes == 0) return ETP_OK;
   if (n_edges > 0) {
     etp_status st = launch_recv_of_edge(row_ptr, n_nodes, n_edges, recv, s);
     if (st != ETP_OK) return st;
   }
-  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.dim_in);
+  int covered = 0;
+  for (int q = 0; q < g.n_in_groups; ++q) covered += g.in_grp[q].size;
+  if (grad_x && covered < g.dim_in) {
+    k_gen_zero_unread<<<gen_blocks(n_nodes), 256, 0, s>>>(g, n_nodes, grad_x);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "general backward zero launch");
+  }
+  const bool split = grad_edge_vec && g.n_in_groups > 1 && n_edges > 0;
+  float* vec_out = split ? part : grad_edge_vec;
+  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.max_in_size + 32 * kGeoB + 32 * kRed + 64);
   cudaError_t e = cudaFuncSetAttribute(k_gen_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_status(e, "general backward smem attribute");
-  k_gen_bwd<<<gen_blocks(n_nodes), 32 * kGenWarps, smem, s>>>(g, n_nodes, t_row_ptr, t_perm, recv, edge_vec, x, W,
-                                                               grad_out, grad_x, grad_edge_vec);
-  return cuda_status(cudaGetLastError(), "general backward launch");
+  k_gen_bwd<<<gen_blocks(n_nodes * g.n_in_groups), 32 * kGenWarps, smem, s>>>(g, n_nodes, n_edges, t_row_ptr, t_perm,
+                                                                               recv, edge_vec, x, W, grad_out, grad_x,
+                                                                               vec_out);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "general backward launch");
+  if (split) {
+    k_gen_sum_parts<<<gen_blocks(3 * n_edges), 256, 0, s>>>(part, g.n_in_groups, 3 * n_edges, grad_edge_vec);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_status(e, "general backward sum launch");
+  }
+  return ETP_OK;
 }
 
 }  // namespace etp

@@ -17,10 +17,17 @@ constexpr int kMaxL = 3;
 // General irreps (any multiplicities and parities, rank <= 4): the path table the kernels read
 // from their parameter block. Path p couples input block component rows starting at in_off with
 // the harmonics of rank l2 into the output block at out_off, over mul channels, with weight
-// columns woff .. woff + mul - 1; tri is the coupling index of (l1, l2, l3).
-constexpr int kGenMaxPaths = 160;
+// columns woff .. woff + mul - 1; tri is the coupling index of (l1, l2, l3). The paths are also
+// listed grouped by output block (forward work units) and by input block (backward work units),
+// each group keeping the lexicographic path order.
+constexpr int kGenMaxPaths = 128;
+constexpr int kGenMaxBlocks = 16;
 struct GenPath {
   int in_off, out_off, woff, mul, tri;
+};
+struct GenGroup {
+  int off, size;      // the block's row segment: offset and mul (2l + 1) floats
+  int beg, end;       // its paths: order[beg .. end - 1]
 };
 struct GenParams {
   int n_paths = 0;
@@ -29,8 +36,17 @@ struct GenParams {
   int cols = 0;        // weight columns per basis function (sum of the paths' multiplicities)
   int sh_lmax = 0;
   float inv_rc = 0.f;
+  int n_out_groups = 0;
+  int n_in_groups = 0;
+  int max_out_size = 0;
+  int max_in_size = 0;
   GenPath p[kGenMaxPaths];
+  GenGroup out_grp[kGenMaxBlocks];
+  GenGroup in_grp[kGenMaxBlocks];
+  unsigned char order_out[kGenMaxPaths];
+  unsigned char order_in[kGenMaxPaths];
 };
+static_assert(sizeof(GenParams) <= 4000, "the path table travels as a kernel parameter");
 
 struct Ctx {
   int lmax = 0;
@@ -108,15 +124,17 @@ etp_status launch_weight_grad(const Ctx& c, int n_nodes, int n_edges, const int*
                               const float* edge_vec, const float* x, const float* grad_out, float* grad_W,
                               int* recv, void* ws, cudaStream_t s);
 
-// ---- general irreps (etp_general.cu); recv: n_edges ints of scratch
-constexpr int kGenMaxDim = 4096;   // floats per node row (the kernels keep one row per warp in shared memory)
+// ---- general irreps (etp_general.cu); recv: n_edges ints of scratch; part: the per-input-block
+// edge-gradient partials (general_backward_partials_bytes)
+constexpr int kGenMaxDim = 4096;   // floats per node row
+size_t general_backward_partials_bytes(const GenParams& g, int n_edges);
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                   const int* sender, const float* edge_vec, const float* x, const float* W,
                                   float* out, cudaStream_t s);
 etp_status launch_general_backward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                    const float* edge_vec, const int* t_row_ptr, const int* t_perm,
                                    const float* x, const float* W, const float* grad_out, float* grad_x,
-                                   float* grad_edge_vec, int* recv, cudaStream_t s);
+                                   float* grad_edge_vec, int* recv, float* part, cudaStream_t s);
 
 // ---- node-local product ladder (etp_product.cu)
 etp_status launch_node_ladder(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,

@@ -674,6 +674,7 @@ GENERAL = [
     ("32x0e+32x1o+32x2e+32x3o+32x4e", 4, "32x0e+32x1o+32x2e+32x3o+32x4e"),   # rank 4
     ("16x0e+16x1o", 2, "16x0e+16x1o+16x1e+16x2e"),                         # irreps_out != irreps_in
     ("6x0e+6x1o+6x2e", 2, "6x0e+6x1o+6x2e"),                               # C not a multiple of 4
+    ("8x0e+4x2e", 0, "8x0e+4x1o"),         # an input block no path reads, an output block none writes
 ]
 
 
