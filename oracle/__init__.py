@@ -10,15 +10,17 @@ arithmetic).
 What it computes (plain definitions, no blocking, fusion or reordering):
 
 * ``cg``     -- Clebsch-Gordan coefficients from Racah's closed form, exact in
-               rational arithmetic, moved to the real spherical-harmonic basis.
+               rational arithmetic, moved to the real spherical-harmonic basis
+               (for l1 + l2 + l3 odd: the imaginary part of the moved tensor).
 * ``sh``     -- real spherical harmonics, component normalisation, as solid
                harmonic polynomials, with their analytic gradient.
 * ``wigner`` -- Wigner D matrices from Wigner's small-d formula (used by the
                equivariance pins).
 * ``radial`` -- Bessel radial basis times the polynomial cutoff envelope.
 * ``graph``  -- brute-force neighbour list and canonical receiver-sorted CSR.
-* ``conv``   -- irreps/path enumeration, the forward edge convolution and its
-               analytic vector-Jacobian product.
+* ``conv``   -- irreps/path enumeration (any multiplicities and parities), the
+               forward edge convolution and its analytic vector-Jacobian product.
+* ``product``-- the node-local path-reduced product and product ladder.
 
 Sources. The pages behind this build ("Fast and Accurate Foundation Models for
 Equivariant MLIPs", section VII Methods; "FlashCart", Fig. 3 caption, Table C1,
