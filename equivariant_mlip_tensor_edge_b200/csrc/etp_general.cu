@@ -7,9 +7,10 @@
 // u on lane u % 32, so every node-row access of a warp is one coalesced row segment.
 //
 //   forward : a warp per (receiver, output block): the block's row segment accumulated in shared
-//             memory (each element belongs to one lane), edges in CSR order, paths in order:
-//             deterministic. The geometry of 32 edges at a time (harmonics, radial basis) is
-//             computed one edge per lane and shared through shared memory.
+//             memory (each element belongs to one lane). The geometry of 32 edges at a time
+//             (harmonics, radial basis) is computed one edge per lane and staged in shared memory;
+//             then, path by path, each lane runs its channel over the 32 edges with the path's W
+//             column and sums in registers. Fixed order (chunks, paths, edges): deterministic.
 //   backward: a warp per (sender, input block) over the transposed order; grad_x accumulated like
 //             the forward output; per edge, dL/dY and dL/dR_b summed over the lanes in a fixed
 //             butterfly and turned into the block's share of dL/dr_e by lane 0 (chain through the
@@ -57,7 +58,9 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Per-edge geometry staged in shared memory, one edge per lane, read back by every lane.
-constexpr int kGeoF = kY + kNumBasis;                      // forward: Y, R (odd stride: no bank conflicts)
+constexpr int kGeoF = etp_gen::kGenGeoF;                   // forward: Y, R (odd stride: no bank conflicts)
+static_assert(kGeoF == kY + kNumBasis, "staged forward geometry");
+constexpr int kRun = 32;                                   // forward: edges per path-major run (the whole chunk)
 constexpr int kGeoB = kY + 2 * kNumBasis + 4;              // backward: Y, R, dR, n, 1/d
 
 __device__ __forceinline__ void edge_geometry(const float* __restrict__ edge_vec, int e, int sh_lmax, float inv_rc,
@@ -108,20 +111,18 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_fwd(const __grid_constan
       }
       __syncwarp();
       const int cnt = e1 - c0 < 32 ? e1 - c0 : 32;
-      for (int k = 0; k < cnt; ++k) {
-        const float* Y = geo + k * kGeoF;   // harmonics of edge k, read where the coupling uses them
-        float R[kNumBasis];
-#pragma unroll
-        for (int b = 0; b < kNumBasis; ++b) R[b] = geo[k * kGeoF + kY + b];
-        const float* xj = x + static_cast<size_t>(sj[k]) * g.dim_in;
+      // path-major over runs of kRun edges: the channel's W column and path sums stay in
+      // registers, and the run's sender rows stay in L1 across the paths
+      for (int r0 = 0; r0 < cnt; r0 += kRun) {
+        const int rc = cnt - r0 < kRun ? cnt - r0 : kRun;
         for (int pi = G.beg; pi < G.end; ++pi) {
           const GenPath& P = g.p[g.order_out[pi]];
           for (int u = lane; u < P.mul; u += 32) {
-            float w = 0.0f;
+            float wb[kNumBasis];
 #pragma unroll
-            for (int b = 0; b < kNumBasis; ++b)
-              w = fmaf(R[b], __ldg(W + static_cast<size_t>(b) * g.cols + P.woff + u), w);
-            etp_gen::gen_fwd(P.tri, xj + P.in_off + u, P.mul, Y, w, acc + (P.out_off - G.off) + u);
+            for (int b = 0; b < kNumBasis; ++b) wb[b] = __ldg(W + static_cast<size_t>(b) * g.cols + P.woff + u);
+            etp_gen::gen_fwd_chunk(P.tri, geo + r0 * kGeoF, sj + r0, rc, x + P.in_off + u, g.dim_in, P.mul, wb,
+                                   acc + (P.out_off - G.off) + u);
           }
         }
       }

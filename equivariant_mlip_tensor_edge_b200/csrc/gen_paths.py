@@ -540,9 +540,10 @@ def gen_triples():
 
 
 def emit_general(out):
-    """Per coupling t = (l1, l2, l3): gfwd_t adds w sum C Y x into acc[m3 * stride] and gbwd_t
-    accumulates grad_x, dL/dY and dL/dw for one channel. x, g and acc point at the channel's
-    element of component 0 of their block; components are `stride` floats apart."""
+    """Per coupling t = (l1, l2, l3): gbwd_t accumulates grad_x, dL/dY and dL/dw for one channel
+    and one edge, gfwdc_t adds sum_edges w sum C Y x over a chunk of staged edges into
+    acc[m3 * stride]. x, g and acc point at the channel's element of component 0 of their block;
+    components are `stride` floats apart."""
     tri = gen_triples()
     out.append(f"constexpr int kGenLmax = {GEN_LMAX};")
     out.append(f"constexpr int kGenTriples = {len(tri)};")
@@ -562,26 +563,7 @@ def emit_general(out):
                 terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
                 if terms:
                     groups.append((m3, m1, terms))
-        # forward
         out.append(f"// ({l1},{l2},{l3})")
-        out.append(f"__device__ __forceinline__ void gfwd_{t}(const float* __restrict__ x, int stride, const float* Y,")
-        out.append("                                       float w, float* acc) {")
-        for m1 in range(2 * l1 + 1):
-            out.append(f"  const float x{m1} = x[{m1} * stride];")
-        for m3 in range(2 * l3 + 1):
-            row = [(m1, terms) for (a3, m1, terms) in groups if a3 == m3]
-            if not row:
-                continue
-            first = True
-            for m1, terms in row:
-                mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
-                if first:
-                    out.append(f"  float s{m3} = ({mexpr}) * x{m1};")
-                    first = False
-                else:
-                    out.append(f"  s{m3} = fmaf({mexpr}, x{m1}, s{m3});")
-            out.append(f"  acc[{m3} * stride] = fmaf(w, s{m3}, acc[{m3} * stride]);")
-        out.append("}")
         # backward
         out.append(f"__device__ __forceinline__ void gbwd_{t}(const float* __restrict__ x, const float* __restrict__ g,")
         out.append("                                       int stride, const float* Y, float w, float* gx, float* gY,")
@@ -603,11 +585,52 @@ def emit_general(out):
         for m1 in range(2 * l1 + 1):
             out.append(f"  gx[{m1} * stride] = fmaf(w, a{m1}, gx[{m1} * stride]);")
         out.append("}")
-    out.append("__device__ __forceinline__ void gen_fwd(int t, const float* x, int stride, const float* Y, float w,")
-    out.append("                                        float* acc) {")
+    # forward over a chunk of staged edges: the channel's path sums stay in registers across the
+    # chunk, and the path's radial weights are projected per edge from the staged R
+    out.append(f"constexpr int kGenGeoF = 33;   // staged floats per edge: Y (25), R (8)")
+    for t, (l1, l2, l3) in enumerate(tri):
+        c = real_cg_any(l1, l2, l3)
+        groups = []
+        for m3 in range(2 * l3 + 1):
+            for m1 in range(2 * l1 + 1):
+                terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
+                if terms:
+                    groups.append((m3, m1, terms))
+        out.append(f"__device__ __forceinline__ void gfwdc_{t}(const float* geo, const int* sj, int cnt,")
+        out.append("                                        const float* __restrict__ xu, int dim_in, int stride,")
+        out.append("                                        const float* wb, float* acc) {")
+        rows = sorted({m3 for m3, _, _ in groups})
+        for m3 in rows:
+            out.append(f"  float a{m3} = 0.0f;")
+        out.append("  for (int k = 0; k < cnt; ++k) {")
+        out.append("    const float* Y = geo + k * kGenGeoF;")
+        out.append("    float w = 0.0f;")
+        out.append("    #pragma unroll")
+        out.append("    for (int b = 0; b < 8; ++b) w = fmaf(Y[25 + b], wb[b], w);")
+        out.append("    const float* x = xu + static_cast<size_t>(sj[k]) * dim_in;")
+        for m1 in range(2 * l1 + 1):
+            out.append(f"    const float x{m1} = x[{m1} * stride];")
+        for m3 in rows:
+            row = [(m1, terms) for (a3, m1, terms) in groups if a3 == m3]
+            first = True
+            for m1, terms in row:
+                mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                if first:
+                    out.append(f"    float s{m3} = ({mexpr}) * x{m1};")
+                    first = False
+                else:
+                    out.append(f"    s{m3} = fmaf({mexpr}, x{m1}, s{m3});")
+            out.append(f"    a{m3} = fmaf(w, s{m3}, a{m3});")
+        out.append("  }")
+        for m3 in rows:
+            out.append(f"  acc[{m3} * stride] += a{m3};")
+        out.append("}")
+    out.append("__device__ __forceinline__ void gen_fwd_chunk(int t, const float* geo, const int* sj, int cnt,")
+    out.append("                                              const float* xu, int dim_in, int stride, const float* wb,")
+    out.append("                                              float* acc) {")
     out.append("  switch (t) {")
     for t in range(len(tri)):
-        out.append(f"    case {t}: gfwd_{t}(x, stride, Y, w, acc); break;")
+        out.append(f"    case {t}: gfwdc_{t}(geo, sj, cnt, xu, dim_in, stride, wb, acc); break;")
     out.append("    default: break;")
     out.append("  }")
     out.append("}")
