@@ -335,8 +335,12 @@ def run_gpu(args, rank, world, local_rank):
     for _ in range(3):
         gen_fwd()
         gen_bwd()
+    g_dw = torch.empty((gi["n_basis"], gi["weight_numel"] // gi["n_basis"]), device=dev)
+    gen_dw = lambda: gconv.backward_weights(gr, g_x, g_g, grad_W=g_dw, workspace=g_ws)
+    gen_dw()
     ms_gen_fwd = timed(gen_fwd, reps, host_ahead=True)
     ms_gen_bwd = timed(gen_bwd, reps, host_ahead=True)
+    ms_gen_dw = timed(gen_dw, reps, host_ahead=True)
     clocks = sampler.stop() if rank == 0 else None
 
     # end to end through the public API with host buffers (copies inside the timed region)
@@ -357,9 +361,9 @@ def run_gpu(args, rank, world, local_rank):
     d2h = out_h.numel() * 4 + f_h.numel() * 4
 
     e = gr.n_edges
-    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd), total_edges = \
-        combine_ranks([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd], e, world,
-                      dev)
+    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd, ms_gen_dw), total_edges = \
+        combine_ranks([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd, ms_gen_dw],
+                      e, world, dev)
     if rank != 0:
         return None
 
@@ -403,7 +407,9 @@ def run_gpu(args, rank, world, local_rank):
                 "hbm_frac_of_" + peak_kind: round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
 
     def general_roof(ms, kind):
-        flop = float(gi[f"flop_{kind}"]) * e
+        # the weight gradient's per-path factor costs what the forward contraction does, plus the
+        # edge reduction sum_e R_b gw (2 n_basis cols flop per edge)
+        flop = (float(gi["flop_fwd"]) + 2.0 * gi["weight_numel"]) * e if kind == "dw" else float(gi[f"flop_{kind}"]) * e
         ach = flop / (ms * 1e-3) / 1e12
         return {"workload": f"{gen_irreps}, harmonics to l = 3, {wl.name} graph ({e} edges)",
                 "kernel": f"k_gen_{kind}", "ms_per_launch": round(ms, 5), "bound": "alu", "achieved": round(ach, 3),
@@ -437,6 +443,7 @@ def run_gpu(args, rank, world, local_rank):
         "node_ladder": ladder_roof(ms_ladder),
         "general_irreps_fwd": general_roof(ms_gen_fwd, "fwd"),
         "general_irreps_bwd": general_roof(ms_gen_bwd, "bwd"),
+        "general_irreps_dw": general_roof(ms_gen_dw, "dw"),
         "e2e": {"value": round(total_edges / (ms_e2e * 1e-3), 1), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step(info, n) * args.steps,

@@ -289,13 +289,15 @@ class EdgeConv:
         return (grad_x if want_grad_x else None), (grad_vec if want_grad_vec else None)
 
     def backward_weights(self, graph, x, grad_out, grad_W=None, workspace=None):
-        """dL/dW [n_basis, n_paths, C] for L = <grad_out, forward(graph, x, W)>."""
+        """dL/dW for L = <grad_out, forward(graph, x, W)>: [n_basis, n_paths, C], or [n_basis, cols] for
+        a general irreps handle."""
         torch = _torch()
         _need_cuda(x, grad_out)
         x, grad_out = _f32(x), _f32(grad_out)
         if grad_W is None:
-            grad_W = torch.empty((self.info["n_basis"], self.info["n_paths"], self.info["channels"]),
-                                 dtype=torch.float32, device=x.device)
+            shape = ((self.info["n_basis"], self.info["n_paths"], self.info["channels"]) if not self.info["general"]
+                     else (self.info["n_basis"], self.info["weight_numel"] // self.info["n_basis"]))
+            grad_W = torch.empty(shape, dtype=torch.float32, device=x.device)
         ws, nb = self._workspace(graph.n_nodes, graph.n_edges, x.device, workspace)
         _check(load_library().etp_backward_weights(
             self._h, graph.n_nodes, graph.n_edges, _ptr(graph.row_ptr), _ptr(graph.sender), _ptr(graph.edge_vec),

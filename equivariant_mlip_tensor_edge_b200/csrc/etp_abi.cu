@@ -345,8 +345,11 @@ static size_t ws_tc_offset(int n_edges) {
 
 size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   if (!h || n_edges < 0 || n_nodes < 0) return 0;
-  if (h->c.general)   // receiver of each edge + validation scratch + edge-gradient partials
-    return ws_tc_offset(n_edges) + general_backward_partials_bytes(h->c.gen, n_edges);
+  if (h->c.general) {   // receiver of each edge + validation scratch + edge-gradient or dW partials
+    const size_t b = general_backward_partials_bytes(h->c.gen, n_edges);
+    const size_t w = general_weight_grad_bytes(h->c.gen, n_edges);
+    return ws_tc_offset(n_edges) + (b > w ? b : w);
+  }
   const size_t f = tc::forward_tc_workspace_bytes(h->c, n_nodes);
   const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
   const size_t w = weight_grad_workspace_bytes(h->c, n_edges);
@@ -572,10 +575,7 @@ etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const in
     set_error("etp_backward_weights: NULL handle");
     return ETP_ERR_INVALID_ARG;
   }
-  if (h->c.general) {
-    set_error("etp_backward_weights: not implemented for general irreps handles");
-    return ETP_ERR_UNSUPPORTED;
-  }
+
   if (n_nodes < 0 || n_edges < 0) {
     set_error("etp_backward_weights: negative size");
     return ETP_ERR_INVALID_ARG;
@@ -600,6 +600,9 @@ etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const in
   }
   int* recv = static_cast<int*>(workspace);
   void* part = workspace ? static_cast<char*>(workspace) + ws_tc_offset(n_edges) : nullptr;
+  if (h->c.general)
+    return launch_general_weight_grad(h->c.gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, grad_out, grad_W,
+                                      recv, static_cast<float*>(part), s);
   return launch_weight_grad(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, grad_out, grad_W, recv, part, s);
 }
 

@@ -302,6 +302,80 @@ __global__ void __launch_bounds__(32 * kGenWarps, 3) k_gen_bwd(const __grid_cons
   }
 }
 
+// dL/dW for general irreps: work unit (canonical edge range r of kDwRange edges, output block q).
+// The range's geometry (harmonics, radial basis, sender, receiver) is staged once; then path by
+// path each lane runs its channel u over the range (gdwc_t: gw = g . sum C Y x per edge, and
+// sum_e R_b gw for the 8 basis functions) and writes its column of the range's partial sums,
+// part[r][b][column]. k_gen_dw_sum adds the ranges in a fixed order.
+constexpr int kDwRange = 128;
+
+__global__ void __launch_bounds__(32 * kGenWarps) k_gen_dw(const __grid_constant__ GenParams g, int n_edges,
+                                                           int n_ranges, const int* __restrict__ recv,
+                                                           const int* __restrict__ sender,
+                                                           const float* __restrict__ edge_vec,
+                                                           const float* __restrict__ x,
+                                                           const float* __restrict__ gout,
+                                                           float* __restrict__ part) {
+  extern __shared__ float smem[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  float* geo = smem + wib * (kDwRange * kGeoF + 2 * kDwRange);
+  int* sj = reinterpret_cast<int*>(geo + kDwRange * kGeoF);
+  int* si = sj + kDwRange;
+  const int n_items = n_ranges * g.n_out_groups;
+  const int stride = gridDim.x * kGenWarps;
+  for (int it = blockIdx.x * kGenWarps + wib; it < n_items; it += stride) {
+    const int r = it / g.n_out_groups;
+    const GenGroup& G = g.out_grp[it - r * g.n_out_groups];
+    const int e0 = r * kDwRange;
+    const int cnt = n_edges - e0 < kDwRange ? n_edges - e0 : kDwRange;
+    __syncwarp();   // the previous unit's staged rows have been read
+    for (int k = lane; k < cnt; k += 32) {
+      float Y[kY], R[kNumBasis], dR[kNumBasis], nv[3], inv_d;
+      edge_geometry(edge_vec, e0 + k, g.sh_lmax, g.inv_rc, Y, R, dR, nv, inv_d, false);
+#pragma unroll
+      for (int c = 0; c < kY; ++c) geo[k * kGeoF + c] = Y[c];
+#pragma unroll
+      for (int b = 0; b < kNumBasis; ++b) geo[k * kGeoF + kY + b] = R[b];
+      sj[k] = sender[e0 + k];
+      si[k] = recv[e0 + k];
+    }
+    __syncwarp();
+    float* pr = part + static_cast<size_t>(r) * kNumBasis * g.cols;
+    for (int pi = G.beg; pi < G.end; ++pi) {
+      const GenPath& P = g.p[g.order_out[pi]];
+      for (int u = lane; u < P.mul; u += 32) {
+        float acc8[kNumBasis];
+#pragma unroll
+        for (int b = 0; b < kNumBasis; ++b) acc8[b] = 0.0f;
+        etp_gen::gen_dw_chunk(P.tri, geo, sj, si, cnt, x + P.in_off + u, gout + P.out_off + u, g.dim_in, g.dim_out,
+                              P.mul, acc8);
+#pragma unroll
+        for (int b = 0; b < kNumBasis; ++b) pr[static_cast<size_t>(b) * g.cols + P.woff + u] = acc8[b];
+      }
+    }
+  }
+}
+
+// dW[o] = sum over ranges of part[r][o]: a block per 32 outputs, warp w adds the ranges w, w + 8,
+// ... in order, then warp 0 adds the 8 warp sums in order.
+__global__ void __launch_bounds__(256) k_gen_dw_sum(const float* __restrict__ part, int n_ranges, int n_out,
+                                                    float* __restrict__ dW) {
+  __shared__ float ws[8][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int o = blockIdx.x * 32 + lane;
+  float s = 0.0f;
+  if (o < n_out)
+    for (int r = w; r < n_ranges; r += 8) s += part[static_cast<size_t>(r) * n_out + o];
+  ws[w][lane] = s;
+  __syncthreads();
+  if (w == 0 && o < n_out) {
+    float t = ws[0][lane];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) t += ws[k][lane];
+    dW[o] = t;
+  }
+}
+
 // grad_edge_vec = sum of the input blocks' partials, in block order.
 __global__ void k_gen_sum_parts(const float* __restrict__ part, int n_groups, int n, float* __restrict__ out) {
   for (int v = blockIdx.x * blockDim.x + threadIdx.x; v < n; v += gridDim.x * blockDim.x) {
@@ -341,6 +415,35 @@ int gen_blocks(int n_nodes) {
 
 size_t general_backward_partials_bytes(const GenParams& g, int n_edges) {
   return g.n_in_groups > 1 ? align256(sizeof(float) * 3 * static_cast<size_t>(n_edges) * g.n_in_groups) : 0;
+}
+
+size_t general_weight_grad_bytes(const GenParams& g, int n_edges) {
+  const long long n_ranges = (static_cast<long long>(n_edges) + kDwRange - 1) / kDwRange;
+  return align256(sizeof(float) * static_cast<size_t>(n_ranges > 0 ? n_ranges : 1) * kNumBasis * g.cols);
+}
+
+etp_status launch_general_weight_grad(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
+                                      const int* sender, const float* edge_vec, const float* x,
+                                      const float* grad_out, float* grad_W, int* recv, float* part,
+                                      cudaStream_t s) {
+  const int n_out = kNumBasis * g.cols;
+  // columns of paths whose output block no unit visits do not exist: every path has a block
+  if (n_edges == 0) {
+    cudaError_t e = cudaMemsetAsync(grad_W, 0, sizeof(float) * n_out, s);
+    return e == cudaSuccess ? ETP_OK : cuda_status(e, "general weight gradient memset");
+  }
+  etp_status st = launch_recv_of_edge(row_ptr, n_nodes, n_edges, recv, s);
+  if (st != ETP_OK) return st;
+  const int n_ranges = (n_edges + kDwRange - 1) / kDwRange;
+  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(kDwRange * kGeoF + 2 * kDwRange);
+  cudaError_t e = cudaFuncSetAttribute(k_gen_dw, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return cuda_status(e, "general weight gradient smem attribute");
+  k_gen_dw<<<gen_blocks(n_ranges * g.n_out_groups), 32 * kGenWarps, smem, s>>>(g, n_edges, n_ranges, recv, sender,
+                                                                                edge_vec, x, grad_out, part);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "general weight gradient launch");
+  k_gen_dw_sum<<<(n_out + 31) / 32, 256, 0, s>>>(part, n_ranges, n_out, grad_W);
+  return cuda_status(cudaGetLastError(), "general weight gradient sum launch");
 }
 
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,

@@ -128,6 +128,11 @@ etp_status launch_weight_grad(const Ctx& c, int n_nodes, int n_edges, const int*
 // edge-gradient partials (general_backward_partials_bytes)
 constexpr int kGenMaxDim = 4096;   // floats per node row
 size_t general_backward_partials_bytes(const GenParams& g, int n_edges);
+size_t general_weight_grad_bytes(const GenParams& g, int n_edges);
+etp_status launch_general_weight_grad(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
+                                      const int* sender, const float* edge_vec, const float* x,
+                                      const float* grad_out, float* grad_W, int* recv, float* part,
+                                      cudaStream_t s);
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                   const int* sender, const float* edge_vec, const float* x, const float* W,
                                   float* out, cudaStream_t s);

@@ -625,6 +625,51 @@ def emit_general(out):
         for m3 in rows:
             out.append(f"  acc[{m3} * stride] += a{m3};")
         out.append("}")
+    # weight gradient over a chunk of staged edges: gw = sum_m3 g[m3] sum C Y x per edge, then
+    # acc8[b] += R_b gw (the channel's column of dL/dW)
+    for t, (l1, l2, l3) in enumerate(tri):
+        c = real_cg_any(l1, l2, l3)
+        groups = []
+        for m3 in range(2 * l3 + 1):
+            for m1 in range(2 * l1 + 1):
+                terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
+                if terms:
+                    groups.append((m3, m1, terms))
+        rows = sorted({m3 for m3, _, _ in groups})
+        out.append(f"__device__ __forceinline__ void gdwc_{t}(const float* geo, const int* sj, const int* si, int cnt,")
+        out.append("                                       const float* __restrict__ xu, const float* __restrict__ gu,")
+        out.append("                                       int dim_in, int dim_out, int stride, float* acc8) {")
+        out.append("  for (int k = 0; k < cnt; ++k) {")
+        out.append("    const float* Y = geo + k * kGenGeoF;")
+        out.append("    const float* x = xu + static_cast<size_t>(sj[k]) * dim_in;")
+        out.append("    const float* g = gu + static_cast<size_t>(si[k]) * dim_out;")
+        for m1 in range(2 * l1 + 1):
+            out.append(f"    const float x{m1} = x[{m1} * stride];")
+        out.append("    float gw = 0.0f;")
+        for m3 in rows:
+            row = [(m1, terms) for (a3, m1, terms) in groups if a3 == m3]
+            first = True
+            for m1, terms in row:
+                mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                if first:
+                    out.append(f"    float s{m3} = ({mexpr}) * x{m1};")
+                    first = False
+                else:
+                    out.append(f"    s{m3} = fmaf({mexpr}, x{m1}, s{m3});")
+            out.append(f"    gw = fmaf(g[{m3} * stride], s{m3}, gw);")
+        out.append("    #pragma unroll")
+        out.append("    for (int b = 0; b < 8; ++b) acc8[b] = fmaf(Y[25 + b], gw, acc8[b]);")
+        out.append("  }")
+        out.append("}")
+    out.append("__device__ __forceinline__ void gen_dw_chunk(int t, const float* geo, const int* sj, const int* si, int cnt,")
+    out.append("                                             const float* xu, const float* gu, int dim_in, int dim_out,")
+    out.append("                                             int stride, float* acc8) {")
+    out.append("  switch (t) {")
+    for t in range(len(tri)):
+        out.append(f"    case {t}: gdwc_{t}(geo, sj, si, cnt, xu, gu, dim_in, dim_out, stride, acc8); break;")
+    out.append("    default: break;")
+    out.append("  }")
+    out.append("}")
     out.append("__device__ __forceinline__ void gen_fwd_chunk(int t, const float* geo, const int* sj, int cnt,")
     out.append("                                              const float* xu, int dim_in, int stride, const float* wb,")
     out.append("                                              float* acc) {")

@@ -97,8 +97,8 @@ typedef struct {
  *    1 x 1 -> 1). W is [n_basis][cols] with path p's mul_p columns after the earlier paths'
  *    (the same as [n_basis][n_paths][C] when all blocks have C channels); node rows hold the
  *    blocks in string order, block b as [m][u] with mul_b channels. General handles support
- *    etp_forward, etp_forward_noalloc (no scratch needed) and etp_backward; the masked, weight
- *    gradient and radial-weight calls return ETP_ERR_UNSUPPORTED for them.
+ *    etp_forward, etp_forward_noalloc (no scratch needed), etp_backward and etp_backward_weights;
+ *    the masked and radial-weight calls return ETP_ERR_UNSUPPORTED for them.
  * Both need n_basis == 8 and r_cut > 0. Malformed strings -> ETP_ERR_IRREPS; anything else
  * outside these sets -> ETP_ERR_UNSUPPORTED. The path list is the enumeration described above. */
 etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_basis,
@@ -163,7 +163,10 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
  *   dL/dW[b][p][u] = sum_e R_b(d_e) sum_{m1,m3} x[send, l1, m1, u] (sum_m2 C Y_{l2 m2}) g[recv, l3, m3, u].
  * Runs over the canonical (receiver-sorted) order, with the channels on the lanes; partial sums
  * per range of edges are added in range order, so repeated calls give identical bits.
- * grad_W is overwritten (zero for a graph without edges). Uses the etp_workspace_bytes workspace. */
+ * grad_W is overwritten (zero for a graph without edges). Uses the etp_workspace_bytes workspace.
+ * For a general irreps handle grad_W has the W layout [n_basis][cols]; the kernel stages the
+ * geometry of 128 canonical edges at a time, runs each path's channels over them and writes one
+ * partial column per range; the ranges are added in order (also bit-reproducible). */
 /* Node-local product ladder of correlation order nu (FlashCart Fig. 3b and Fig. E1, path-reduced):
  *   B_1 = A,  B_{q+1}[l3, m3, u] = sum_{p=(l1,l2,l3)} W[q-1][p][u] sum_{m1,m2} C B_q[l1, m1, u] A[l2, m2, u],
  *   out = B_1 + ... + B_nu,
