@@ -500,8 +500,8 @@ etp_status etp_forward_masked(etp_handle h, int n_nodes, int n_edges, const int*
                               size_t workspace_bytes, void* stream) {
   etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_forward_masked");
   if (st != ETP_OK) return st;
-  if (h->c.general) {
-    set_error("etp_forward_masked: not implemented for general irreps handles");
+  if (h->c.general && h->c.n_paths > 32) {
+    set_error("etp_forward_masked: a 32-bit path mask covers at most 32 paths");
     return ETP_ERR_UNSUPPORTED;
   }
   if (!out || !aligned16(out) || (n_edges > 0 && !path_mask)) {
@@ -519,6 +519,9 @@ etp_status etp_forward_masked(etp_handle h, int n_nodes, int n_edges, const int*
     if (st != ETP_OK) return st;
   }
   if (n_nodes == 0) return ETP_OK;
+  if (h->c.general)
+    return launch_general_forward(h->c.gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, s,
+                                  n_edges > 0 ? path_mask : nullptr);
   void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
   st = tc::launch_forward_tc(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s,
                              n_edges > 0 ? path_mask : nullptr);
@@ -534,8 +537,8 @@ etp_status etp_backward_masked(etp_handle h, int n_nodes, int n_edges, const int
                                void* stream) {
   etp_status st = check_common(h, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, "etp_backward_masked");
   if (st != ETP_OK) return st;
-  if (h->c.general) {
-    set_error("etp_backward_masked: not implemented for general irreps handles");
+  if (h->c.general && h->c.n_paths > 32) {
+    set_error("etp_backward_masked: a 32-bit path mask covers at most 32 paths");
     return ETP_ERR_UNSUPPORTED;
   }
   if (!t_row_ptr || (n_edges > 0 && (!t_perm || !grad_out || !path_mask)) || (!grad_x && !grad_edge_vec)) {
@@ -557,6 +560,11 @@ etp_status etp_backward_masked(etp_handle h, int n_nodes, int n_edges, const int
     if (st != ETP_OK) return st;
   }
   if (n_nodes == 0) return ETP_OK;
+  if (h->c.general)
+    return launch_general_backward(h->c.gen, n_nodes, n_edges, row_ptr, edge_vec, t_row_ptr, t_perm, x, W,
+                                   grad_out, grad_x, grad_edge_vec, static_cast<int*>(workspace),
+                                   reinterpret_cast<float*>(static_cast<char*>(workspace) + ws_tc_offset(n_edges)),
+                                   s, n_edges > 0 ? path_mask : nullptr);
   if (n_edges == 0)   // nothing is sent: zero outputs from the kernel without edges
     return launch_backward(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, t_row_ptr, t_perm, x, W, grad_out,
                            grad_x, grad_edge_vec, static_cast<int*>(workspace), s);

@@ -85,12 +85,14 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_fwd(const __grid_constan
                                                             const float* __restrict__ edge_vec,
                                                             const float* __restrict__ x,
                                                             const float* __restrict__ W,
+                                                            const uint32_t* __restrict__ mask,
                                                             float* __restrict__ out) {
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  float* acc = smem + wib * (g.max_out_size + 32 * kGeoF + 32);
+  float* acc = smem + wib * (g.max_out_size + 32 * kGeoF + 64);
   float* geo = acc + g.max_out_size;
   int* sj = reinterpret_cast<int*>(geo + 32 * kGeoF);
+  unsigned* sm = reinterpret_cast<unsigned*>(sj + 32);
   const int n_items = n_nodes * g.n_out_groups;
   const int stride = gridDim.x * kGenWarps;
   for (int it = blockIdx.x * kGenWarps + wib; it < n_items; it += stride) {
@@ -108,6 +110,7 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_fwd(const __grid_constan
 #pragma unroll
         for (int b = 0; b < kNumBasis; ++b) geo[lane * kGeoF + kY + b] = R[b];
         sj[lane] = sender[c0 + lane];
+        if (mask) sm[lane] = mask[c0 + lane];
       }
       __syncwarp();
       const int cnt = e1 - c0 < 32 ? e1 - c0 : 32;
@@ -122,7 +125,8 @@ __global__ void __launch_bounds__(32 * kGenWarps) k_gen_fwd(const __grid_constan
 #pragma unroll
             for (int b = 0; b < kNumBasis; ++b) wb[b] = __ldg(W + static_cast<size_t>(b) * g.cols + P.woff + u);
             etp_gen::gen_fwd_chunk(P.tri, geo + r0 * kGeoF, sj + r0, rc, x + P.in_off + u, g.dim_in, P.mul, wb,
-                                   acc + (P.out_off - G.off) + u);
+                                   acc + (P.out_off - G.off) + u, mask ? sm + r0 : nullptr,
+                                   1u << (g.order_out[pi] & 31));
           }
         }
       }
@@ -166,15 +170,17 @@ __global__ void __launch_bounds__(32 * kGenWarps, 3) k_gen_bwd(const __grid_cons
                                                             const float* __restrict__ x,
                                                             const float* __restrict__ W,
                                                             const float* __restrict__ gout,
+                                                            const uint32_t* __restrict__ mask,
                                                             float* __restrict__ grad_x,
                                                             float* __restrict__ vec_out) {
   extern __shared__ float smem[];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  float* gx = smem + wib * (g.max_in_size + 32 * kGeoB + 32 * kRed + 64);
+  float* gx = smem + wib * (g.max_in_size + 32 * kGeoB + 32 * kRed + 96);
   float* geo = gx + g.max_in_size;
   float* red = geo + 32 * kGeoB;
   int* si = reinterpret_cast<int*>(red + 32 * kRed);
   int* se = si + 32;
+  unsigned* sm = reinterpret_cast<unsigned*>(se + 32);
   const bool wide = g.sh_lmax > 3;   // 25 + 8 values: one more than the scatter-reduction holds
   const int n_items = n_nodes * g.n_in_groups;
   const int stride = gridDim.x * kGenWarps;
@@ -206,6 +212,7 @@ __global__ void __launch_bounds__(32 * kGenWarps, 3) k_gen_bwd(const __grid_cons
         o[kY + 2 * kNumBasis + 3] = inv_d;
         si[lane] = recv[e];
         se[lane] = e;
+        sm[lane] = mask ? mask[e] : ~0u;
       }
       __syncwarp();
       const int cnt = t1 - c0 < 32 ? t1 - c0 : 32;
@@ -222,6 +229,7 @@ __global__ void __launch_bounds__(32 * kGenWarps, 3) k_gen_bwd(const __grid_cons
         for (int b = 0; b < kNumBasis; ++b) gR[b] = 0.0f;
         const float* gi = gout + static_cast<size_t>(si[k]) * g.dim_out;
         for (int pi = G.beg; pi < G.end; ++pi) {
+          if (!(sm[k] & (1u << (g.order_in[pi] & 31)))) continue;   // path off for this edge
           const GenPath& P = g.p[g.order_in[pi]];
           for (int u = lane; u < P.mul; u += 32) {
             float wb[kNumBasis];
@@ -448,7 +456,7 @@ etp_status launch_general_weight_grad(const GenParams& g, int n_nodes, int n_edg
 
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                   const int* sender, const float* edge_vec, const float* x, const float* W,
-                                  float* out, cudaStream_t s) {
+                                  float* out, cudaStream_t s, const uint32_t* path_mask) {
   (void)n_edges;
   if (n_nodes == 0) return ETP_OK;
   int covered = 0;
@@ -458,18 +466,19 @@ etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, 
     cudaError_t e = cudaMemsetAsync(out, 0, sizeof(float) * static_cast<size_t>(n_nodes) * g.dim_out, s);
     if (e != cudaSuccess) return cuda_status(e, "general forward memset");
   }
-  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.max_out_size + 32 * kGeoF + 32);
+  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.max_out_size + 32 * kGeoF + 64);
   cudaError_t e = cudaFuncSetAttribute(k_gen_fwd, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_status(e, "general forward smem attribute");
   k_gen_fwd<<<gen_blocks(n_nodes * g.n_out_groups), 32 * kGenWarps, smem, s>>>(g, n_nodes, row_ptr, sender, edge_vec,
-                                                                                x, W, out);
+                                                                                x, W, path_mask, out);
   return cuda_status(cudaGetLastError(), "general forward launch");
 }
 
 etp_status launch_general_backward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                    const float* edge_vec, const int* t_row_ptr, const int* t_perm,
                                    const float* x, const float* W, const float* grad_out, float* grad_x,
-                                   float* grad_edge_vec, int* recv, float* part, cudaStream_t s) {
+                                   float* grad_edge_vec, int* recv, float* part, cudaStream_t s,
+                                   const uint32_t* path_mask) {
   if (n_nodes == 0) return ETP_OK;
   if (n_edges > 0) {
     etp_status st = launch_recv_of_edge(row_ptr, n_nodes, n_edges, recv, s);
@@ -484,12 +493,12 @@ etp_status launch_general_backward(const GenParams& g, int n_nodes, int n_edges,
   }
   const bool split = grad_edge_vec && g.n_in_groups > 1 && n_edges > 0;
   float* vec_out = split ? part : grad_edge_vec;
-  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.max_in_size + 32 * kGeoB + 32 * kRed + 64);
+  const size_t smem = sizeof(float) * kGenWarps * static_cast<size_t>(g.max_in_size + 32 * kGeoB + 32 * kRed + 96);
   cudaError_t e = cudaFuncSetAttribute(k_gen_bwd, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return cuda_status(e, "general backward smem attribute");
   k_gen_bwd<<<gen_blocks(n_nodes * g.n_in_groups), 32 * kGenWarps, smem, s>>>(g, n_nodes, n_edges, t_row_ptr, t_perm,
-                                                                               recv, edge_vec, x, W, grad_out, grad_x,
-                                                                               vec_out);
+                                                                               recv, edge_vec, x, W, grad_out, path_mask,
+                                                                               grad_x, vec_out);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "general backward launch");
   if (split) {

@@ -135,11 +135,12 @@ etp_status launch_general_weight_grad(const GenParams& g, int n_nodes, int n_edg
                                       cudaStream_t s);
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                   const int* sender, const float* edge_vec, const float* x, const float* W,
-                                  float* out, cudaStream_t s);
+                                  float* out, cudaStream_t s, const uint32_t* path_mask = nullptr);
 etp_status launch_general_backward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                    const float* edge_vec, const int* t_row_ptr, const int* t_perm,
                                    const float* x, const float* W, const float* grad_out, float* grad_x,
-                                   float* grad_edge_vec, int* recv, float* part, cudaStream_t s);
+                                   float* grad_edge_vec, int* recv, float* part, cudaStream_t s,
+                                   const uint32_t* path_mask = nullptr);
 
 // ---- node-local product ladder (etp_product.cu)
 etp_status launch_node_ladder(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,

@@ -598,11 +598,12 @@ def emit_general(out):
                     groups.append((m3, m1, terms))
         out.append(f"__device__ __forceinline__ void gfwdc_{t}(const float* geo, const int* sj, int cnt,")
         out.append("                                        const float* __restrict__ xu, int dim_in, int stride,")
-        out.append("                                        const float* wb, float* acc) {")
+        out.append("                                        const float* wb, float* acc, const unsigned* mk, unsigned bit) {")
         rows = sorted({m3 for m3, _, _ in groups})
         for m3 in rows:
             out.append(f"  float a{m3} = 0.0f;")
         out.append("  for (int k = 0; k < cnt; ++k) {")
+        out.append("    if (mk && !(mk[k] & bit)) continue;   // path off for this edge")
         out.append("    const float* Y = geo + k * kGenGeoF;")
         out.append("    float w = 0.0f;")
         out.append("    #pragma unroll")
@@ -670,12 +671,13 @@ def emit_general(out):
     out.append("    default: break;")
     out.append("  }")
     out.append("}")
+    out.append("// mk: per-edge path masks of the chunk (null: every path on); bit: this path's bit")
     out.append("__device__ __forceinline__ void gen_fwd_chunk(int t, const float* geo, const int* sj, int cnt,")
     out.append("                                              const float* xu, int dim_in, int stride, const float* wb,")
-    out.append("                                              float* acc) {")
+    out.append("                                              float* acc, const unsigned* mk, unsigned bit) {")
     out.append("  switch (t) {")
     for t in range(len(tri)):
-        out.append(f"    case {t}: gfwdc_{t}(geo, sj, cnt, xu, dim_in, stride, wb, acc); break;")
+        out.append(f"    case {t}: gfwdc_{t}(geo, sj, cnt, xu, dim_in, stride, wb, acc, mk, bit); break;")
     out.append("    default: break;")
     out.append("  }")
     out.append("}")

@@ -781,14 +781,46 @@ def test_general_irreps_weight_grad_full_size(wls):
     assert abs(lhs - rhs) <= 1e-4 * max(1.0, abs(rhs))
 
 
+@pytest.mark.parametrize("irin,sh,irout", [("16x0e+16x1o+16x1e+16x2e+16x2o", 2, "16x0e+16x1o+16x1e+16x2e+16x2o"),
+                                          ("128x0e+64x1o+32x2e+32x3o", 3, "128x0e+64x1o+32x2e+32x3o")])
+def test_general_irreps_path_mask_parity(wls, irin, sh, irout):
+    """Per-edge path masks on general handles (at most 32 paths) against the oracle."""
+    wl = wls("tiny")
+    conv = etp.EdgeConv(irin, sh, irout, 8, float(wl.r_cut))
+    spec = ConvSpec(irin, sh, irout, 8, float(wl.r_cut))
+    x, W, gout = _general_inputs(spec, wl.n_nodes, 41)
+    g = _gpu_graph(wl)
+    ref_g = full_graph(wl)
+    n_p = len(spec.paths)
+    rng = np.random.default_rng(43)
+    mask = rng.integers(0, 1 << n_p, size=g.n_edges).astype(np.int64)
+    mask[: g.n_edges // 3] = (1 << n_p) - 1
+    md = torch.from_numpy(mask.astype(np.uint32).view(np.int32)).to(DEV)
+    xd, Wd, gd = (torch.from_numpy(a).to(DEV) for a in (x, W, gout))
+    out = conv.forward(g, xd, Wd, path_mask=md)
+    ref = conv_forward(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, path_mask=mask)
+    assert_irrep_blocks_close(_np(out), ref, spec, "out", f"{irin} masked forward")
+    gx, gv = conv.backward(g, xd, Wd, gd, path_mask=md)
+    rgx, rgv = conv_vjp(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, gout, path_mask=mask)
+    assert_irrep_blocks_close(_np(gx), rgx, spec, "in", f"{irin} masked grad_x")
+    assert_close_rel(_np(gv), rgv, f"{irin} masked grad_edge_vec")
+    # all bits set is the unmasked call, bit for bit
+    ones = torch.full((g.n_edges,), -1, dtype=torch.int32, device=DEV)
+    assert torch.equal(conv.forward(g, xd, Wd, path_mask=ones), conv.forward(g, xd, Wd))
+
+
 def test_general_irreps_unsupported_calls_refuse(wls):
     wl = wls("tiny")
-    conv = etp.EdgeConv("8x0e+8x1e", 1, "8x0e+8x1e", 8, float(wl.r_cut))
-    spec = ConvSpec("8x0e+8x1e", 1, "8x0e+8x1e", 8, float(wl.r_cut))
+    irr = "32x0e+32x1o+32x2e+32x3o+32x4e"      # 42 paths: more than a 32-bit mask holds
+    conv = etp.EdgeConv(irr, 4, irr, 8, float(wl.r_cut))
+    spec = ConvSpec(irr, 4, irr, 8, float(wl.r_cut))
     x, W, gout = _general_inputs(spec, wl.n_nodes, 5)
     g = _gpu_graph(wl)
     xd, Wd, gd = (torch.from_numpy(a).to(DEV) for a in (x, W, gout))
     mask = torch.ones(g.n_edges, dtype=torch.int32, device=DEV)
     with pytest.raises(etp.EtpError) as ei:
         conv.forward(g, xd, Wd, path_mask=mask)
+    assert ei.value.status == 3
+    with pytest.raises(etp.EtpError) as ei:
+        conv.radial_weights(g.edge_vec, Wd)
     assert ei.value.status == 3
