@@ -96,6 +96,9 @@ KERNEL_SOURCES = {
     "k_bwd_tc": ["etp_bwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_dw": ["etp_dw.cu", "etp_device.h", "generated/etp_paths.h"],
     "k_node_ladder": ["etp_product.cu", "etp_device.h", "generated/etp_paths.h"],
+    "k_gen_fwd": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
+    "k_gen_bwd": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
+    "k_gen_dw": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
 }
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised in
 # profiles/<kernel>_<workload>.md, keyed by a hash of the kernel's sources at capture time.
@@ -414,7 +417,8 @@ def run_gpu(args, rank, world, local_rank):
         return {"workload": f"{gen_irreps}, harmonics to l = 3, {wl.name} graph ({e} edges)",
                 "kernel": f"k_gen_{kind}", "ms_per_launch": round(ms, 5), "bound": "alu", "achieved": round(ach, 3),
                 "peak": round(fp32_peak, 2), "unit": "TFLOP/s", "frac": round(ach / fp32_peak, 4),
-                "edges_per_s": round(e / (ms * 1e-3), 1), "traffic": None}
+                "edges_per_s": round(e / (ms * 1e-3), 1),
+                "traffic": recorded_traffic(f"k_gen_{kind}", f"nequipl_{wl.name}")}
 
     line = {
         "metric": METRIC,
