@@ -103,9 +103,12 @@ KERNEL_SOURCES = {
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised in
 # profiles/<kernel>_<workload>.md, keyed by a hash of the kernel's sources at capture time.
 RECORDED_TRAFFIC = {
-    ("k_fwd_tc", "diamond1k"): (3857664 + 0, "2ef350fce27bf8a2"),
-    ("k_bwd_tc", "diamond1k"): (6545152 + 256, "fa34cf52cc7c6eaa"),
-    ("k_node_ladder", "ladder4096_l2"): (18898432 + 0, "6f03787ca5847418"),
+    ("k_fwd_tc", "diamond1k"): (3857920 + 0, "ea8f138b574dd70f"),
+    ("k_bwd_tc", "diamond1k"): (6545152 + 256, "467f958b73c2e96d"),
+    ("k_dw", "diamond1k"): (6419968 + 1024, "09ca90502fe891fa"),
+    ("k_node_ladder", "ladder4096_l2"): (18899200 + 0, "066bbc29265202a3"),
+    ("k_gen_fwd", "nequipl_diamond1k"): (4377344 + 0, "837463c03e03e26a"),
+    ("k_gen_bwd", "nequipl_diamond1k"): (7540480 + 0, "837463c03e03e26a"),
 }
 
 
