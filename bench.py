@@ -353,11 +353,29 @@ def run_gpu(args, rank, world, local_rank):
     out_h = torch.empty_like(bufs["out"], device="cpu").pin_memory()
     f_h = torch.empty((n, 3), dtype=torch.float32).pin_memory()
 
+    # the copies run on a second stream where the data flow allows: x, W and the cotangent travel
+    # while the neighbour list is built from the positions, and the forward output travels back
+    # while the backward runs
+    copy_stream = torch.cuda.Stream(device=dev)
+    in_d = [torch.empty_like(t, device=dev) for t in (pos_h, x_h, W_h, g_h)]
+
     def e2e_step():
-        pd, xd, Wd, gd = (t.to(dev, non_blocking=True) for t in (pos_h, x_h, W_h, g_h))
-        step(pd, xd, Wd, gd)
-        out_h.copy_(bufs["out"], non_blocking=True)
+        main = torch.cuda.current_stream(dev)
+        copy_stream.wait_stream(main)                  # the previous step is done with the buffers
+        in_d[0].copy_(pos_h, non_blocking=True)
+        with torch.cuda.stream(copy_stream):
+            for d_, h_ in zip(in_d[1:], (x_h, W_h, g_h)):
+                d_.copy_(h_, non_blocking=True)
+        gr_ = graph_step(in_d[0])
+        main.wait_stream(copy_stream)
+        conv_fwd(gr_, in_d[1], in_d[2])
+        copy_stream.wait_stream(main)
+        with torch.cuda.stream(copy_stream):
+            out_h.copy_(bufs["out"], non_blocking=True)
+        conv_bwd(gr_, in_d[1], in_d[2], in_d[3])
+        etp.forces(gr_, bufs["gv"][:gr_.n_edges], out=bufs["f"])
         f_h.copy_(bufs["f"], non_blocking=True)
+        main.wait_stream(copy_stream)
 
     for _ in range(2):
         e2e_step()
