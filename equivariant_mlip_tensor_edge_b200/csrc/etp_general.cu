@@ -12,9 +12,12 @@
 //             then, path by path, each lane runs its channel over the 32 edges with the path's W
 //             column and sums in registers. Fixed order (chunks, paths, edges): deterministic.
 //   backward: a warp per (sender, input block) over the transposed order; grad_x accumulated like
-//             the forward output; per edge, dL/dY and dL/dR_b summed over the lanes in a fixed
-//             butterfly and turned into the block's share of dL/dr_e by lane 0 (chain through the
-//             harmonics' gradient and dR/dd); the shares are added over the blocks in order.
+//             the forward output; per edge, dL/dY and dL/dR_b summed over the lanes by a fixed
+//             scatter-reduction, and once per 32 edges lane k turns edge k's sums into the block's
+//             share of dL/dr_e (chain through the harmonics' gradient and dR/dd); the shares are
+//             added over the blocks in order.
+//   dL/dW   : a warp per (range of 128 edges, output block): per path and channel, the sum over
+//             the range of R_b gw; the ranges' partial columns are added in order.
 #include <cstdint>
 #include <string>
 
@@ -435,7 +438,6 @@ etp_status launch_general_weight_grad(const GenParams& g, int n_nodes, int n_edg
                                       const float* grad_out, float* grad_W, int* recv, float* part,
                                       cudaStream_t s) {
   const int n_out = kNumBasis * g.cols;
-  // columns of paths whose output block no unit visits do not exist: every path has a block
   if (n_edges == 0) {
     cudaError_t e = cudaMemsetAsync(grad_W, 0, sizeof(float) * n_out, s);
     return e == cudaSuccess ? ETP_OK : cuda_status(e, "general weight gradient memset");
