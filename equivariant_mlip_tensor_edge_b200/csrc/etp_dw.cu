@@ -107,9 +107,12 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_dw(int n_edges, int C, 
     }
     __syncwarp();
     const int n = e_end - e0 < 32 ? e_end - e0 : 32;
+    // the sender row of edge k + 1 is requested before edge k's contraction (one edge ahead)
+    float xn[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) xn[c] = cu ? __ldg(x + static_cast<size_t>(sJ[wb][0]) * dim + c * C + u) : 0.0f;
     for (int k = 0; k < n; ++k) {
       const int i = sI[wb][k];
-      const int j = sJ[wb][k];
       if (i != cur_i) {
         cur_i = i;
 #pragma unroll
@@ -117,7 +120,12 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) k_dw(int n_edges, int C, 
       }
       float xv[D][1];
 #pragma unroll
-      for (int c = 0; c < D; ++c) xv[c][0] = cu ? __ldg(x + static_cast<size_t>(j) * dim + c * C + u) : 0.0f;
+      for (int c = 0; c < D; ++c) xv[c][0] = xn[c];
+      if (k + 1 < n) {
+        const int jn = sJ[wb][k + 1];
+#pragma unroll
+        for (int c = 0; c < D; ++c) xn[c] = cu ? __ldg(x + static_cast<size_t>(jn) * dim + c * C + u) : 0.0f;
+      }
       float Y[D], R[NB];
 #pragma unroll
       for (int c = 0; c < D; ++c) Y[c] = sY[wb][k][c];
