@@ -36,6 +36,7 @@ SIGNATURES = {
     "etp_create": (_i, [ctypes.c_char_p, _i, ctypes.c_char_p, _i, _f, ctypes.POINTER(_vp)]),
     "etp_destroy": (_i, [_vp]),
     "etp_get_info": (_i, [_vp, ctypes.POINTER(EtpInfo)]),
+    "etp_get_paths": (_i, [_vp, _ip, _i]),
     "etp_status_string": (ctypes.c_char_p, [_i]),
     "etp_last_error": (ctypes.c_char_p, []),
     "etp_workspace_bytes": (_sz, [_vp, _i, _i]),
@@ -229,6 +230,14 @@ class EdgeConv:
     @property
     def n_paths(self):
         return self.info["n_paths"]
+
+    @property
+    def paths(self):
+        """[(input block, l2, output block)] in W's column order."""
+        n = self.n_paths
+        buf = (ctypes.c_int * (3 * n))()
+        _check(load_library().etp_get_paths(self._h, buf, n), "etp_get_paths")
+        return [tuple(buf[3 * p:3 * p + 3]) for p in range(n)]
 
     def workspace_bytes(self, n_nodes, n_edges):
         return load_library().etp_workspace_bytes(self._h, n_nodes, n_edges)

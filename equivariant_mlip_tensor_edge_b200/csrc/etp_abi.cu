@@ -173,6 +173,9 @@ bool general_config(const std::vector<Block>& bin, int sh_lmax, const std::vecto
         }
         const int tri = etp_gen::kGenTriId[(A.l * 5 + l2) * 5 + B.l];
         g.p[n] = GenPath{in_off[a], out_off[b], cols, A.mul, tri};
+        c->path_blocks[n][0] = static_cast<short>(a);
+        c->path_blocks[n][1] = static_cast<short>(l2);
+        c->path_blocks[n][2] = static_cast<short>(b);
         cols += A.mul;
         nnz += etp_gen::kGenTriNnz[tri];
         s3 += 2 * B.l + 1;
@@ -296,6 +299,8 @@ etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out
     set_error("etp_create: path enumeration does not match the generated path tables");
     return ETP_ERR_UNSUPPORTED;
   }
+  for (int p = 0; p < c.n_paths; ++p)   // blocks are l = 0..L in order: block index = rank
+    for (int k = 0; k < 3; ++k) c.path_blocks[p][k] = static_cast<short>(ls[3 * p + k]);
   etp_ctx* h = new (std::nothrow) etp_ctx;
   if (!h) {
     set_error("etp_create: out of host memory");
@@ -305,6 +310,21 @@ etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out
   c.flop_bwd = 2 * (3 * c.cg_nnz + 2 * c.sum_2l3p1) * C;
   h->c = c;
   *out = h;
+  return ETP_OK;
+}
+
+etp_status etp_get_paths(etp_handle h, int* paths, int capacity) {
+  if (!h || (!paths && capacity > 0) || capacity < 0) {
+    set_error("etp_get_paths: NULL handle or bad buffer");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (capacity < h->c.n_paths) {
+    set_error("etp_get_paths: capacity " + std::to_string(capacity) + " below the " +
+              std::to_string(h->c.n_paths) + " paths");
+    return ETP_ERR_CAPACITY;
+  }
+  for (int p = 0; p < h->c.n_paths; ++p)
+    for (int k = 0; k < 3; ++k) paths[3 * p + k] = h->c.path_blocks[p][k];
   return ETP_OK;
 }
 

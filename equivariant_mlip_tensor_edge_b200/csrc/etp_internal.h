@@ -60,6 +60,7 @@ struct Ctx {
   int flop_bwd = 0;
   bool general = false;   // true: the table-driven kernels of etp_general.cu serve this handle
   GenParams gen;
+  short path_blocks[kGenMaxPaths][3] = {};   // host copy of the path list: (input block, l2, output block)
 };
 
 // Configuration behind a handle (NULL for a NULL handle).

@@ -110,6 +110,11 @@ etp_status etp_destroy(etp_handle h);
 /* Dimensions and path statistics of a handle (info: host pointer). */
 etp_status etp_get_info(etp_handle h, etp_info_t* info);
 
+/* The handle's path list, in the order W's columns use: paths[3 p + 0..2] = (input block index,
+ * l2, output block index) of path p, block indices counting from 0 in irreps-string order.
+ * paths: host array of at least 3 * capacity ints; capacity < n_paths -> ETP_ERR_CAPACITY. */
+etp_status etp_get_paths(etp_handle h, int* paths, int capacity);
+
 /* Static text for a status code, and the last detailed error message of this host thread. */
 const char* etp_status_string(etp_status s);
 const char* etp_last_error(void);

@@ -74,6 +74,9 @@ def test_info_matches_independent_path_enumeration(lmax, c):
     assert conv.info["dim_in"] == spec.dim_in == conv.info["dim_out"]
     assert conv.info["weight_numel"] == 8 * len(spec.paths) * c
     assert conv.info["flop_fwd"] == fc["fwd_tp"] and conv.info["flop_bwd"] == fc["bwd_tp"]
+    assert conv.paths == [tuple(p) for p in spec.paths]
+    buf = (ctypes.c_int * 3)()
+    assert etp.load_library().etp_get_paths(conv._h, buf, 1) == 6    # capacity below n_paths
     assert conv.workspace_bytes(100, 1000) >= 2 * 4 * 1000
 
 
@@ -95,6 +98,7 @@ def test_general_info_matches_independent_path_enumeration(irin, sh, irout):
     assert conv.info["weight_numel"] == 8 * spec.weight_numel
     assert conv.info["channels"] == (spec.channels or 0)
     assert conv.info["flop_fwd"] == fc["fwd_tp"] and conv.info["flop_bwd"] == fc["bwd_tp"]
+    assert conv.paths == [tuple(p) for p in spec.paths]
     assert etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x1o", 8, 5.0).info["general"] == 0
 
 
