@@ -105,7 +105,7 @@ KERNEL_SOURCES = {
 RECORDED_TRAFFIC = {
     ("k_fwd_tc", "diamond1k"): (3857920 + 0, "ea8f138b574dd70f"),
     ("k_bwd_tc", "diamond1k"): (6545152 + 256, "467f958b73c2e96d"),
-    ("k_dw", "diamond1k"): (6419968 + 1024, "09ca90502fe891fa"),
+    ("k_dw", "diamond1k"): (6418688 + 0, "342f85c428c1d6a6"),
     ("k_node_ladder", "ladder4096_l2"): (18899200 + 0, "066bbc29265202a3"),
     ("k_gen_fwd", "nequipl_diamond1k"): (4377344 + 0, "43e26cc213b58ccd"),
     ("k_gen_bwd", "nequipl_diamond1k"): (7540480 + 0, "43e26cc213b58ccd"),
