@@ -208,7 +208,12 @@ def forces(graph, grad_edge_vec, out=None):
 
 
 class EdgeConv:
-    """Handle for one convolution configuration (irreps, SH lmax, radial basis, cutoff)."""
+    """Handle for one convolution configuration (irreps, SH lmax, radial basis, cutoff).
+
+    Uniform irreps (C x (0e + 1o + ... + Le), SH lmax L <= 3) run on the tensor-core kernels;
+    anything else the library supports (per-block multiplicities, both parities, rank <= 4) on the
+    general kernels (``info["general"] == 1``), whose W is [n_basis, cols] in ``paths`` order.
+    """
 
     def __init__(self, irreps_in, sh_lmax, irreps_out, n_basis=8, r_cut=5.0):
         lib = load_library()

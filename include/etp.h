@@ -15,13 +15,17 @@
  *
  *   with C the real-basis Clebsch-Gordan coefficients, paths p = (l1, l2, l3) enumerated
  *   lexicographically over (input block, l2 = 0..sh_lmax, output block) with the triangle rule
- *   and parity p1 (-1)^l2 = p3, and "uvu" channel pairing (output channel = input channel).
+ *   and parity p1 (-1)^l2 = p3, and "uvu" channel pairing (output channel = input channel, so a
+ *   path joins blocks of equal multiplicity only; see etp_create for general irreps).
  *
  * Layouts (all row-major, 32-bit):
  *   node features x, out, grad_x, grad_out : [n_nodes][dim], dim = C (L+1)^2; the row holds the
  *       blocks l = 0..L in order, block l is [m = -l..l][u = 0..C-1] (channels contiguous):
- *       element (l, m, u) sits at (l*l + l + m) * C + u.
- *   W           : [n_basis][n_paths][C]
+ *       element (l, m, u) sits at (l*l + l + m) * C + u. General irreps handles: the blocks in
+ *       irreps-string order, block b as [m][u] with its own multiplicity (dim_in / dim_out in
+ *       etp_info_t).
+ *   W           : [n_basis][n_paths][C]; general irreps handles: [n_basis][cols], path p's mul_p
+ *                 columns after the earlier paths' (etp_get_paths gives the order)
  *   edge arrays : receiver-sorted CSR. row_ptr [n_nodes+1], sender [n_edges], edge_vec [n_edges][3]
  *                 (float32 r_e). Canonical edge order: (receiver, sender, S0, S1, S2).
  *   transposed  : t_row_ptr [n_nodes+1] (edges per sender), t_perm [n_edges]: the edge ids in

@@ -123,3 +123,19 @@ def test_null_arguments_rejected_without_cuda(lib):
     assert lib.etp_forces(-1, 0, None, None, None, None, None, None) == 1
     assert lib.etp_neighbors(None, -1, None, None, 1.0, 0, None, None, None, None, None, None, None, None, 0,
                              None) == 1
+
+
+def test_general_workspace_covers_every_scratch():
+    """General handles: receiver map + validation scratch + the larger of the edge-gradient shares
+    (3 floats per edge and input block) and the weight gradient's partial columns (8 x cols per
+    range of 128 edges)."""
+    irr = "128x0e+64x1o+32x2e+32x3o"
+    conv = etp.EdgeConv(irr, 3, irr, 8, 5.0)
+    spec = ConvSpec(irr, 3, irr, 8, 5.0)
+    for n_nodes, n_edges in ((10, 0), (1000, 89156), (5, 129)):
+        nb = conv.workspace_bytes(n_nodes, n_edges)
+        in_blocks = len({bi for bi, _, _ in spec.paths})
+        ranges = max(1, -(-n_edges // 128))
+        need = 4 * n_edges + 4 * (n_edges + 1) + max(12 * n_edges * in_blocks if in_blocks > 1 else 0,
+                                                       4 * 8 * spec.weight_numel * ranges)
+        assert nb >= need, (n_nodes, n_edges, nb, need)
