@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 import equivariant_mlip_tensor_edge_b200 as etp
@@ -139,3 +140,47 @@ def test_general_workspace_covers_every_scratch():
         need = 4 * n_edges + 4 * (n_edges + 1) + max(12 * n_edges * in_blocks if in_blocks > 1 else 0,
                                                        4 * 8 * spec.weight_numel * ranges)
         assert nb >= need, (n_nodes, n_edges, nb, need)
+
+
+def _irreps_str(blocks):
+    return "+".join(f"{m}x{l}{'e' if p > 0 else 'o'}" for m, l, p in blocks)
+
+
+def test_create_matches_the_oracle_path_set_on_random_irreps():
+    """etp_create on random irreps strings (seeded): when the oracle finds paths and the sizes fit,
+    the handle exists and its path list, dimensions and weight columns equal the oracle's; otherwise
+    the call is refused as unsupported. No other outcome."""
+    rng = np.random.default_rng(2024)
+    lib = etp.load_library()
+    seen_general = seen_uniform = seen_refused = 0
+    for _ in range(300):
+        def blocks():
+            k = int(rng.integers(1, 6))
+            return [(int(rng.choice([1, 3, 4, 8, 16, 32])), int(rng.integers(0, 5)), int(rng.choice([1, -1])))
+                    for _ in range(k)]
+        bin_, bout = blocks(), (blocks() if rng.random() < 0.5 else None)
+        bout = bout if bout is not None else list(bin_)
+        sh = int(rng.integers(0, 5))
+        irin, irout = _irreps_str(bin_), _irreps_str(bout)
+        spec = ConvSpec(irin, sh, irout, 8, 5.0)
+        h = ctypes.c_void_p()
+        st = lib.etp_create(irin.encode(), sh, irout.encode(), 8, 5.0, ctypes.byref(h))
+        fits = (len(spec.paths) >= 1 and len(spec.paths) <= 128 and spec.dim_in <= 4096 and spec.dim_out <= 4096
+                and len(bin_) <= 16 and len(bout) <= 16)
+        if not fits:
+            assert st == 3, (irin, sh, irout, st)
+            seen_refused += 1
+            continue
+        assert st == 0, (irin, sh, irout, st, lib.etp_last_error())
+        info = etp.EtpInfo()
+        assert lib.etp_get_info(h, ctypes.byref(info)) == 0
+        buf = (ctypes.c_int * (3 * len(spec.paths)))()
+        assert lib.etp_get_paths(h, buf, len(spec.paths)) == 0
+        got = [tuple(buf[3 * p:3 * p + 3]) for p in range(len(spec.paths))]
+        assert got == [tuple(p) for p in spec.paths]
+        assert (info.dim_in, info.dim_out, info.n_paths) == (spec.dim_in, spec.dim_out, len(spec.paths))
+        assert info.weight_numel == 8 * spec.weight_numel
+        seen_general += info.general
+        seen_uniform += 1 - info.general
+        lib.etp_destroy(h)
+    assert seen_general > 50 and seen_refused > 5
