@@ -824,3 +824,22 @@ def test_general_irreps_unsupported_calls_refuse(wls):
     with pytest.raises(etp.EtpError) as ei:
         conv.radial_weights(g.edge_vec, Wd)
     assert ei.value.status == 3
+
+
+def test_general_irreps_autograd_function(wls):
+    """The autograd wrapper on a general handle: x, edge-vector and W gradients equal the ABI calls."""
+    wl = wls("tiny")
+    irr = "4x0e+3x1o+3x1e+4x2e"
+    conv = etp.EdgeConv(irr, 2, irr, 8, float(wl.r_cut))
+    spec = ConvSpec(irr, 2, irr, 8, float(wl.r_cut))
+    x, W, gout = _general_inputs(spec, wl.n_nodes, 12)
+    g = _gpu_graph(wl)
+    fn = etp.edge_conv_function()
+    xt = torch.from_numpy(x).to(DEV).requires_grad_(True)
+    vt = g.edge_vec.clone().requires_grad_(True)
+    Wt = torch.from_numpy(W).to(DEV).requires_grad_(True)
+    gd = torch.from_numpy(gout).to(DEV)
+    (fn.apply(conv, g, xt, vt, Wt) * gd).sum().backward()
+    gx, gv = conv.backward(g, xt.detach(), Wt.detach(), gd)
+    assert torch.equal(xt.grad, gx) and torch.equal(vt.grad, gv)
+    assert torch.equal(Wt.grad, conv.backward_weights(g, xt.detach(), gd).reshape(Wt.shape))
