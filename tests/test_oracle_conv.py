@@ -371,3 +371,109 @@ def test_flop_counts_formulae(tiny):
     assert fc["radial_proj"] == 2 * 8 * 4 * c
     nnz = sum(int(np.count_nonzero(cg_real(*tiny["spec"].path_ls(p)))) for p in range(4))
     assert fc["nnz"] == nnz
+
+
+# ----------------------------------------------------------------- forces and periodic images
+
+def _edges_from_positions(pos, nb, cell):
+    """Edge vectors rebuilt from atom positions with the neighbour set held fixed:
+    r_e = pos[sender] - pos[receiver] + S cell (float64)."""
+    shift = nb["shift"].astype(np.float64)
+    sv = shift @ (np.zeros((3, 3)) if cell is None else np.asarray(cell, dtype=np.float64))
+    return pos[nb["sender"]] - pos[nb["receiver"]] + sv
+
+
+def test_forces_are_minus_the_position_gradient(tiny):
+    """F = -dL/dpos by central differences in the atom positions (neighbour set fixed), for
+    L = <g, out>: pins the sign of forces_from_edge_grads and which end of an edge gets +g."""
+    spec, nb, wl = tiny["spec"], tiny["nb"], tiny["wl"]
+    pos = wl.pos.astype(np.float64)
+
+    def loss(p):
+        vec = _edges_from_positions(p, nb, wl.cell)
+        return (conv_forward(spec, tiny["row_ptr"], nb["sender"], vec, tiny["x"], tiny["W"]) * tiny["g"]).sum()
+
+    vec = _edges_from_positions(pos, nb, wl.cell)
+    _, gv = conv_vjp(spec, tiny["row_ptr"], nb["sender"], vec, tiny["x"], tiny["W"], tiny["g"])
+    f = forces_from_edge_grads(gv, nb["receiver"], nb["sender"], wl.n_nodes)
+    h = 1e-6
+    rng = np.random.default_rng(5)
+    for _ in range(8):
+        k, a = int(rng.integers(wl.n_nodes)), int(rng.integers(3))
+        pp, pm = pos.copy(), pos.copy()
+        pp[k, a] += h
+        pm[k, a] -= h
+        fd = (loss(pp) - loss(pm)) / (2 * h)
+        assert abs(f[k, a] + fd) < 1e-6 * max(1.0, abs(fd)), (k, a, f[k, a], fd)
+    # a flipped convention (receiver and sender swapped) gives -F and fails the check above
+    assert np.abs(f).max() > 1e-3
+
+
+def test_torque_of_the_forces_vanishes(tiny):
+    """sum_i pos_i x F_i = 0 for a rotation-invariant loss of a non-periodic system: with
+    scalar-only features, L = <a, out_0e> does not change when all positions rotate."""
+    spec, nb, wl = tiny["spec"], tiny["nb"], tiny["wl"]
+    assert wl.cell is None
+    rng = np.random.default_rng(3)
+    g = np.zeros_like(tiny["g"])
+    g[:, spec.out_slice(0)] = rng.standard_normal((wl.n_nodes, spec.channels))
+    xs = np.zeros_like(tiny["x"])
+    xs[:, spec.in_slice(0)] = tiny["x"][:, spec.in_slice(0)]
+    pos = wl.pos.astype(np.float64)
+    vec = _edges_from_positions(pos, nb, None)
+    _, gv = conv_vjp(spec, tiny["row_ptr"], nb["sender"], vec, xs, tiny["W"], g)
+    f = forces_from_edge_grads(gv, nb["receiver"], nb["sender"], wl.n_nodes)
+    assert np.abs(f.sum(0)).max() < 1e-12 * max(1.0, np.abs(f).max())
+    torque = np.cross(pos, f).sum(0)
+    assert np.abs(torque).max() < 1e-10 * max(1.0, np.abs(f).max() * np.abs(pos).max())
+    # and it is a real check: with vector features the loss is not invariant and the torque is not 0
+    _, gv2 = conv_vjp(spec, tiny["row_ptr"], nb["sender"], vec, tiny["x"], tiny["W"], tiny["g"])
+    f2 = forces_from_edge_grads(gv2, nb["receiver"], nb["sender"], wl.n_nodes)
+    assert np.abs(np.cross(pos, f2).sum(0)).max() > 1e-6
+
+
+def _cell_case(case):
+    """The periodic cells of the GPU image-scan tests (same seeds and shapes)."""
+    if case == "orthorhombic_small":
+        cell, n, seed, pbc = np.diag([7.1, 7.6, 8.3]), 40, 21, (True, True, True)
+    elif case == "triclinic":
+        cell, n, seed, pbc = [[11.0, 0.0, 0.0], [3.1, 10.5, 0.0], [-1.7, 2.2, 12.0]], 60, 22, (True, True, True)
+    else:
+        cell, n, seed, pbc = np.diag([12.0, 12.5, 30.0]), 50, 23, (True, True, False)
+    rng = np.random.default_rng(seed)
+    frac = rng.random((n, 3))
+    cell = np.asarray(cell, dtype=np.float64)
+    return (frac @ cell).astype(np.float32), cell, pbc, np.float32(5.0)
+
+
+@pytest.mark.parametrize("case", ["orthorhombic_small", "triclinic", "slab"])
+def test_neighbors_against_an_all_images_scan(case):
+    """The oracle scans |S_a| <= ceil(r_cut / plane spacing) images per periodic axis; an
+    independent scan of every image with |S_a| <= 3 (far more than any pair at r < 5 A can use in
+    these cells) must find exactly the same (receiver, sender, S) triples and vectors."""
+    pos32, cell, pbc, rc = _cell_case(case)
+    nb = neighbors(pos32, cell, pbc, rc)
+    pos = pos32.astype(np.float64)
+    n = len(pos)
+    rng3 = [range(-3, 4) if p else range(0, 1) for p in pbc]
+    found = {}
+    for s0 in rng3[0]:
+        for s1 in rng3[1]:
+            for s2 in rng3[2]:
+                sv = np.array([s0, s1, s2], dtype=np.float64) @ cell
+                r = pos[None, :, :] - pos[:, None, :] + sv          # [receiver, sender, 3]
+                d = np.sqrt((r * r).sum(-1))
+                keep = d < float(rc)
+                if (s0, s1, s2) == (0, 0, 0):
+                    keep &= ~np.eye(n, dtype=bool)
+                for i, j in zip(*np.nonzero(keep)):
+                    found[(int(i), int(j), s0, s1, s2)] = r[i, j]
+    got = {(int(i), int(j), *map(int, s)): v for i, j, s, v in
+           zip(nb["receiver"], nb["sender"], nb["shift"], nb["edge_vec"])}
+    assert set(got) == set(found)
+    for k, v in got.items():
+        assert np.abs(v.astype(np.float64) - found[k]).max() < 1e-5
+    # the small cell really has several images of one pair (the case the range rule is for)
+    if case == "orthorhombic_small":
+        pairs = [(k[0], k[1]) for k in got]
+        assert len(pairs) > len(set(pairs))
