@@ -31,6 +31,12 @@ METRIC = "edges/sec for TP conv fwd and fwd+bwd (fp32), % of HBM/FP32 roofline"
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 FALLBACK_HBM_GBS = 6650.0
+KERNEL_WARMUP = 20
+KERNEL_REPS = 200
+# the other workloads (besides the diamond1k headline) and their oracle sample sizes (receivers),
+# chosen so that each float64 sample takes a few seconds on one host core
+OTHER_WORKLOADS = ("tiny", "sweep1", "sweep2", "sweep3", "diamond8k", "melt32k")
+ORACLE_SAMPLE = {"tiny": 32, "sweep1": 256, "sweep2": 48, "sweep3": 12, "diamond8k": 8, "melt32k": 16}
 
 
 # ---------------------------------------------------------------- peaks and counts
@@ -91,7 +97,9 @@ def algorithmic_counts(info, n_nodes, n_edges):
 # ---------------------------------------------------------------- recorded DRAM traffic
 
 CSRC = os.path.join(ROOT, "equivariant_mlip_tensor_edge_b200", "csrc")
+FWD_KERNEL = "k_fwd_cx"     # the default forward for l_max <= 2, C <= 128
 KERNEL_SOURCES = {
+    "k_fwd_cx": ["etp_fwd_cx.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_fwd_tc": ["etp_fwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_bwd_tc": ["etp_bwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_dw": ["etp_dw.cu", "etp_device.h", "generated/etp_paths.h"],
@@ -273,10 +281,14 @@ def run_gpu(args, rank, world, local_rank):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # > 126 MB L2
 
     def timed(fn, k, host_ahead=False):
-        """Mean device time of fn over k calls, L2 flushed before each. host_ahead: a device-side
-        sleep after the flush lets the host enqueue fn entirely before the first event, so the
-        time is the kernels' alone, not the host's launch latency."""
-        total = 0.0
+        """Mean device time of fn over k calls (the step's contract: exactly k timed calls), L2
+        flushed before each. host_ahead: a device-side sleep after the flush lets the host enqueue
+        fn entirely before the first event, so the time is the kernels' alone, not the host's
+        launch latency."""
+        return statistics.fmean(event_times(fn, k, host_ahead))
+
+    def event_times(fn, k, host_ahead):
+        out = []
         for _ in range(k):
             flush.fill_(1.0)
             if host_ahead:
@@ -286,8 +298,15 @@ def run_gpu(args, rank, world, local_rank):
             fn()
             b.record()
             b.synchronize()
-            total += a.elapsed_time(b)
-        return total / k
+            out.append(a.elapsed_time(b))
+        return out
+
+    def kernel_ms(fn):
+        """Median device time of one call over KERNEL_REPS calls after KERNEL_WARMUP untimed ones,
+        L2 flushed before each call."""
+        for _ in range(KERNEL_WARMUP):
+            fn()
+        return statistics.median(event_times(fn, KERNEL_REPS, True))
 
     # warm-up
     for _ in range(args.warmup):
@@ -307,13 +326,11 @@ def run_gpu(args, rank, world, local_rank):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    # per-kernel timings on the same stream (dominant kernels), same flush discipline
-    reps = max(args.steps, 5)
-    ms_fwd = timed(lambda: conv_fwd(gr, x, W), reps, host_ahead=True)
-    ms_bwd = timed(lambda: conv_bwd(gr, x, W, gout), reps, host_ahead=True)
-    ms_graph = timed(lambda: graph_step(pos), reps)
-    ms_dw = timed(lambda: conv.backward_weights(gr, x, gout, grad_W=bufs["dw"], workspace=bufs["ws"]), reps,
-                  host_ahead=True)
+    # per-kernel timings on the same stream (median of KERNEL_REPS calls after KERNEL_WARMUP)
+    ms_fwd = kernel_ms(lambda: conv_fwd(gr, x, W))
+    ms_bwd = kernel_ms(lambda: conv_bwd(gr, x, W, gout))
+    ms_graph = kernel_ms(lambda: graph_step(pos))
+    ms_dw = kernel_ms(lambda: conv.backward_weights(gr, x, gout, grad_W=bufs["dw"], workspace=bufs["ws"]))
     # node-local product ladder: 4096 nodes x 128 channels, correlation order 3, the workload's rank
     lad = dict(n=4096, c=128, nu=3, lmax=wl.lmax)
     gen = torch.Generator().manual_seed(1234)
@@ -323,7 +340,7 @@ def run_gpu(args, rank, world, local_rank):
     lad_out = torch.empty_like(lad_A)
     for _ in range(3):
         etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out)
-    ms_ladder = timed(lambda: etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out), reps, host_ahead=True)
+    ms_ladder = kernel_ms(lambda: etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out))
     # general irreps: NequIP-L channel counts on the same graph (table-driven kernels)
     gen_irreps = "128x0e+64x1o+32x2e+32x3o"
     gconv = etp.EdgeConv(gen_irreps, 3, gen_irreps, wl.n_basis, float(wl.r_cut))
@@ -344,9 +361,16 @@ def run_gpu(args, rank, world, local_rank):
     g_dw = torch.empty((gi["n_basis"], gi["weight_numel"] // gi["n_basis"]), device=dev)
     gen_dw = lambda: gconv.backward_weights(gr, g_x, g_g, grad_W=g_dw, workspace=g_ws)
     gen_dw()
-    ms_gen_fwd = timed(gen_fwd, reps, host_ahead=True)
-    ms_gen_bwd = timed(gen_bwd, reps, host_ahead=True)
-    ms_gen_dw = timed(gen_dw, reps, host_ahead=True)
+    ms_gen_fwd = kernel_ms(gen_fwd)
+    ms_gen_bwd = kernel_ms(gen_bwd)
+    ms_gen_dw = kernel_ms(gen_dw)
+    # every other workload of the benchmark set: forward (and backward) edges/s and roofline
+    # fractions, each with its own bounded float64 oracle sample on the host
+    others = {}
+    if not args.headline_only:
+        for name in OTHER_WORKLOADS:
+            others[name] = measure_workload(name, dev, kernel_ms, fp32_peak_tflops(measured_peaks()[0].get(
+                "sm_max_mhz", 1965.0)), with_oracle=(world == 1 and not args.no_cpu_baseline))
     clocks = sampler.stop() if rank == 0 else None
 
     # end to end through the public API with host buffers (copies inside the timed region)
@@ -400,12 +424,12 @@ def run_gpu(args, rank, world, local_rank):
     def roof(kind, ms):
         flop = cnt[f"{kind}_flop"]
         ach = flop / (ms * 1e-3) / 1e12
-        kernel = {"bwd": "k_bwd_tc", "fwd": "k_fwd_tc", "dw": "k_dw"}[kind]
+        kernel = {"bwd": "k_bwd_tc", "fwd": FWD_KERNEL, "dw": "k_dw"}[kind]
         return {"bound": "alu", "achieved": round(ach, 3), "peak": round(fp32_peak, 2), "unit": "TFLOP/s",
                 "frac": round(ach / fp32_peak, 4), "traffic": recorded_traffic(kernel, wl.name),
                 "kernel": kernel,
                 "timed": {"bwd": "the whole etp_backward call (k_bprep, k_recv_of_edge, k_bwd_tc, k_sum_units)",
-                          "fwd": "the whole etp_forward call (k_prep, k_fwd_tc)",
+                          "fwd": f"the whole etp_forward call (k_cx_prep, {FWD_KERNEL})",
                           "dw": "the whole etp_backward_weights call (k_recv_of_edge, k_dw, k_dw_sum)"}[kind],
                 "peak_source": f"derived: 148 SM x 128 FP32 lanes x 2 x {sm_max:.0f} MHz ({peak_kind} sm_max_mhz)",
                 "ms_per_launch": round(ms, 5),
@@ -461,6 +485,7 @@ def run_gpu(args, rank, world, local_rank):
         "fwd_edges_per_s": round(total_edges / (ms_fwd * 1e-3), 1),
         "conv_fwd_bwd_edges_per_s": round(total_edges / ((ms_fwd + ms_bwd) * 1e-3), 1),
         "ms_fwd": round(ms_fwd, 5), "ms_bwd": round(ms_bwd, 5), "ms_graph": round(ms_graph, 5),
+        "kernel_timing": f"median of {KERNEL_REPS} calls after {KERNEL_WARMUP} warm-up, L2 flushed before each",
         "roofline": roof(dominant, ms_bwd if dominant == "bwd" else ms_fwd),
         "roofline_fwd": roof("fwd", ms_fwd),
         "ms_weight_grad": round(ms_dw, 5),
@@ -469,6 +494,7 @@ def run_gpu(args, rank, world, local_rank):
         "general_irreps_fwd": general_roof(ms_gen_fwd, "fwd"),
         "general_irreps_bwd": general_roof(ms_gen_bwd, "bwd"),
         "general_irreps_dw": general_roof(ms_gen_dw, "dw"),
+        "workloads": others,
         "e2e": {"value": round(total_edges / (ms_e2e * 1e-3), 1), "unit": "edges/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": launches_per_step(info, n) * args.steps,
@@ -477,6 +503,99 @@ def run_gpu(args, rank, world, local_rank):
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline(wl, budget_s=args.cpu_budget)
     return line
+
+
+# ---------------------------------------------------------------- other workloads
+
+def measure_workload(name, dev, kernel_ms, fp32_peak, with_oracle=True):
+    """Forward (and, except for the forward-only rank sweeps, backward) of one workload: graph build
+    time, per-call device times, edges/s and FP32 roofline fractions of the whole calls."""
+    import torch
+
+    import equivariant_mlip_tensor_edge_b200 as etp
+    import workloads
+
+    wl = workloads.make(name)
+    conv = etp.EdgeConv(wl.irreps, wl.lmax, wl.irreps, wl.n_basis, float(wl.r_cut))
+    info = conv.info
+    x = torch.from_numpy(wl.features()).to(dev)
+    W = torch.from_numpy(wl.weights(conv.n_paths)).to(dev)
+    if wl.given_receiver is not None:
+        recv = torch.from_numpy(wl.given_receiver).to(dev)
+        send = torch.from_numpy(wl.given_sender).to(dev)
+        vec = torch.from_numpy(wl.given_edge_vec).to(dev)
+        build = lambda: etp.build_csr(wl.n_nodes, recv, send, vec)
+        graph_kind = "CSR from the given edge list"
+    else:
+        pos = torch.from_numpy(wl.pos).to(dev)
+        build = lambda: etp.neighbors(pos, float(wl.r_cut), cell=wl.cell, pbc=wl.pbc)
+        graph_kind = "neighbour list + CSR"
+    gr = build()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    gr = build()
+    torch.cuda.synchronize()
+    ms_graph = 1000.0 * (time.perf_counter() - t0)
+    e = gr.n_edges
+    ws = torch.empty(max(conv.workspace_bytes(wl.n_nodes, e), 1), dtype=torch.uint8, device=dev)
+    out = torch.empty((wl.n_nodes, info["dim_out"]), device=dev)
+    ms_fwd = kernel_ms(lambda: conv.forward(gr, x, W, out=out, workspace=ws))
+    cnt = algorithmic_counts(info, wl.n_nodes, e)
+    ent = {"n_nodes": wl.n_nodes, "n_edges": e, "irreps": wl.irreps, "sh_lmax": wl.lmax,
+           "ms_graph_wall": round(ms_graph, 3), "graph": graph_kind,
+           "ms_fwd": round(ms_fwd, 5), "fwd_edges_per_s": round(e / (ms_fwd * 1e-3), 1),
+           "roofline_fwd_frac": round(cnt["fwd_flop"] / (ms_fwd * 1e-3) / 1e12 / fp32_peak, 4)}
+    if not name.startswith("sweep"):
+        g = torch.from_numpy(wl.cotangent()).to(dev)
+        gx = torch.empty((wl.n_nodes, info["dim_in"]), device=dev)
+        gv = torch.empty((e, 3), device=dev)
+        ms_bwd = kernel_ms(lambda: conv.backward(gr, x, W, g, grad_x=gx, grad_vec=gv, workspace=ws))
+        ent.update({"ms_bwd": round(ms_bwd, 5),
+                    "fwd_bwd_edges_per_s": round(e / ((ms_fwd + ms_bwd) * 1e-3), 1),
+                    "roofline_bwd_frac": round(cnt["bwd_flop"] / (ms_bwd * 1e-3) / 1e12 / fp32_peak, 4)})
+    ent["roofline_peak"] = {"unit": "TFLOP/s", "value": round(fp32_peak, 2), "bound": "alu"}
+    if with_oracle:
+        ent["cpu_baseline"] = oracle_workload_sample(wl, ORACLE_SAMPLE[name], backward=not name.startswith("sweep"))
+    return ent
+
+
+def oracle_workload_sample(wl, n_recv, backward=True):
+    """The float64 oracle, as it stands, on n_recv sampled receivers of the workload (one BLAS
+    thread): their neighbour rows (or given edges), the forward, and the VJP."""
+    import numpy as np
+    from threadpoolctl import threadpool_limits
+
+    from oracle.conv import ConvSpec, conv_forward, conv_vjp
+    from oracle.graph import neighbors
+
+    spec = ConvSpec(wl.irreps, wl.lmax, wl.irreps, wl.n_basis, float(wl.r_cut))
+    x, W = wl.features(), wl.weights(len(spec.paths))
+    n_recv = min(n_recv, wl.n_nodes)
+    sample = sorted(np.random.default_rng(0).choice(wl.n_nodes, size=n_recv, replace=False).tolist())
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        if wl.given_receiver is not None:
+            order = np.lexsort((wl.given_sender, wl.given_receiver))
+            r, s_, v = wl.given_receiver[order], wl.given_sender[order], wl.given_edge_vec[order]
+            keep = np.isin(r, sample)
+            r, s_, v = r[keep], s_[keep], v[keep]
+        else:
+            rows = neighbors(wl.pos, wl.cell, wl.pbc, wl.r_cut, receivers=sample)
+            r, s_, v = rows["receiver"], rows["sender"], rows["edge_vec"]
+        rp = np.zeros(wl.n_nodes + 1, dtype=np.int64)
+        np.add.at(rp, np.asarray(r) + 1, 1)
+        rp = np.cumsum(rp)
+        conv_forward(spec, rp, s_, v, x, W, receivers=sample)
+        if backward:
+            conv_vjp(spec, rp, s_, v, x, W, wl.cotangent())
+        dt = time.perf_counter() - t0
+    edges = len(s_)
+    return {"value": round(edges / dt, 1), "unit": "edges/s", "cores": 1, "host_cores": os.cpu_count(),
+            "kind": "oracle",
+            "sample": f"{n_recv} of {wl.n_nodes} receivers ({edges} edges): "
+                      f"{'neighbour rows' if wl.given_receiver is None else 'given edges'}, forward"
+                      f"{', VJP' if backward else ''} in float64 numpy on one BLAS thread, {dt:.2f} s",
+            "seconds": round(dt, 3)}
 
 
 # ---------------------------------------------------------------- oracle (CPU) timing
@@ -513,7 +632,8 @@ def cpu_baseline(wl, budget_s=15.0, steps=1):
         for _ in range(steps):
             edges += _oracle_sample_step(wl, sample)
         dt = time.perf_counter() - t0
-    return {"value": round(edges / dt, 1), "unit": "edges/s", "cores": 1, "kind": "oracle",
+    return {"value": round(edges / dt, 1), "unit": "edges/s", "cores": 1, "host_cores": os.cpu_count(),
+            "kind": "oracle",
             "sample": f"{n_s} of {wl.n_nodes} receivers ({edges // steps} edges): neighbour rows, forward, VJP, "
                       f"forces in float64 numpy, {steps} step(s), {dt:.1f} s",
             "seconds": round(dt, 3)}
@@ -546,6 +666,7 @@ def main():
     ap.add_argument("--workload", default="diamond1k")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--headline-only", action="store_true", help="skip the per-workload entries")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

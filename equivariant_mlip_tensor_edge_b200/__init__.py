@@ -53,6 +53,8 @@ SIGNATURES = {
     "etp_graph_workspace_bytes": (_sz, [_i, _i]),
     "etp_neighbors": (_i, [_vp, _i, _dp, _ip, _f, _i, _ip, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "etp_build_csr": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "etp_get_status": (_i, [_vp, _vp, _ip]),
+    "etp_status_word": (_ip, [_vp]),
 }
 
 _lib = None
@@ -246,6 +248,13 @@ class EdgeConv:
 
     def workspace_bytes(self, n_nodes, n_edges):
         return load_library().etp_workspace_bytes(self._h, n_nodes, n_edges)
+
+    def check_status(self, device=None):
+        """Synchronise the current stream and raise if a kernel of an earlier call on this handle
+        gave up a bounded pipeline wait (the code is cleared)."""
+        code = ctypes.c_int(0)
+        stream = _stream(device) if device is not None else None
+        _check(load_library().etp_get_status(self._h, stream, ctypes.byref(code)), "etp_get_status")
 
     def _workspace(self, n_nodes, n_edges, device, workspace):
         torch = _torch()

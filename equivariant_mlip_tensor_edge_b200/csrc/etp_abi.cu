@@ -14,6 +14,51 @@ struct etp_ctx {
   etp::Ctx c;
 };
 
+namespace {
+
+// Gives the handle its sticky status word: pinned host memory mapped into the device address space
+// where a device is present (the kernels store their timeout codes there), plain host memory
+// otherwise (no kernel can run then). Returns false on failure (message set).
+bool attach_status_word(etp_ctx* h) {
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e == cudaSuccess && ndev > 0) {
+    void* p = nullptr;
+    e = cudaHostAlloc(&p, 64, cudaHostAllocMapped | cudaHostAllocPortable);
+    void* d = nullptr;
+    if (e == cudaSuccess) e = cudaHostGetDevicePointer(&d, p, 0);
+    if (e != cudaSuccess) {
+      if (p) cudaFreeHost(p);
+      etp::cuda_status(e, "etp_create: pinned status word");
+      return false;
+    }
+    *static_cast<volatile int*>(p) = 0;
+    h->c.status = static_cast<int*>(p);
+    h->c.status_dev = static_cast<int*>(d);
+    h->c.status_mapped = true;
+    return true;
+  }
+  cudaGetLastError();   // no device: clear the runtime's error state
+  void* p = std::calloc(1, 64);
+  if (!p) {
+    etp::set_error("etp_create: out of host memory");
+    return false;
+  }
+  h->c.status = static_cast<int*>(p);
+  h->c.status_dev = nullptr;
+  h->c.status_mapped = false;
+  return true;
+}
+
+void release_status_word(etp_ctx* h) {
+  if (!h || !h->c.status) return;
+  if (h->c.status_mapped) cudaFreeHost(h->c.status);
+  else std::free(h->c.status);
+  h->c.status = nullptr;
+}
+
+}  // namespace
+
 namespace etp {
 
 static thread_local std::string g_last_error;
@@ -27,6 +72,30 @@ etp_status cuda_status(cudaError_t e, const char* what) {
   set_error(std::string(what) + ": " + cudaGetErrorString(e));
   return ETP_ERR_CUDA;
 }
+
+etp_status read_status(const Ctx& c, cudaStream_t s, const char* who) {
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e, who);
+  const int code = c.status ? *reinterpret_cast<volatile int*>(c.status) : 0;
+  if (code != 0) {
+    set_error(std::string(who) + ": a bounded pipeline wait gave up (code " + std::to_string(code) +
+              "); the output is incomplete");
+    return ETP_ERR_CUDA;
+  }
+  return ETP_OK;
+}
+
+// Entry gate of every compute call: a code left in the handle's status word by an earlier call's
+// kernel fails the call until etp_get_status has read and cleared it.
+static etp_status status_gate(const Ctx& c, const char* who) {
+  const int code = c.status ? *reinterpret_cast<volatile int*>(c.status) : 0;
+  if (code == 0) return ETP_OK;
+  set_error(std::string(who) + ": a kernel of an earlier call on this handle gave up a bounded pipeline wait (code " +
+            std::to_string(code) + "); outputs since then may be incomplete; etp_get_status reads and clears it");
+  return ETP_ERR_CUDA;
+}
+
+etp_status gate(etp_handle h, const char* who) { return h ? status_gate(h->c, who) : ETP_OK; }
 
 namespace {
 
@@ -283,6 +352,10 @@ etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out
       set_error("etp_create: unsupported irreps (" + why + ")");
       return ETP_ERR_UNSUPPORTED;
     }
+    if (!attach_status_word(h)) {
+      delete h;
+      return ETP_ERR_CUDA;
+    }
     *out = h;
     return ETP_OK;
   }
@@ -309,6 +382,10 @@ etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out
   c.flop_fwd = 2 * (c.cg_nnz + c.sum_2l3p1) * C;
   c.flop_bwd = 2 * (3 * c.cg_nnz + 2 * c.sum_2l3p1) * C;
   h->c = c;
+  if (!attach_status_word(h)) {
+    delete h;
+    return ETP_ERR_CUDA;
+  }
   *out = h;
   return ETP_OK;
 }
@@ -329,7 +406,31 @@ etp_status etp_get_paths(etp_handle h, int* paths, int capacity) {
 }
 
 etp_status etp_destroy(etp_handle h) {
+  release_status_word(h);
   delete h;
+  return ETP_OK;
+}
+
+int* etp_status_word(etp_handle h) { return h ? h->c.status : nullptr; }
+
+etp_status etp_get_status(etp_handle h, void* stream, int* code) {
+  if (!h) {
+    set_error("etp_get_status: NULL handle");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (h->c.status_mapped) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e, "etp_get_status: stream synchronisation");
+  }
+  volatile int* w = reinterpret_cast<volatile int*>(h->c.status);
+  const int v = w ? *w : 0;
+  if (w) *w = 0;
+  if (code) *code = v;
+  if (v != 0) {
+    set_error("etp_get_status: a bounded pipeline wait gave up (code " + std::to_string(v) +
+              "); outputs of the calls since the previous check may be incomplete");
+    return ETP_ERR_CUDA;
+  }
   return ETP_OK;
 }
 
@@ -374,23 +475,29 @@ size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
   const size_t w = weight_grad_workspace_bytes(h->c, n_edges);
   const size_t cmw = cm::workspace_bytes(h->c);
+  const size_t cxw = cx::workspace_bytes(h->c);
   size_t m = f > b ? f : b;
   m = m > w ? m : w;
-  return ws_tc_offset(n_edges) + (m > cmw ? m : cmw);
+  m = m > cmw ? m : cmw;
+  return ws_tc_offset(n_edges) + (m > cxw ? m : cxw);
 }
 
-// Forward kernels: the edge-major tensor-core kernel by default. ETP_FORWARD=channel selects the
-// channel-major kernel where it applies (l_max <= 2, C in {32, 64, 128}; faster on graphs with
-// irregular degrees, slower on the regular ones) and ETP_FORWARD=generic the all-FP32 one. Every
-// kernel is tested.
-static bool use_tc_forward() {
+// Forward kernels. By default the channel-major path-subset kernel (etp_fwd_cx.cu) where it
+// applies (l_max <= 2, C <= 128), else the edge-major tensor-core kernel. ETP_FORWARD=edge selects
+// the edge-major kernel, ETP_FORWARD=channel the single-subset channel-major kernel (l_max <= 2,
+// C in {32, 64, 128}) and ETP_FORWARD=generic the all-FP32 one. Every kernel is tested.
+static bool forward_env_is(const char* name) {
   const char* v = std::getenv("ETP_FORWARD");
-  return !(v && std::strcmp(v, "generic") == 0);
+  return v && std::strcmp(v, name) == 0;
 }
 
-static bool use_cm_forward(const Ctx& c) {
+static bool use_tc_forward() { return !forward_env_is("generic"); }
+
+static bool use_cm_forward(const Ctx& c) { return cm::supported(c) && forward_env_is("channel"); }
+
+static bool use_cx_forward(const Ctx& c) {
   const char* v = std::getenv("ETP_FORWARD");
-  return cm::supported(c) && v && std::strcmp(v, "channel") == 0;
+  return cx::supported(c) && (!v || v[0] == 0 || std::strcmp(v, "default") == 0);
 }
 
 // Likewise for the backward: ETP_BACKWARD=generic selects the all-FP32 kernel.
@@ -423,7 +530,7 @@ static etp_status check_common(etp_handle h, int n_nodes, int n_edges, const int
     set_error(std::string(who) + ": x and W must be 16-byte aligned");
     return ETP_ERR_INVALID_ARG;
   }
-  return ETP_OK;
+  return status_gate(h->c, who);
 }
 
 static bool validate_requested() {
@@ -459,6 +566,11 @@ etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_pt
       return ETP_ERR_INVALID_ARG;
     }
     void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
+    if (use_cx_forward(h->c)) {
+      st = cx::launch(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);
+      if (st == ETP_OK && validate_requested()) st = cx::status(h->c, tcws, s);
+      return st;
+    }
     if (use_cm_forward(h->c)) {
       st = cm::launch(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);
       if (st == ETP_OK && validate_requested()) st = cm::status(h->c, tcws, s);
@@ -620,6 +732,7 @@ etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const in
     set_error("etp_backward_weights: workspace missing or smaller than etp_workspace_bytes()");
     return ETP_ERR_INVALID_ARG;
   }
+  if (status_gate(h->c, "etp_backward_weights") != ETP_OK) return ETP_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (validate_requested() && n_edges > 0) {
     int* scratch = reinterpret_cast<int*>(static_cast<char*>(workspace) + ws_scratch_offset(n_edges));
@@ -674,6 +787,7 @@ etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, 
     set_error("etp_radial_weights: not implemented for general irreps handles");
     return ETP_ERR_UNSUPPORTED;
   }
+  if (status_gate(h->c, "etp_radial_weights") != ETP_OK) return ETP_ERR_CUDA;
   if (n_edges == 0) return ETP_OK;
   return launch_radial_weights(h->c, n_edges, edge_vec, W, w_out, static_cast<cudaStream_t>(stream));
 }

@@ -163,11 +163,9 @@ __device__ __forceinline__ void tmem_ld16x(uint32_t taddr, float* v) {
 
 // Pre-split weights for the backward's pass width: wt[unit][pass][hl][canonical NCOL x 8].
 template <int L>
-__global__ void k_bprep(const float* __restrict__ W, int C, int n_units, float* __restrict__ wt,
-                        int* __restrict__ err) {
+__global__ void k_bprep(const float* __restrict__ W, int C, int n_units, float* __restrict__ wt) {
   using G = BCfg<L>;
   constexpr int K = G::K;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
   const int per_pass = 2 * G::NCOL * 8;
   const int total = n_units * G::NPASS * per_pass;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
@@ -224,7 +222,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
   uint64_t* sfree = rready + 1;
   uint64_t* wload = sfree + 1;
   uint64_t* wfree = wload + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(wfree + 2);
+  uint64_t* drainb = wfree + 2;   // final commit of the producer (abort-safe drain)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drainb + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* rp = reinterpret_cast<int*>(smem + G::OFF_G);
   float* Atile = reinterpret_cast<float*>(smem + G::OFF_A);   // [tile][4][128 x 8]
@@ -258,6 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
     mbar_init(wload + 1, 1);
     mbar_init(wfree + 0, 1);
     mbar_init(wfree + 1, 1);
+    mbar_init(drainb, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -271,12 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  bool drained = true;   // false: issued tensor-core work did not finish; TMEM is then not released
 
   if (warp == kQuads) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_tf32(NCOL);
-      uint32_t titem = 0, n_setup = 0, n_loads = 0;
+      uint32_t titem = 0, n_setup = 0, n_loads = 0, n_issued = 0;
       int cached_rg = -1, cached_round = -1;
       bool ok = true;
       auto load_w = [&](int g, uint32_t n) -> bool {
@@ -285,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
         if (n >= 2 && !mbar_wait(wfree + wb, ((n >> 1) - 1) & 1, abort_flag, a.err, 31)) return false;
         mbar_expect_tx(wload + wb, G::WBUF);
         bulk_g2s(Wbuf + wb * (G::WBUF / 4), a.wt + static_cast<size_t>(unit) * (G::WBUF / 4), G::WBUF, wload + wb);
+        ++n_issued;
         return true;
       };
       if (g_beg < g_end) ok = load_w(g_beg, 0);
@@ -331,9 +333,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
         mma_commit(wfree + wb);
         if (ok && g + 1 < g_end) ok = load_w(g + 1, n_loads);
       }
-      if (n_loads > 0) mbar_wait(wfree + ((n_loads - 1) & 1), ((n_loads - 1) >> 1) & 1, abort_flag, a.err, 35);
+      // drain, ignoring the abort flag: one more commit tracks every MMA issued so far, and the
+      // weight load issued for a group that was never consumed may still be in flight
+      mma_commit(drainb);
+      bool dr = mbar_wait_drain(drainb, 0);
+      if (dr && n_issued > n_loads)
+        dr = mbar_wait_drain(wload + ((n_issued - 1) & 1), ((n_issued - 1) >> 1) & 1);
+      if (!dr) {
+        report_code(a.err, 35);
+        *abort_flag = 1;
+        drained = false;
+      }
     }
-    __syncwarp();
+    drained = __shfl_sync(kFull, drained ? 1 : 0, 0) != 0;
   } else {
     // ---------------------------------------------------------------- consumers
     const int q = warp;
@@ -601,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kQuads) {
+  if (warp == kQuads && drained) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
@@ -622,7 +634,7 @@ int bnum_sms() {
 template <int L>
 size_t bws_bytes(int channels, int n_edges) {
   const int n_units = (channels + kUnitC - 1) / kUnitC;
-  size_t b = align256(static_cast<size_t>(n_units) * BCfg<L>::WBUF) + 256;
+  size_t b = align256(static_cast<size_t>(n_units) * BCfg<L>::WBUF);
   if (n_units > 1) b += align256(sizeof(float) * 3 * static_cast<size_t>(n_units) * n_edges);
   return b;
 }
@@ -636,10 +648,8 @@ etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, c
   char* p = static_cast<char*>(ws);
   float* wt = reinterpret_cast<float*>(p);
   p += align256(static_cast<size_t>(n_units) * G::WBUF);
-  int* err = reinterpret_cast<int*>(p);
-  p += 256;
   float* part = n_units > 1 ? reinterpret_cast<float*>(p) : grad_vec;
-  k_bprep<L><<<32, 256, 0, s>>>(W, c.channels, n_units, wt, err);
+  k_bprep<L><<<32, 256, 0, s>>>(W, c.channels, n_units, wt);
   if (n_edges > 0) {
     int blocks = (n_edges + 255) / 256;
     if (blocks > 8 * bnum_sms()) blocks = 8 * bnum_sms();
@@ -668,7 +678,7 @@ etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, c
   a.grad_x = grad_x;
   a.gpart = grad_vec ? part : nullptr;
   a.n_edges = n_edges;
-  a.err = err;
+  a.err = c.status_dev;
   long long grid = bnum_sms();
   const long long n_rg = (n_nodes + kQuads - 1) / kQuads;
   const long long min_grid = (n_rg + G::MAXRG - 3) / (G::MAXRG - 2);
@@ -688,12 +698,6 @@ etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, c
   return ETP_OK;
 }
 
-template <int L>
-int* bstatus_word(const Ctx& c, void* ws) {
-  const int n_units = (c.channels + kUnitC - 1) / kUnitC;
-  return reinterpret_cast<int*>(static_cast<char*>(ws) + align256(static_cast<size_t>(n_units) * BCfg<L>::WBUF));
-}
-
 }  // namespace
 
 size_t backward_tc_workspace_bytes(const Ctx& c, int n_edges) {
@@ -705,17 +709,8 @@ size_t backward_tc_workspace_bytes(const Ctx& c, int n_edges) {
 }
 
 etp_status backward_tc_status(const Ctx& c, const void* ws, cudaStream_t s) {
-  void* w = const_cast<void*>(ws);
-  const int* err = c.lmax == 1 ? bstatus_word<1>(c, w) : (c.lmax == 2 ? bstatus_word<2>(c, w) : bstatus_word<3>(c, w));
-  int code = 0;
-  cudaError_t e = cudaMemcpyAsync(&code, err, sizeof(int), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_status(e, "backward status read");
-  if (code != 0) {
-    set_error("tensor-core backward: pipeline wait exceeded its limit (code " + std::to_string(code) + ")");
-    return ETP_ERR_CUDA;
-  }
-  return ETP_OK;
+  (void)ws;
+  return read_status(c, s, "tensor-core backward");
 }
 
 etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const float* edge_vec,

@@ -98,9 +98,8 @@ struct CmArgs {
 // W^T blocks: row r of block blk is (path Lay::path[g][blk], channel 32 sl + r % 32) with
 // quadrant r / 32 = NSL g + sl; tf32 hi / lo in canonical K-major order. Clears the status word.
 template <int L, int C>
-__global__ void k_cm_prep(const float* __restrict__ W, float* __restrict__ wa, int* __restrict__ err) {
+__global__ void k_cm_prep(const float* __restrict__ W, float* __restrict__ wa) {
   using G = CmCfg<L, C>;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
   const int total = G::NBLK * 2 * 128 * 8;
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < total; i += gridDim.x * blockDim.x) {
     const int blk = i / (2 * 1024);
@@ -562,17 +561,11 @@ size_t cm_ws_bytes() {
 }
 
 template <int L, int C>
-int* cm_status_word(void* ws) {
-  return reinterpret_cast<int*>(static_cast<char*>(ws) + align256(static_cast<size_t>(CmCfg<L, C>::NBLK) * 2 * 4096));
-}
-
-template <int L, int C>
 etp_status cm_launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
                      const float* edge_vec, const float* x, const float* W, float* out, void* ws, cudaStream_t s) {
   using G = CmCfg<L, C>;
   float* wa = static_cast<float*>(ws);
-  int* err = cm_status_word<L, C>(ws);
-  k_cm_prep<L, C><<<16, 256, 0, s>>>(W, wa, err);
+  k_cm_prep<L, C><<<16, 256, 0, s>>>(W, wa);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "channel-major forward prep");
   e = cudaFuncSetAttribute(k_fwd_cm<L, C>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM);
@@ -588,7 +581,7 @@ etp_status cm_launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr,
   a.x = x;
   a.wa = wa;
   a.out = out;
-  a.err = err;
+  a.err = c.status_dev;
   k_fwd_cm<L, C><<<cm_num_sms(), kThreads, G::SMEM, s>>>(a);
   return cuda_status(cudaGetLastError(), "channel-major forward launch");
 }
@@ -615,15 +608,6 @@ size_t cm_ws_c(int channels) {
   }
 }
 
-template <int L>
-int* cm_err_c(int channels, void* ws) {
-  switch (channels) {
-    case 32: return cm_status_word<L, 32>(ws);
-    case 64: return cm_status_word<L, 64>(ws);
-    default: return cm_status_word<L, 128>(ws);
-  }
-}
-
 }  // namespace
 
 bool supported(const Ctx& c) {
@@ -644,17 +628,8 @@ etp_status launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, co
 }
 
 etp_status status(const Ctx& c, const void* ws, cudaStream_t s) {
-  void* w = const_cast<void*>(ws);
-  const int* err = c.lmax == 1 ? cm_err_c<1>(c.channels, w) : cm_err_c<2>(c.channels, w);
-  int code = 0;
-  cudaError_t e = cudaMemcpyAsync(&code, err, sizeof(int), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_status(e, "channel-major forward status read");
-  if (code != 0) {
-    set_error("channel-major forward: pipeline wait exceeded its limit (code " + std::to_string(code) + ")");
-    return ETP_ERR_CUDA;
-  }
-  return ETP_OK;
+  (void)ws;
+  return read_status(c, s, "channel-major forward");
 }
 
 }  // namespace cm

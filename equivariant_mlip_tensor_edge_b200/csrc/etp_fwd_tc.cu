@@ -140,13 +140,11 @@ __device__ __forceinline__ int group_tiles(const GroupInfo& gi, int round) {
 }
 
 // Per call: wt[unit][pass][hl][canonical NCOL x 8] (row n = K p' + k: W[b][p'][16 unit + K pass + k],
-// tf32 hi / lo) and the cleared status word.
+// tf32 hi / lo).
 template <int L>
-__global__ void k_prep(const float* __restrict__ W, int C, int n_units, float* __restrict__ wt,
-                       int* __restrict__ err) {
+__global__ void k_prep(const float* __restrict__ W, int C, int n_units, float* __restrict__ wt) {
   using G = Cfg<L>;
   constexpr int K = G::K;
-  if (blockIdx.x == 0 && threadIdx.x == 0) *err = 0;
   const int tid = blockIdx.x * blockDim.x + threadIdx.x;
   const int nthr = gridDim.x * blockDim.x;
   const int per_pass = 2 * G::NCOL * 8;
@@ -182,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   uint64_t* sfree = rready + 1;
   uint64_t* wload = sfree + 1;    // [2]
   uint64_t* wfree = wload + 2;    // [2]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(wfree + 2);
+  uint64_t* drainb = wfree + 2;   // final commit of the producer (abort-safe drain)
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drainb + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* rp = reinterpret_cast<int*>(smem + G::OFF_G);
   float* Atile = reinterpret_cast<float*>(smem + G::OFF_A);     // [SMAX][hl][128 x 8 canonical]
@@ -216,6 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
     mbar_init(wload + 1, 1);
     mbar_init(wfree + 0, 1);
     mbar_init(wfree + 1, 1);
+    mbar_init(drainb, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -229,11 +229,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  bool drained = true;   // false: issued tensor-core work did not finish; TMEM is then not released
 
   if (warp == kQuads) {
     // ---------------------------------------------------------------- producer warp
     constexpr uint32_t idesc = idesc_tf32(NCOL);
-    uint32_t titem = 0, n_setup = 0, n_loads = 0;
+    uint32_t titem = 0, n_setup = 0, n_loads = 0, n_issued = 0;
     int cached_rg = -1, cached_round = -1;
     bool ok = true;
     // weight slices of the k-th group of this CTA go to buffer k & 1; the next group's load is
@@ -245,6 +246,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
         if (n >= 2 && !mbar_wait(wfree + wb, ((n >> 1) - 1) & 1, abort_flag, a.err, 11)) return false;
         mbar_expect_tx(wload + wb, G::WBUF);
         bulk_g2s(Wbuf + wb * (G::WBUF / 4), a.wt + static_cast<size_t>(unit) * (G::WBUF / 4), G::WBUF, wload + wb);
+        ++n_issued;
       }
       return true;
     };
@@ -296,10 +298,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
       if (ok && g + 1 < g_end) ok = load_w(g + 1, n_loads);
       ok = __shfl_sync(kFull, ok ? 1 : 0, 0) != 0;
     }
-    // drain: the last commit covers every MMA this CTA issued
-    if (lane == 0 && n_loads > 0)
-      mbar_wait(wfree + ((n_loads - 1) & 1), ((n_loads - 1) >> 1) & 1, abort_flag, a.err, 15);
-    __syncwarp();
+    // drain, ignoring the abort flag: one more commit tracks every MMA issued so far, and the weight
+    // load issued for a group that was never consumed may still be in flight
+    if (lane == 0) {
+      mma_commit(drainb);
+      bool dr = mbar_wait_drain(drainb, 0);
+      if (dr && n_issued > n_loads)
+        dr = mbar_wait_drain(wload + ((n_issued - 1) & 1), ((n_issued - 1) >> 1) & 1);
+      if (!dr) {
+        report_code(a.err, 15);
+        *abort_flag = 1;
+        drained = false;
+      }
+    }
+    drained = __shfl_sync(kFull, drained ? 1 : 0, 0) != 0;
   } else {
     // ---------------------------------------------------------------- consumer warps
     const int q = warp;
@@ -508,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_tc(Args a) {
   // teardown: every thread reaches this barrier exactly once
   tc_fence_before();
   __syncthreads();
-  if (warp == kQuads) {
+  if (warp == kQuads && drained) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
   }
@@ -526,7 +538,7 @@ int num_sms() {
   return g_sms;
 }
 
-// Workspace: [wt][status word]
+// Workspace: [wt]
 template <int L>
 size_t wt_bytes(int channels) {
   const int n_units = (channels + kUnitC - 1) / kUnitC;
@@ -536,12 +548,7 @@ size_t wt_bytes(int channels) {
 template <int L>
 size_t ws_bytes(int channels, int n_nodes) {
   (void)n_nodes;
-  return wt_bytes<L>(channels) + 256;
-}
-
-template <int L>
-int* status_word(const Ctx& c, void* ws) {
-  return reinterpret_cast<int*>(static_cast<char*>(ws) + wt_bytes<L>(c.channels));
+  return wt_bytes<L>(channels);
 }
 
 template <int L>
@@ -550,8 +557,7 @@ etp_status launch(const Ctx& c, int n_nodes, const int* row_ptr, const int* send
   using G = Cfg<L>;
   const int n_units = (c.channels + kUnitC - 1) / kUnitC;
   float* wt = static_cast<float*>(ws);
-  int* err = status_word<L>(c, ws);
-  k_prep<L><<<32, 256, 0, s>>>(W, c.channels, n_units, wt, err);
+  k_prep<L><<<32, 256, 0, s>>>(W, c.channels, n_units, wt);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "forward prep");
   e = a_mask ? cudaFuncSetAttribute(k_fwd_tc<L, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, G::SMEM)
@@ -571,7 +577,7 @@ etp_status launch(const Ctx& c, int n_nodes, const int* row_ptr, const int* send
   a.wt = wt;
   a.mask = a_mask;
   a.out = out;
-  a.err = err;
+  a.err = c.status_dev;
   // enough CTAs that no CTA spans more than MAXRG receiver groups (row-pointer cache size)
   long long grid = num_sms();
   const long long n_rg = (n_nodes + kQuads - 1) / kQuads;
@@ -593,20 +599,10 @@ size_t forward_tc_workspace_bytes(const Ctx& c, int n_nodes) {
   }
 }
 
-// Reads the pipeline status word of the last tensor-core forward that used this workspace
-// (synchronises the stream). Nonzero = a bounded wait gave up (the output is incomplete).
+// Synchronises the stream and reads the handle's status word (nonzero: a bounded wait gave up).
 etp_status forward_tc_status(const Ctx& c, const void* ws, cudaStream_t s) {
-  void* w = const_cast<void*>(ws);
-  const int* err = c.lmax == 1 ? status_word<1>(c, w) : (c.lmax == 2 ? status_word<2>(c, w) : status_word<3>(c, w));
-  int code = 0;
-  cudaError_t e = cudaMemcpyAsync(&code, err, sizeof(int), cudaMemcpyDeviceToHost, s);
-  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return cuda_status(e, "forward status read");
-  if (code != 0) {
-    set_error("tensor-core forward: pipeline wait exceeded its limit (code " + std::to_string(code) + ")");
-    return ETP_ERR_CUDA;
-  }
-  return ETP_OK;
+  (void)ws;
+  return read_status(c, s, "tensor-core forward");
 }
 
 etp_status launch_forward_tc(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,

@@ -59,6 +59,12 @@ struct Ctx {
   int flop_fwd = 0;       // FP32 flop per edge of the forward / backward contraction
   int flop_bwd = 0;
   bool general = false;   // true: the table-driven kernels of etp_general.cu serve this handle
+  // Sticky pipeline status word: pinned host memory mapped into the device address space (status
+  // for the host, status_dev for kernels; the same address under unified addressing). A kernel
+  // whose bounded wait gives up stores its code there; every later call on the handle reports it.
+  int* status = nullptr;
+  int* status_dev = nullptr;
+  bool status_mapped = false;
   GenParams gen;
   short path_blocks[kGenMaxPaths][3] = {};   // host copy of the path list: (input block, l2, output block)
 };
@@ -69,6 +75,10 @@ const Ctx* ctx_of(etp_handle h);
 // Error message of the last failing call on this host thread.
 void set_error(const std::string& msg);
 etp_status cuda_status(cudaError_t e, const char* what);
+// Synchronises s, then reads the handle's status word: ETP_ERR_CUDA (word left set) if nonzero.
+etp_status read_status(const Ctx& c, cudaStream_t s, const char* who);
+// ETP_ERR_CUDA (message set) while the handle's status word holds a code, else ETP_OK.
+etp_status gate(etp_handle h, const char* who);
 
 // ---- conv kernels (etp_conv.cu)
 etp_status launch_forward(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr,
@@ -115,6 +125,15 @@ etp_status launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, co
                   const float* edge_vec, const float* x, const float* W, float* out, void* ws, cudaStream_t s);
 etp_status status(const Ctx& c, const void* ws, cudaStream_t s);
 }  // namespace cm
+
+// ---- channel-major forward with path subsets (etp_fwd_cx.cu): l_max <= 2, C <= 128
+namespace cx {
+bool supported(const Ctx& c);
+size_t workspace_bytes(const Ctx& c);
+etp_status launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
+                  const float* edge_vec, const float* x, const float* W, float* out, void* ws, cudaStream_t s);
+etp_status status(const Ctx& c, const void* ws, cudaStream_t s);
+}  // namespace cx
 
 // receiver of every canonical edge, recv[e] (etp_bwd_tc.cu)
 etp_status launch_recv_of_edge(const int* row_ptr, int n_nodes, int n_edges, int* recv, cudaStream_t s);

@@ -1,10 +1,10 @@
 // Forward entry point whose scratch lives in a fixed, statically sized device array of this
-// module instead of a caller-supplied workspace. It runs the same tensor-core forward as
-// etp_forward; only the origin of the scratch differs.
+// module instead of a caller-supplied workspace. For uniform handles it always runs the
+// edge-major tensor-core forward (whatever ETP_FORWARD says); general handles run the
+// table-driven forward, which needs no scratch.
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 #include <string>
 
 #include "etp_internal.h"
@@ -13,35 +13,21 @@ namespace etp {
 namespace {
 
 constexpr size_t kScratchBytes = 256 * 1024;
-constexpr int kMaxDevices = 64;
 
-// Pre-split weights and the pipeline status word of the tensor-core forward. One copy per
-// device (a __device__ variable is instantiated in every context that loads the module).
+// Pre-split weights of the tensor-core forward. One copy per device (a __device__ variable is
+// instantiated in every context that loads the module).
 __device__ __align__(256) unsigned char g_fixed_scratch[kScratchBytes];
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-std::mutex g_mutex;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of g_fixed_scratch on the current device, looked up once per device.
+// Device address of g_fixed_scratch in the current device's context. Looked up on every call (a
+// host-side query, cheap next to the launches), so a context that was torn down and re-created,
+// which may load the module at another address, never sees a stale pointer.
 etp_status fixed_scratch(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_status(e, "etp_forward_noalloc: cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) {
-    set_error("etp_forward_noalloc: device ordinal " + std::to_string(dev) + " beyond the supported " +
-              std::to_string(kMaxDevices));
-    return ETP_ERR_UNSUPPORTED;
-  }
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_fixed_scratch);
-    if (e != cudaSuccess) return cuda_status(e, "etp_forward_noalloc: cudaGetSymbolAddress");
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_fixed_scratch);
+  if (e != cudaSuccess) return cuda_status(e, "etp_forward_noalloc: cudaGetSymbolAddress");
+  *out = p;
   return ETP_OK;
 }
 
@@ -74,6 +60,7 @@ extern "C" etp_status etp_forward_noalloc(etp_handle h, int n_nodes, int n_edges
     set_error("etp_forward_noalloc: x, W and out must be 16-byte aligned");
     return ETP_ERR_INVALID_ARG;
   }
+  if (etp::gate(h, "etp_forward_noalloc") != ETP_OK) return ETP_ERR_CUDA;
   if (c->general) {   // the general kernels need no scratch at all
     if (static_cast<long long>(n_nodes) * c->gen.dim_out >= (1LL << 31)) {
       set_error("etp_forward_noalloc: n_nodes * dim must stay below 2^31");
@@ -93,9 +80,9 @@ extern "C" etp_status etp_forward_noalloc(etp_handle h, int n_nodes, int n_edges
   void* scratch = nullptr;
   etp_status st = etp::fixed_scratch(&scratch);
   if (st != ETP_OK) return st;
-  // The status word inside the scratch is cleared by the first kernel of the launch sequence and
-  // the pre-split weights are rewritten in full on every call, so nothing depends on its contents
-  // from an earlier call.
+  // The pre-split weights are rewritten in full on every call, so nothing depends on the array's
+  // contents from an earlier call. A bounded wait that gives up stores its code in the handle's
+  // status word (pinned host memory), which etp_get_status and every later call report.
   return etp::tc::launch_forward_tc(*c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, scratch,
                                     static_cast<cudaStream_t>(stream));
 }

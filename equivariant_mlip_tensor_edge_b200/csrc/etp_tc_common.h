@@ -46,8 +46,16 @@ __device__ __forceinline__ bool mbar_test(uint64_t* b, uint32_t parity) {
   return ok != 0;
 }
 
+// Records a pipeline error code in the handle's status word. The word lives in pinned host memory
+// mapped into the device address space, so it is written with a plain store (atomics on host
+// memory are not relied on) and made visible to the host with a system-scope fence.
+__device__ __forceinline__ void report_code(int* err, int code) {
+  *reinterpret_cast<volatile int*>(err) = code;
+  __threadfence_system();
+}
+
 // Bounded wait on the phase of the given parity. Returns false (and raises the CTA abort flag and
-// the global error code) when the limit is exceeded or another thread has aborted.
+// records the error code) when the limit is exceeded or another thread has aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* err,
                                           int code) {
   if (mbar_test(b, parity)) return true;
@@ -56,7 +64,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
     if (mbar_test(b, parity)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) {
-      atomicExch(err, code);
+      report_code(err, code);
       *abort_flag = 1;
       return false;
     }
@@ -69,6 +77,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* b, uint32_t parity, volatile
                                           int code) {
   const bool ok = mbar_wait(b, parity, abort_flag, err, code);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+// Drain wait: ignores the abort flag. Used before a CTA releases TMEM or shared memory that
+// asynchronous copies or MMAs it issued may still write. Returns false if the bound is exceeded.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* b, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_test(b, parity)) {
+    if (clock64() - t0 > kWaitCycles) return false;
+  }
+  return true;
 }
 
 __device__ __forceinline__ void fence_proxy_async() {

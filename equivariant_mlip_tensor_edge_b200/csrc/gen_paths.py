@@ -529,6 +529,130 @@ def emit_cm(out, lmax):
             out.append("}")
 
 
+# ---------------------------------------------------------------- channel-major forward, path subsets
+
+CX_LMAX = (1, 2)
+
+
+def cx_subsets(lmax):
+    """The two path subsets of the channel-major forward: subset 0 holds the paths with l1 < lmax,
+    subset 1 those with l1 = lmax. Splitting by l1 means the warps of the two subsets read disjoint
+    components of a sender row, so no component is loaded twice."""
+    paths = paths_for(lmax)
+    return [[p for p, t in enumerate(paths) if t[0] < lmax], [p for p, t in enumerate(paths) if t[0] == lmax]]
+
+
+def cx_coefficients(lmax, subset):
+    """Unique per-edge coefficients of a subset. Every nonzero M[m3][m1] = sum_m2 C Y[l2 m2] of a
+    path with l2 > 0 is a fixed combination of one rank's harmonics; entries whose combinations agree
+    up to sign share one stored value. Returns (keys, entry map): keys[i] = (l2, canonical vector),
+    entry map[(p, m3, m1)] = (coefficient index, sign)."""
+    paths = paths_for(lmax)
+    ent = path_m_entries(lmax)
+    keys, emap = [], {}
+    for p in subset:
+        l1, l2, l3 = paths[p]
+        if l2 == 0:
+            continue
+        for m3, m1, terms in ent[p]:
+            vec = [0.0] * (2 * l2 + 1)
+            for v, i in terms:
+                vec[i - idx(l2, -l2)] = v
+            first = next(v for v in vec if v != 0.0)
+            sgn = 1.0 if first > 0 else -1.0
+            key = (l2, tuple(round(sgn * v, 12) for v in vec))
+            if key not in keys:
+                keys.append(key)
+            emap[(p, m3, m1)] = (keys.index(key), sgn)
+    return keys, emap
+
+
+def emit_cx(out, lmax):
+    paths = paths_for(lmax)
+    ent = path_m_entries(lmax)
+    subsets = cx_subsets(lmax)
+    for s, sub in enumerate(subsets):
+        keys, emap = cx_coefficients(lmax, sub)
+        nc = max(4, -(-len(keys) // 4) * 4)
+        l1s = sorted({paths[p][0] for p in sub})
+        xcomps = [idx(l1, m) for l1 in l1s for m in range(-l1, l1 + 1)]
+        ocomps = sorted({idx(paths[p][2], m) for p in sub for m in range(-paths[p][2], paths[p][2] + 1)})
+        xi = {c: i for i, c in enumerate(xcomps)}
+        oi = {c: i for i, c in enumerate(ocomps)}
+        fma = 0
+        out.append(f"// ---- channel-major forward, l_max = {lmax}, subset {s}: paths {sub}")
+        out.append(f"template <> struct CxSub<{lmax}, {s}> {{")
+        out.append(f"  static constexpr int NP = {len(sub)};   // paths")
+        out.append(f"  static constexpr int NC = {nc};   // stored coefficients per edge (multiple of 4)")
+        out.append(f"  static constexpr int NX = {len(xcomps)};   // sender-row components read")
+        out.append(f"  static constexpr int NO = {len(ocomps)};   // output components written")
+        for name, lst in (("path", sub), ("xcomp", xcomps), ("ocomp", ocomps)):
+            out.append(f"  __host__ __device__ static constexpr int {name}(int i) {{")
+            out.append(f"    constexpr int t[{len(lst)}] = {{{', '.join(str(v) for v in lst)}}};")
+            out.append("    return t[i];")
+            out.append("  }")
+        # setup side: the coefficients from the harmonics
+        out.append(f"  __device__ __forceinline__ static void coef(const float* Y, float (&c)[{nc}]) {{")
+        for i, (l2, vec) in enumerate(keys):
+            terms = [f"{repr_f32(np.float32(v))}*Y[{idx(l2, m2 - l2)}]" for m2, v in enumerate(vec) if v != 0.0]
+            out.append(f"    c[{i}] = {' + '.join(terms)};")
+        for i in range(len(keys), nc):
+            out.append(f"    c[{i}] = 0.0f;")
+        out.append("  }")
+        # consumer side: one edge, NSL channels per lane
+        out.append("  template <int NSL>")
+        out.append(f"  __device__ __forceinline__ static void fwd(const float4* __restrict__ cf, const float (&x)[NSL][{len(xcomps)}],")
+        out.append(f"      const float (&w)[NSL][{len(sub)}], float (&acc)[NSL][{len(ocomps)}]) {{")
+        for q in range(nc // 4):
+            out.append(f"    const float4 c4_{q} = cf[{q}];")
+        out.append(f"    const float cv[{nc}] = {{" + ", ".join(f"c4_{q // 4}.{'xyzw'[q % 4]}" for q in range(nc)) + "};")
+        out.append("    #pragma unroll")
+        out.append("    for (int k = 0; k < NSL; ++k) {")
+        for pi, p in enumerate(sub):
+            l1, l2, l3 = paths[p]
+            e = ent[p]
+            out.append(f"      {{ // path {p}: ({l1},{l2},{l3})")
+            out.append(f"        const float wp = w[k][{pi}];")
+            if l2 == 0:
+                for m3, m1, terms in e:
+                    assert m3 == m1 and len(terms) == 1 and abs(terms[0][0] - 1.0) < 1e-12
+                    o, xx = oi[idx(l3, m3 - l3)], xi[idx(l1, m1 - l1)]
+                    out.append(f"        acc[k][{o}] = fmaf(wp, x[k][{xx}], acc[k][{o}]);")
+                    fma += 1
+            elif (2 * l1 + 1) < (2 * l3 + 1):
+                for m1 in range(2 * l1 + 1):
+                    out.append(f"        const float xs{m1} = wp * x[k][{xi[idx(l1, m1 - l1)]}];")
+                    fma += 1
+                for m3, m1, _ in e:
+                    ci, sg = emap[(p, m3, m1)]
+                    o = oi[idx(l3, m3 - l3)]
+                    cexpr = f"cv[{ci}]" if sg > 0 else f"-cv[{ci}]"
+                    out.append(f"        acc[k][{o}] = fmaf({cexpr}, xs{m1}, acc[k][{o}]);")
+                    fma += 1
+            else:
+                for m3 in range(2 * l3 + 1):
+                    row = [(a, m1) for (a, m1, _) in e if a == m3]
+                    if not row:
+                        continue
+                    o = oi[idx(l3, m3 - l3)]
+                    for j, (a, m1) in enumerate(row):
+                        ci, sg = emap[(p, a, m1)]
+                        cexpr = f"cv[{ci}]" if sg > 0 else f"-cv[{ci}]"
+                        xv = f"x[k][{xi[idx(l1, m1 - l1)]}]"
+                        if j == 0:
+                            out.append(f"        float s{m3} = {cexpr} * {xv};")
+                        else:
+                            out.append(f"        s{m3} = fmaf({cexpr}, {xv}, s{m3});")
+                        fma += 1
+                    out.append(f"        acc[k][{o}] = fmaf(wp, s{m3}, acc[k][{o}]);")
+                    fma += 1
+            out.append("      }")
+        out.append("    }")
+        out.append("  }")
+        out.append(f"  static constexpr int FMA = {fma};   // FP32 instructions per edge and channel")
+        out.append("};")
+
+
 # ---------------------------------------------------------------- general irreps
 
 GEN_LMAX = 4
@@ -714,12 +838,15 @@ def generate():
            "  }",
            "}",
            "template <int L> struct PathSet;",
-           "template <int L, int G> struct CmLayout;"]
+           "template <int L, int G> struct CmLayout;",
+           "template <int L, int S> struct CxSub;"]
     for lmax in LMAX_SUPPORTED:
         emit_sh(out, lmax)
         emit_paths(out, lmax)
     for lmax in CM_LMAX:
         emit_cm(out, lmax)
+    for lmax in CX_LMAX:
+        emit_cx(out, lmax)
     for lmax in LMAX_SUPPORTED:
         emit_node(out, lmax)
     emit_sh(out, GEN_LMAX)

@@ -42,6 +42,13 @@
  *   Errors: every call returns an etp_status; no call throws or traps. ETP_ERR_CUDA reports a
  *   launch error (no implicit synchronisation). etp_last_error() returns a thread-local message
  *   for the last failing call on the calling host thread.
+ *   Pipeline status: every wait inside the tensor-core kernels is bounded (about 2 s). A kernel
+ *   whose wait gives up stores a nonzero code in its handle's status word, pinned host memory
+ *   mapped into the device address space, and exits early, so that call's outputs are
+ *   incomplete. Kernels run after the call has returned, so the call itself still returned
+ *   ETP_OK; from then on every compute call on the handle returns ETP_ERR_CUDA until
+ *   etp_get_status reads and clears the code (etp_get_status synchronises; with ETP_VALIDATE=1
+ *   the forward and backward also synchronise and report the code of their own launch).
  *   Thread safety: a handle is immutable after etp_create; concurrent calls on different
  *   streams with distinct output and workspace buffers are safe.
  *   Graph validation: with the environment variable ETP_VALIDATE=1, etp_forward and etp_backward
@@ -86,7 +93,10 @@ typedef struct {
   int flop_bwd;      /* the same for the backward: sum_p 2 (3 nnz_p + 2 (2 l3 + 1)) mul_p */
 } etp_info_t;
 
-/* Create a convolution handle. Host-only, synchronous, allocates host memory only.
+/* Create a convolution handle. Host-only, synchronous; allocates host memory only: the handle,
+ * and its 64-byte status word in pinned host memory mapped for the device (plain host memory when
+ * no CUDA device is present). Fails with ETP_ERR_CUDA if a device is present but the pinned word
+ * cannot be allocated.
  * irreps_in / irreps_out: "mulxLp+mulxLp+..." strings, e.g. "64x0e+64x1o+64x2e".
  * Two kinds of handle, chosen here:
  *  - uniform (the tensor-core kernels): every block has the same multiplicity C (C % 4 == 0,
@@ -94,22 +104,35 @@ typedef struct {
  *    sh_lmax == L, L in {1,2,3};
  *  - general (table-driven FP32 kernels, info.general = 1): any blocks with 0 <= l <= 4 and
  *    1 <= mul <= 1024 in any order and either parity, sh_lmax <= 4, node rows of at most 4096
- *    floats, 1 to 160 paths. Paths join blocks of EQUAL multiplicity only (uvu: channel u to
+ *    floats, 1 to 128 paths, at most 16 blocks a side. Paths join blocks of EQUAL multiplicity only (uvu: channel u to
  *    channel u), so irreps like NequIP's 128x0e+64x1o+32x2e+32x3o couple 2e with 3o but not 1o
  *    with 2e. Paths with l1 + l2 + l3 odd use the real antisymmetric coupling (the imaginary
  *    part of the complex-to-real transformed Clebsch-Gordan tensor; the cross product for
  *    1 x 1 -> 1). W is [n_basis][cols] with path p's mul_p columns after the earlier paths'
  *    (the same as [n_basis][n_paths][C] when all blocks have C channels); node rows hold the
  *    blocks in string order, block b as [m][u] with mul_b channels. General handles support
- *    etp_forward, etp_forward_noalloc (no scratch needed), etp_backward and etp_backward_weights;
- *    the masked and radial-weight calls return ETP_ERR_UNSUPPORTED for them.
+ *    etp_forward, etp_forward_noalloc (no scratch needed), etp_backward, etp_backward_weights and,
+ *    for handles with at most 32 paths (the mask has 32 bits), etp_forward_masked and
+ *    etp_backward_masked (more paths: ETP_ERR_UNSUPPORTED); etp_radial_weights returns
+ *    ETP_ERR_UNSUPPORTED for them.
  * Both need n_basis == 8 and r_cut > 0. Malformed strings -> ETP_ERR_IRREPS; anything else
  * outside these sets -> ETP_ERR_UNSUPPORTED. The path list is the enumeration described above. */
 etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_basis,
                       float r_cut, etp_handle* out);
 
-/* Release a handle (host memory only). NULL is accepted. */
+/* Release a handle and its status word. NULL is accepted. */
 etp_status etp_destroy(etp_handle h);
+
+/* Pipeline status of a handle: synchronises `stream`, stores the handle's status word in *code
+ * (host pointer, may be NULL) and clears it. ETP_OK when the word was 0; ETP_ERR_CUDA (with a
+ * message naming the code) when a kernel of an earlier call on the handle gave up a bounded
+ * wait, in which case the outputs of the calls since the previous check may be incomplete.
+ * Without a CUDA device nothing is synchronised. */
+etp_status etp_get_status(etp_handle h, void* stream, int* code);
+
+/* Host address of the handle's status word (NULL for a NULL handle), for callers that poll it
+ * without synchronising: nonzero means a kernel gave up a bounded wait. Writing 0 clears it. */
+int* etp_status_word(etp_handle h);
 
 /* Dimensions and path statistics of a handle (info: host pointer). */
 etp_status etp_get_info(etp_handle h, etp_info_t* info);
@@ -131,25 +154,34 @@ size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges);
  * Spherical harmonics, radial basis, radial projection, Clebsch-Gordan contraction and the
  * per-receiver segmented sum run in one kernel pass; receivers without edges get zero rows.
  * Edges with d >= r_cut contribute zero (u = 0). workspace may be NULL when
- * etp_workspace_bytes returns 0. */
+ * etp_workspace_bytes returns 0. Kernel: for uniform handles with L <= 2 and C <= 128 the
+ * channel-major path-subset kernel (the CTAs take equal contiguous ranges of canonical edges;
+ * a receiver whose edges cross a range boundary is summed by the CTA that adds its last part,
+ * in CTA order, so the result is still bitwise reproducible), else the edge-major tensor-core
+ * kernel; the environment variable ETP_FORWARD=edge, channel or generic selects another
+ * kernel (all agree with the float64 reference within the same tolerance). */
 etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
                        const int* sender, const float* edge_vec, const float* x, const float* W,
                        float* out, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Forward without a workspace argument: the same computation, kernels and results as
- * etp_forward, but its scratch (the tf32-split radial weight matrix and a status word) sits in
- * a fixed 256 KiB array inside libetp's device module, one per device, so the call allocates no
- * memory and takes nothing from the caller but the tensors.
+/* Forward without a workspace argument: the same computation as etp_forward, but its scratch
+ * (the tf32-split radial weight matrix) sits in a fixed 256 KiB array inside libetp's device
+ * module, one per device, so the call allocates no memory and takes nothing from the caller but
+ * the tensors. For uniform handles it always runs the edge-major tensor-core forward and ignores
+ * ETP_FORWARD, so its bits can differ from etp_forward's default kernel (both agree with the
+ * float64 reference within the same tolerance); general handles run the table-driven forward,
+ * which needs no scratch.
  * The method has no such call; it is an interface convenience. It is for callers that cannot
  * provide device scratch: for instance a host program that reaches the model through a fixed
  * plugin interface that hands over only the input and output tensors, with no allocator of its
  * own and nowhere to keep a workspace alive between calls.
  * Limit: a handle whose scratch would exceed the 256 KiB (lmax 3 with more than 160 channels)
  * is refused with ETP_ERR_CAPACITY and a message naming both sizes; use etp_forward for it.
- * The first call on each device looks up the array's device address once, with that device
- * current (cudaGetSymbolAddress); make that first call before beginning any stream capture.
- * Nothing in the array needs to start at zero: each call rewrites the weights in full and its
- * first kernel clears the status word.
+ * Every call looks up the array's device address in the current device's context
+ * (cudaGetSymbolAddress, a host-side query that does not synchronise); the first call in a
+ * context also loads the module there, so make a first call before beginning any stream
+ * capture. Nothing in the array needs to start at zero: each call rewrites the weights in full.
+ * A bounded wait that gives up is reported through the handle's status word (etp_get_status).
  * Overlapping calls on one device (different streams or host threads) share the array and race
  * with each other; order them (one stream, or events). The ETP_VALIDATE graph checks are not run. */
 etp_status etp_forward_noalloc(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
@@ -167,15 +199,6 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
                         float* grad_x, float* grad_edge_vec, void* workspace,
                         size_t workspace_bytes, void* stream);
 
-/* Weight gradient of the convolution for the cotangent grad_out (the training path):
- *   grad_W[n_basis][n_paths][C] = dL/dW,  L = <grad_out, out>,
- *   dL/dW[b][p][u] = sum_e R_b(d_e) sum_{m1,m3} x[send, l1, m1, u] (sum_m2 C Y_{l2 m2}) g[recv, l3, m3, u].
- * Runs over the canonical (receiver-sorted) order, with the channels on the lanes; partial sums
- * per range of edges are added in range order, so repeated calls give identical bits.
- * grad_W is overwritten (zero for a graph without edges). Uses the etp_workspace_bytes workspace.
- * For a general irreps handle grad_W has the W layout [n_basis][cols]; the kernel stages the
- * geometry of 128 canonical edges at a time, runs each path's channels over them and writes one
- * partial column per range; the ranges are added in order (also bit-reproducible). */
 /* Node-local product ladder of correlation order nu (FlashCart Fig. 3b and Fig. E1, path-reduced):
  *   B_1 = A,  B_{q+1}[l3, m3, u] = sum_{p=(l1,l2,l3)} W[q-1][p][u] sum_{m1,m2} C B_q[l1, m1, u] A[l2, m2, u],
  *   out = B_1 + ... + B_nu,
@@ -204,6 +227,15 @@ etp_status etp_backward_masked(etp_handle h, int n_nodes, int n_edges, const int
                                float* grad_edge_vec, void* workspace, size_t workspace_bytes,
                                void* stream);
 
+/* Weight gradient of the convolution for the cotangent grad_out (the training path):
+ *   grad_W[n_basis][n_paths][C] = dL/dW,  L = <grad_out, out>,
+ *   dL/dW[b][p][u] = sum_e R_b(d_e) sum_{m1,m3} x[send, l1, m1, u] (sum_m2 C Y_{l2 m2}) g[recv, l3, m3, u].
+ * Runs over the canonical (receiver-sorted) order, with the channels on the lanes; partial sums
+ * per range of edges are added in range order, so repeated calls give identical bits.
+ * grad_W is overwritten (zero for a graph without edges). Uses the etp_workspace_bytes workspace.
+ * For a general irreps handle grad_W has the W layout [n_basis][cols]; the kernel stages the
+ * geometry of 128 canonical edges at a time, runs each path's channels over them and writes one
+ * partial column per range; the ranges are added in order (also bit-reproducible). */
 etp_status etp_backward_weights(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
                                 const int* sender, const float* edge_vec, const float* x,
                                 const float* grad_out, float* grad_W, void* workspace,

@@ -22,6 +22,14 @@ int main(void) {
   if (etp_get_paths(h, paths, 64) != ETP_OK) return fail("paths uniform");
   if (paths[0] != 0 || paths[1] != 0 || paths[2] != 0) return fail("first path (0,0,0)");
   if (etp_workspace_bytes(h, 1000, 89156) < 2 * 4 * 89156) return fail("workspace size");
+  {
+    int code = -1;
+    int* word = etp_status_word(h);
+    if (!word || *word != 0) return fail("status word starts clear");
+    *word = 9;
+    if (etp_get_status(h, NULL, &code) != ETP_ERR_CUDA || code != 9 || *word != 0) return fail("status read");
+    if (etp_get_status(h, NULL, &code) != ETP_OK || code != 0) return fail("status cleared");
+  }
   etp_destroy(h);
   printf("ok uniform: %d paths, dim %d, weights %d\n", info.n_paths, info.dim_in, info.weight_numel);
 

@@ -184,3 +184,35 @@ def test_create_matches_the_oracle_path_set_on_random_irreps():
         seen_uniform += 1 - info.general
         lib.etp_destroy(h)
     assert seen_general > 50 and seen_refused > 5
+
+
+def test_status_word_gates_calls_until_get_status_clears_it(lib):
+    """A kernel that gives up a bounded wait stores its code in the handle's status word; every
+    later compute call on the handle then fails with ETP_ERR_CUDA (before any CUDA work) until
+    etp_get_status has read and cleared the word. Here the test writes the word itself."""
+    conv = etp.EdgeConv("8x0e+8x1o", 1, "8x0e+8x1o", 8, 4.0)
+    word = lib.etp_status_word(conv._h)
+    assert word and word[0] == 0
+    assert not lib.etp_status_word(None)
+    # a clean handle: radial weights of an empty edge list is a no-op that succeeds
+    assert lib.etp_radial_weights(conv._h, 0, None, None, None, None) == 0
+    word[0] = 37
+    fake = ctypes.c_void_p(0x1000)   # 16-byte aligned, never dereferenced: the gate comes first
+    assert lib.etp_forward(conv._h, 4, 4, fake, fake, fake, fake, fake, fake, fake, 1 << 20, None) == 5
+    assert "code 37" in lib.etp_last_error().decode()
+    assert lib.etp_forward_noalloc(conv._h, 4, 4, fake, fake, fake, fake, fake, fake, None) == 5
+    assert lib.etp_backward_weights(conv._h, 4, 4, fake, fake, fake, fake, fake, fake, fake, 1 << 20, None) == 5
+    assert lib.etp_radial_weights(conv._h, 0, None, None, None, None) == 5
+    code = ctypes.c_int(-1)
+    assert lib.etp_get_status(conv._h, None, ctypes.byref(code)) == 5
+    assert code.value == 37
+    assert word[0] == 0
+    assert lib.etp_get_status(conv._h, None, ctypes.byref(code)) == 0 and code.value == 0
+    assert lib.etp_radial_weights(conv._h, 0, None, None, None, None) == 0
+    assert lib.etp_get_status(None, None, None) == 1
+    # the binding raises on a set word
+    word[0] = 12
+    with pytest.raises(etp.EtpError) as ei:
+        conv.check_status()
+    assert ei.value.status == 5 and "code 12" in str(ei.value)
+    conv.check_status()

@@ -368,7 +368,7 @@ def test_no_cpu_fallback():
 
 # ------------------------------------------------------------------ forward kernels: both implementations
 
-@pytest.mark.parametrize("impl", ["default", "channel", "generic"])
+@pytest.mark.parametrize("impl", ["default", "edge", "channel", "generic"])
 @pytest.mark.parametrize("name", ["tiny", "diamond1k"])
 def test_forward_both_kernels(wls, name, impl, monkeypatch):
     if impl != "default":
@@ -600,6 +600,38 @@ def test_forward_channel_major_ragged(lmax, c, monkeypatch):
     monkeypatch.delenv("ETP_FORWARD")
     edge = _np(conv.forward(g, xd, Wd))
     assert_blocks_close(o, edge.astype(np.float64), c, lmax, f"channel-major vs edge-major lmax={lmax} C={c}")
+
+
+@pytest.mark.parametrize("lmax,c", [(1, 8), (1, 32), (1, 64), (2, 8), (2, 20), (2, 36), (2, 64)])
+def test_forward_path_subset_kernel_ragged(lmax, c, monkeypatch):
+    """The default forward for l_max <= 2 and C <= 64 (channel-major, two path subsets): empty rows
+    at both ends and in between, receivers whose edges span several CTAs (the kernel cuts the edge
+    list into equal ranges of at least 64 edges, so the 127..300-edge rows cross range
+    boundaries), channel counts that leave lanes idle (8, 20, 36); compared with the oracle and
+    bitwise reproducible."""
+    from oracle.conv import ConvSpec
+    monkeypatch.setenv("ETP_VALIDATE", "1")
+    irr = "+".join(f"{c}x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
+    degrees = np.array([0, 0, 1, 31, 32, 33, 0, 127, 128, 129, 300, 5, 0, 64, 97, 15, 17, 0])
+    n = len(degrees)
+    recv, send, vec = _random_graph(n, degrees, seed=70 + lmax + c)
+    conv = etp.EdgeConv(irr, lmax, irr, 8, 5.0)
+    spec = ConvSpec(irr, lmax, irr, 8, 5.0)
+    rng = np.random.default_rng(700 + lmax + c)
+    x = rng.standard_normal((n, spec.dim_in)).astype(np.float32)
+    W = (rng.standard_normal((8, len(spec.paths), c)) / np.sqrt(8)).astype(np.float32)
+    g = etp.build_csr(n, torch.from_numpy(recv).to(DEV), torch.from_numpy(send).to(DEV),
+                      torch.from_numpy(vec).to(DEV))
+    xd, Wd = torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)
+    out = conv.forward(g, xd, Wd)
+    again = conv.forward(g, xd, Wd)
+    assert torch.equal(out, again), "path-subset forward is not bitwise deterministic"
+    order = np.lexsort((send, recv))
+    rp = np.concatenate([[0], np.cumsum(degrees)])
+    ref = conv_forward(spec, rp, send[order], vec[order], x, W)
+    o = _np(out)
+    assert np.all(o[degrees == 0] == 0.0)
+    assert_blocks_close(o, ref, c, lmax, f"path-subset forward lmax={lmax} C={c}")
 
 
 # ------------------------------------------------------------------ per-edge path masks
