@@ -6,21 +6,23 @@
 // message accumulates in registers of the lanes that own its channels, so no cross-lane sums are
 // needed, and the sender rows of a batch are staged in shared memory by whole-row bulk copies.
 //
-// Roles (one persistent CTA per SM, 12 warps):
-//   setup warps 8, 9 (even and odd batches): one edge per lane: the bulk copy of the sender row
-//     (dim floats, contiguous), the direction, real spherical harmonics, the radial basis R_b(d)
-//     as the tf32 hi/lo rows of the MMA B operand, and the per-edge coefficients
-//     M[m3][m1] = sum_m2 C Y[l2 m2] of both path subsets, deduplicated up to sign.
+// Roles (one persistent CTA per SM, 13 warps):
+//   setup warps 8, 9 (even and odd MMA batches): one edge per lane, 32 edges (two batches) per
+//     pass: the direction, real spherical harmonics, the radial basis R_b(d) as the tf32 hi/lo
+//     rows of the MMA B operand, and the per-edge coefficients M[m3][m1] = sum_m2 C Y[l2 m2] of both
+//     path subsets, deduplicated up to sign, stored with the two edges of a pair interleaved.
 //   MMA warp 10 (one thread): w^T = W^T R^T on the tensor cores, D[(path, channel)][edge]: one
 //     block of 128 rows per path item, three kind::tf32 MMAs (hi*hi + hi*lo + lo*hi) per block,
 //     into a two-slot TMEM ring.
+//   loader warp 12: one bulk copy per edge of the sender's whole row (dim floats, contiguous) into
+//     a ring of batch slots.
 //   consumer warps 0..7: warp w reads TMEM lane quadrant q = w % 4. Quadrants 0, 1 run path
 //     subset 0 (l1 < l_max) on channels 0..31 and 32..63, quadrants 2, 3 subset 1 (l1 = l_max),
 //     so the two subsets read disjoint components of a sender row. The two warps of a quadrant
-//     take the two halves of each batch. Per edge: the lane's sender-row components and the
-//     edge's coefficients from shared memory, w from registers loaded by tcgen05.ld, and the
-//     generated contraction. When the receiver changes, the warp hands its partial message to
-//     the combine warp through a ring of shared-memory slots.
+//     take the two halves of each batch. Edges go in pairs through the packed (f32x2) form of the
+//     generated contraction: the lane's sender-row components and the pair's coefficients from
+//     shared memory, w from registers loaded by tcgen05.ld. When the receiver changes, the warp
+//     hands its partial message to the combine warp through a ring of shared-memory slots.
 //   combine warp 11: per receiver, adds the eight partials in a fixed order and stores the row.
 //     A receiver whose edges span several CTAs is summed by the CTA that adds its last part (a
 //     per-receiver arrival counter, zeroed by the prep kernel), again in a fixed order.
@@ -61,13 +63,17 @@ using tc::warp_wait;
 constexpr int kQ = 4;                    // TMEM lane quadrants
 constexpr int kH = 2;                    // consumer warps per quadrant
 constexpr int kCons = kQ * kH;           // consumer warps
-constexpr int kSetup0 = kCons;           // setup warps kSetup0, kSetup0 + 1
+constexpr int kSetup0 = kCons;           // geometry warps kSetup0, kSetup0 + 1 (even, odd batches)
 constexpr int kMmaWarp = kCons + 2;
 constexpr int kCombWarp = kCons + 3;
-constexpr int kThreads = 32 * (kCons + 4);
-constexpr int kSB = 3;                   // setup ring (batches): coefficients, B operand, sender rows
-constexpr int kNR = 4;                   // receiver ring (partial messages)
-constexpr int kN = 16;                   // edges per batch (MMA N)
+constexpr int kLoadWarp = kCons + 4;     // sender-row loader
+constexpr int kThreads = 32 * (kCons + 5);
+constexpr int kGS = 8;                   // geometry ring (batches): per-edge coefficients
+constexpr int kRS = kGS / 2;             // B operand ring (MMA batches)
+constexpr int kXS = 3;                   // sender-row ring (batches)
+constexpr int kNR = 2;                   // receiver ring (partial messages)
+constexpr int kN = 16;                   // edges per setup / consumer batch
+constexpr int kNM = 2 * kN;              // edges per MMA batch (MMA N): two consecutive batches
 constexpr int kEPW = kN / kH;            // edges per consumer warp and batch
 constexpr int kRW = 4;                   // edges per TMEM load round (the slow path selects among 4)
 constexpr int kMaxC = 64;                // channels: two 32-lane slices
@@ -80,20 +86,23 @@ struct Cfg {
   static constexpr int D = (L + 1) * (L + 1);
   static constexpr int P = etp_gen::PathSet<L>::P;
   static constexpr int NB = S0::NP > S1::NP ? S0::NP : S1::NP;   // MMA blocks: one path item each
-  static constexpr int SLOTC = NB * kN;                          // TMEM columns per ring slot
+  static constexpr int SLOTC = NB * kNM;                         // TMEM columns per ring slot
   static constexpr int CW0 = S0::NC, CW1 = S1::NC;
-  static constexpr int CW = ((CW0 + CW1) / 4) % 2 == 1 ? CW0 + CW1 : CW0 + CW1 + 4;   // odd float4 count
+  // coefficient row of an edge pair: both subsets, the two edges interleaved (coefficient k of edge t
+  // at 2 k + t), padded to 4 mod 32 floats so that the setup warp's 8-byte stores hit distinct banks
+  static constexpr int PW = 2 * (CW0 + CW1) + (4 - (2 * (CW0 + CW1)) % 32 + 32) % 32;
   static constexpr int NOMAX = S0::NO > S1::NO ? S0::NO : S1::NO;
   static constexpr int XROW = kMaxC * D;                         // floats of the largest sender row
   // shared memory map (bytes)
   static constexpr int OFF_WA = 1024;                            // [NB][hi|lo][128 x 8]
-  static constexpr int OFF_CF = OFF_WA + NB * 8192;              // [kSB][kN][CW]
-  static constexpr int OFF_RB = OFF_CF + kSB * kN * CW * 4;      // [kSB][hi|lo][kN x 8]
-  static constexpr int OFF_X = OFF_RB + kSB * 2 * kN * 32;       // [kSB][kN][dim]
-  static constexpr int OFF_PT = OFF_X + kSB * kN * XROW * 4;     // [kNR][kCons][NOMAX][32]
+  static constexpr int OFF_CF = OFF_WA + NB * 8192;              // [kGS][kN / 2][PW]
+  static constexpr int OFF_RB = OFF_CF + kGS * (kN / 2) * PW * 4; // [kRS][hi|lo][kNM x 8]: B operand per MMA batch
+  static constexpr int OFF_X = OFF_RB + kRS * 2 * kNM * 32;      // [kXS][kN][dim]
+  static constexpr int OFF_PT = OFF_X + kXS * kN * XROW * 4;     // [kNR][kCons][NOMAX][32]
   static constexpr int END = OFF_PT + kNR * kCons * NOMAX * 32 * 4;
   static constexpr int SMEM = END < 118 * 1024 ? 118 * 1024 : END;   // > half an SM: one CTA per SM
   static_assert(2 * SLOTC <= kTmemCols, "two TMEM slots");
+  static_assert(PW % 32 == 4 && CW0 % 4 == 0 && CW1 % 4 == 0, "coefficient row layout");
   static_assert(END <= 227 * 1024, "shared memory budget");
   static_assert(OFF_RB % 128 == 0 && OFF_X % 128 == 0 && OFF_WA % 1024 == 0, "operand alignment");
 };
@@ -151,6 +160,24 @@ __device__ __forceinline__ int recv_of_warp(const int* __restrict__ row_ptr, int
   return first - 1;
 }
 
+// D (TMEM) = A (TMEM, M = 128 lanes x K = 8 columns of tf32) x B (shared memory descriptor)
+__device__ __forceinline__ void mma_tf32_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
+               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
   uint32_t r[4];
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
@@ -161,16 +188,16 @@ __device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
   for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-// Bounded wait with a short sleep between polls, for the roles whose latency is hidden (setup,
-// combine): they then take fewer issue slots from the consumer warps on their scheduler.
+// Bounded wait for the roles whose latency is hidden (setup, loader, combine): only lane 0 polls,
+// and it is suspended in hardware between polls (until the phase completes or the hint runs out),
+// so the waiting warp takes no issue slots from the consumer warps on its scheduler.
 __device__ __forceinline__ bool warp_wait_lazy(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* err,
                                                int code) {
   bool ok = true;
   if ((threadIdx.x & 31) == 0 && !mbar_test(b, parity)) {
     const long long t0 = clock64();
     while (true) {
-      __nanosleep(64);
-      if (mbar_test(b, parity)) break;
+      if (tc::mbar_test_sleep(b, parity, 50000u)) break;
       if (*abort_flag) {
         ok = false;
         break;
@@ -189,14 +216,15 @@ __device__ __forceinline__ bool warp_wait_lazy(uint64_t* b, uint32_t parity, vol
 
 struct Bars {
   uint64_t tfull[2], tempty[2];
-  uint64_t sfull[kSB], sfree[kSB], xfull[kSB];
+  uint64_t sfull[kGS], sfree[kGS];   // geometry ring: coefficients and B operand written / read
+  uint64_t xfull[kXS], xfree[kXS];   // sender-row ring: rows landed / read
   uint64_t rfull[kNR], rempty[kNR];
   uint64_t drain;
   uint32_t tmem_holder;
   int abort_flag;
   int r_begin, r_end;
   int e_beg, e_end;
-  int x_last[kSB];   // per slot: the last batch whose sender-row copies were issued into it
+  int x_last[kXS];   // per slot: the last batch whose sender-row copies were issued into it
 };
 static_assert(sizeof(Bars) <= 1024, "barrier block");
 
@@ -210,6 +238,9 @@ __host__ __device__ constexpr int oidx(int c) {
 // ---------------------------------------------------------------- consumer warps
 
 // Consumer warp of quadrant q (path subset SI = q / 2, channel (q % 2) * 32 + lane), batch half h.
+// Edges are taken in pairs: the two edges of a pair run through one packed (f32x2) contraction,
+// component .x the first edge, .y the second, each into its own half of the accumulator; the halves
+// are added (x + y) when the receiver's message is handed on, so the order of every sum is fixed.
 // CT: the channel count when it is a compile-time constant (64), else 0 (a.C at run time).
 template <int L, int SI, int CT>
 __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars* bars, int q, int h, uint32_t tmem,
@@ -217,8 +248,8 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
   using G = Cfg<L>;
   using SUB = etp_gen::CxSub<L, SI>;
   constexpr int NX = SUB::NX, NO = SUB::NO, NP = SUB::NP;
-  constexpr int CW = G::CW;
-  constexpr int CFO = SI == 0 ? 0 : G::CW0;     // the subset's coefficients within an edge's row
+  constexpr int PW = G::PW;
+  constexpr int CFO = SI == 0 ? 0 : 2 * G::CW0;   // the subset's coefficients within a pair's row
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int C = CT > 0 ? CT : a.C;
@@ -235,9 +266,9 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
   int xoff[NX];
 #pragma unroll
   for (int i = 0; i < NX; ++i) xoff[i] = SUB::xcomp(i) * C + ch0;
-  float acc[1][NO];
+  float2 acc[NO];
 #pragma unroll
-  for (int o = 0; o < NO; ++o) acc[0][o] = 0.0f;
+  for (int o = 0; o < NO; ++o) acc[o] = make_float2(0.0f, 0.0f);
 
   int cur = bars->r_begin;
   int nxt = __ldg(a.row_ptr + cur + 1);
@@ -249,8 +280,8 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
     float* pp = part + static_cast<size_t>(slot * kCons + warp) * (G::NOMAX * 32);
 #pragma unroll
     for (int o = 0; o < NO; ++o) {
-      pp[o * 32 + lane] = acc[0][o];
-      acc[0][o] = 0.0f;
+      pp[o * 32 + lane] = acc[o].x + acc[o].y;
+      acc[o] = make_float2(0.0f, 0.0f);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&bars->rfull[slot]);
@@ -262,24 +293,26 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
 
   bool ok = true;
   for (int k = 0; k < nb && ok; ++k) {
-    const int ts = k & 1, sl = k % kSB;
+    const int m = k >> 1, ts = m & 1, sl = k % kGS, xl = k % kXS;   // MMA batch m covers batches 2 m, 2 m + 1
     const int base = e_beg + k * kN + h * kEPW;
     const int nval = e_end - base;   // edges of this batch half (may exceed kEPW or be <= 0)
-    ok = warp_wait(&bars->tfull[ts], (k >> 1) & 1, abort_flag, a.err, 31);
-    if (ok) ok = warp_wait(&bars->sfull[sl], (k / kSB) & 1, abort_flag, a.err, 32);
-    if (ok) ok = warp_wait(&bars->xfull[sl], (k / kSB) & 1, abort_flag, a.err, 38);
+    ok = warp_wait(&bars->tfull[ts], (m >> 1) & 1, abort_flag, a.err, 31);
+    if (ok) ok = warp_wait(&bars->sfull[sl], (k / kGS) & 1, abort_flag, a.err, 32);
+    if (ok) ok = warp_wait(&bars->xfull[xl], (k / kXS) & 1, abort_flag, a.err, 38);
     if (!ok) break;
     tc_fence_after();
-    const float* cfs = cfbase + static_cast<size_t>(sl * kN + h * kEPW) * CW + CFO;
-    const float* xs = xbase + static_cast<size_t>(sl * kN + h * kEPW) * dim;
-    const uint32_t tb = tmem + (static_cast<uint32_t>(32 * q) << 16) + ts * G::SLOTC + h * kEPW;
+    // pair j of this half: coefficient row cfs + j * PW, sender rows xs + (2 j + t) * dim
+    const float* cfs = cfbase + static_cast<size_t>(sl * (kN / 2) + h * (kEPW / 2)) * PW + CFO;
+    const float* xs = xbase + static_cast<size_t>(xl * kN + h * kEPW) * dim;
+    const uint32_t tb = tmem + (static_cast<uint32_t>(32 * q) << 16) + ts * G::SLOTC + (k & 1) * kN + h * kEPW;
+    const bool last_of_mma = (k & 1) || k == nb - 1;   // the MMA batch's columns are all read after this
 #pragma unroll 1
     for (int rr = 0; rr < kEPW / kRW && ok; ++rr) {
       float wv[NP][kRW];
 #pragma unroll
-      for (int b = 0; b < NP; ++b) tmem_ld4(tb + b * kN + rr * kRW, wv[b]);
+      for (int b = 0; b < NP; ++b) tmem_ld4(tb + b * kNM + rr * kRW, wv[b]);
       tc::tmem_wait_ld();
-      if (rr == kEPW / kRW - 1) {   // every column of the slot this warp needs is in registers
+      if (rr == kEPW / kRW - 1 && last_of_mma) {   // every column of the slot this warp needs is read
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->tempty[ts]);
@@ -287,44 +320,65 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
       const int r0 = rr * kRW;
       const int nv = nval - r0 < kRW ? nval - r0 : kRW;   // valid edges of the round (may be <= 0)
       if (nv == kRW && base + r0 + kRW - 1 < nxt) {
-        // common case: four valid edges of the current receiver, one straight-line block
+        // common case: four valid edges of the current receiver, two pairs in straight-line code
 #pragma unroll
-        for (int i0 = 0; i0 < kRW; ++i0) {
-          const int i = r0 + i0;
-          float xv[1][NX];
-          const float* xr = xs + static_cast<size_t>(i) * dim;
+        for (int pr = 0; pr < kRW / 2; ++pr) {
+          const int i = r0 + 2 * pr;
+          const float* xa = xs + static_cast<size_t>(i) * dim;
+          const float* xb = xa + dim;
+          float2 xv[NX];
 #pragma unroll
-          for (int c = 0; c < NX; ++c) xv[0][c] = chv ? xr[xoff[c]] : 0.0f;
-          float w[1][NP];
+          for (int c = 0; c < NX; ++c) xv[c] = chv ? make_float2(xa[xoff[c]], xb[xoff[c]]) : make_float2(0.0f, 0.0f);
+          float2 w[NP];
 #pragma unroll
-          for (int pi = 0; pi < NP; ++pi) w[0][pi] = wv[pi][i0];
-          SUB::template fwd<1>(reinterpret_cast<const float4*>(cfs + i * CW), xv, w, acc);
+          for (int pi = 0; pi < NP; ++pi) w[pi] = make_float2(wv[pi][2 * pr], wv[pi][2 * pr + 1]);
+          SUB::fwd2(reinterpret_cast<const float4*>(cfs + (i >> 1) * PW), xv, w, acc);
         }
       } else {
-        // a receiver boundary or the end of the range inside the round: edge by edge
+        // a receiver boundary or the end of the range inside the round: pair by pair; an edge of
+        // the pair that is invalid or belongs to a later receiver is masked (w = x = 0) and taken
+        // in a second step after the flush
 #pragma unroll 1
-        for (int i0 = 0; i0 < nv && ok; ++i0) {
-          const int i = r0 + i0;
-          while (base + i >= nxt) {
-            ok = flush();
+        for (int pr = 0; pr < kRW / 2 && ok; ++pr) {
+          const int i = r0 + 2 * pr;
+          if (2 * pr >= nv) break;
+          const bool vb = 2 * pr + 1 < nv;
+          const int want = vb ? 3 : 1;
+          int done = 0;   // bit t: edge t of the pair accumulated
+          while (done != want) {
+            const int first = done & 1;   // the next edge still to take
+            while (base + i + first >= nxt) {
+              ok = flush();
+              if (!ok) break;
+            }
             if (!ok) break;
+            const bool m0 = first == 0;
+            const bool m1 = vb && base + i + 1 < nxt;
+            const float* xa = xs + static_cast<size_t>(i) * dim;
+            const float* xb = xa + dim;
+            float2 xv[NX];
+#pragma unroll
+            for (int c = 0; c < NX; ++c)
+              xv[c] = make_float2(chv && m0 ? xa[xoff[c]] : 0.0f, chv && m1 ? xb[xoff[c]] : 0.0f);
+            float2 w[NP];
+#pragma unroll
+            for (int pi = 0; pi < NP; ++pi) {
+              const float wa = pr == 0 ? wv[pi][0] : wv[pi][2];
+              const float wb = pr == 0 ? wv[pi][1] : wv[pi][3];
+              w[pi] = make_float2(m0 ? wa : 0.0f, m1 ? wb : 0.0f);
+            }
+            SUB::fwd2(reinterpret_cast<const float4*>(cfs + (i >> 1) * PW), xv, w, acc);
+            done |= (m0 ? 1 : 0) | (m1 ? 2 : 0);
           }
-          if (!ok) break;
-          float xv[1][NX];
-          const float* xr = xs + static_cast<size_t>(i) * dim;
-#pragma unroll
-          for (int c = 0; c < NX; ++c) xv[0][c] = chv ? xr[xoff[c]] : 0.0f;
-          float w[1][NP];
-#pragma unroll
-          for (int pi = 0; pi < NP; ++pi)
-            w[0][pi] = i0 == 0 ? wv[pi][0] : (i0 == 1 ? wv[pi][1] : (i0 == 2 ? wv[pi][2] : wv[pi][3]));
-          SUB::template fwd<1>(reinterpret_cast<const float4*>(cfs + i * CW), xv, w, acc);
         }
       }
     }
     if (!ok) break;
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars->sfree[sl]);   // coefficients and sender rows of the slot read
+    if (lane == 0) {   // coefficients and sender rows of the batch read
+      mbar_arrive(&bars->sfree[sl]);
+      mbar_arrive(&bars->xfree[xl]);
+    }
   }
   // the receivers this CTA still owes: the current one and any edgeless ones up to r_end
   while (ok && cur <= r_end) ok = flush();
@@ -333,82 +387,92 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
 
 // ---------------------------------------------------------------- setup warps
 
-// Setup warp s handles the batches k = s, s + 2, ...: the sender rows (bulk copies, completion on
-// xfull), then the coefficients and the B operand (sfull).
+// Geometry warp s handles the MMA batches m = s, s + 2, ..., one edge per lane (the 32 edges of
+// batches 2 m and 2 m + 1): the coefficients of both subsets and the radial basis as the rows of
+// the B operand of MMA batch m.
 template <int L>
 __device__ __forceinline__ bool setup(const Args& a, unsigned char* smem, Bars* bars, int nb, int s) {
   using G = Cfg<L>;
-  constexpr int D = G::D, CW = G::CW;
+  constexpr int D = G::D;
   const int lane = threadIdx.x & 31;
   volatile int* abort_flag = &bars->abort_flag;
   float* cfbase = reinterpret_cast<float*>(smem + G::OFF_CF);
   float* rbase = reinterpret_cast<float*>(smem + G::OFF_RB);
-  float* xbase = reinterpret_cast<float*>(smem + G::OFF_X);
   const int e_beg = bars->e_beg, e_end = bars->e_end;
-  const uint32_t row_bytes = static_cast<uint32_t>(a.dim) * 4u;
-  // the edge vector and sender of this warp's next batch are loaded while the current one is set up
-  auto load_edge = [&](int k, float& vx, float& vy, float& vz, int& j) {
-    const int e = e_beg + k * kN + lane;
+  const int nbm = (nb + 1) / 2;
+  // the edge vectors of this warp's next MMA batch are loaded while the current one is set up
+  auto load_edge = [&](int m, float& vx, float& vy, float& vz) {
+    const int e = e_beg + m * kNM + lane;
     vx = vy = vz = 0.0f;
-    j = -1;
-    if (lane < kN && k < nb && e < e_end) {
+    if (m < nbm && e < e_end) {
       vx = __ldg(a.edge_vec + 3 * e);
       vy = __ldg(a.edge_vec + 3 * e + 1);
       vz = __ldg(a.edge_vec + 3 * e + 2);
-      j = __ldg(a.sender + e);
     }
   };
   float nvx, nvy, nvz;
-  int nj;
-  load_edge(s, nvx, nvy, nvz, nj);
+  load_edge(s, nvx, nvy, nvz);
   bool ok = true;
-  for (int k = s; k < nb; k += 2) {
-    const int sl = k % kSB;
-    const int e = e_beg + k * kN + lane;
+  for (int m = s; m < nbm; m += 2) {
+    const int k = 2 * m + (lane >> 4);   // this lane's consumer batch
+    const int sl = k % kGS;
+    const int e = e_beg + m * kNM + lane;
     const float vx = nvx, vy = nvy, vz = nvz;
-    const int j = nj;
-    load_edge(k + 2, nvx, nvy, nvz, nj);
-    if (k >= kSB && !warp_wait_lazy(&bars->sfree[sl], ((k / kSB) - 1) & 1, abort_flag, a.err, 34)) {
-      ok = false;
-      break;
+    load_edge(m + 2, nvx, nvy, nvz);
+    // both slots of the MMA batch must have been released by every consumer
+    if (2 * m >= kGS) {
+      ok = warp_wait_lazy(&bars->sfree[(2 * m) % kGS], ((2 * m / kGS) - 1) & 1, abort_flag, a.err, 34);
+      if (ok && 2 * m + 1 < nb)
+        ok = warp_wait_lazy(&bars->sfree[(2 * m + 1) % kGS], (((2 * m + 1) / kGS) - 1) & 1, abort_flag, a.err, 34);
+      if (!ok) break;
     }
-    // sender rows: one bulk copy per edge into the slot (lane i -> row i)
-    const unsigned valid = __ballot_sync(0xffffffffu, j >= 0);
-    if (lane == 0) {
-      mbar_expect_tx(&bars->xfull[sl], static_cast<uint32_t>(__popc(valid)) * row_bytes);
-      bars->x_last[sl] = k;   // a slot is reused only after sfree, so these writes are ordered
-    }
-    __syncwarp();
-    if (j >= 0)
-      bulk_g2s(xbase + static_cast<size_t>(sl * kN + lane) * a.dim, a.x + static_cast<size_t>(j) * a.dim, row_bytes,
-               &bars->xfull[sl]);
     float Y[D];
     float R[kNumBasis], dR[kNumBasis];
 #pragma unroll
     for (int c = 0; c < D; ++c) Y[c] = 0.0f;
 #pragma unroll
     for (int b = 0; b < kNumBasis; ++b) R[b] = 0.0f;
-    if (lane < kN && e < e_end) {
+    if (e < e_end) {
       const float dd = sqrtf(vx * vx + vy * vy + vz * vz);
       const float inv_d = dd > 0.0f ? 1.0f / dd : 0.0f;
       Gen<L>::sh(vx * inv_d, vy * inv_d, vz * inv_d, Y);
       radial_basis<false>(dd, a.inv_rc, R, dR);
     }
-    if (lane < kN) {
+    {
+      // coefficients of both subsets into the pair row of this edge: lane 2 j + t holds edge t of
+      // pair j; one exchange with the partner lane per two coefficients makes 8-byte stores of
+      // (c_k of edge 0, c_k of edge 1). The slot of a batch past the range is not written: it may
+      // still be read for an earlier batch.
       float c0[G::CW0], c1[G::CW1];
       G::S0::coef(Y, c0);
       G::S1::coef(Y, c1);
-      float4* row = reinterpret_cast<float4*>(cfbase + static_cast<size_t>(sl * kN + lane) * CW);
+      const int t = lane & 1;
+      float* prow = cfbase + static_cast<size_t>(sl * (kN / 2) + ((lane & (kN - 1)) >> 1)) * G::PW + 2 * t;
 #pragma unroll
-      for (int i = 0; i < G::CW0 / 4; ++i) row[i] = make_float4(c0[4 * i], c0[4 * i + 1], c0[4 * i + 2], c0[4 * i + 3]);
+      for (int i = 0; i < G::CW0 / 2; ++i) {
+        const float give = t == 0 ? c0[2 * i + 1] : c0[2 * i];
+        const float got = __shfl_xor_sync(kFull, give, 1);
+        if (k < nb)
+          *reinterpret_cast<float2*>(prow + 4 * i) = t == 0 ? make_float2(c0[2 * i], got) : make_float2(got, c0[2 * i + 1]);
+      }
 #pragma unroll
-      for (int i = 0; i < G::CW1 / 4; ++i)
-        row[G::CW0 / 4 + i] = make_float4(c1[4 * i], c1[4 * i + 1], c1[4 * i + 2], c1[4 * i + 3]);
+      for (int i = 0; i < G::CW1 / 2; ++i) {
+        const float give = t == 0 ? c1[2 * i + 1] : c1[2 * i];
+        const float got = __shfl_xor_sync(kFull, give, 1);
+        if (k < nb)
+          *reinterpret_cast<float2*>(prow + 2 * G::CW0 + 4 * i) =
+              t == 0 ? make_float2(c1[2 * i], got) : make_float2(got, c1[2 * i + 1]);
+      }
+    }
+    {
       float hh[kNumBasis], ll[kNumBasis];
 #pragma unroll
       for (int b = 0; b < kNumBasis; ++b) split_tf32(R[b], &hh[b], &ll[b]);
-      float* th = rbase + static_cast<size_t>(sl) * (2 * kN * 8);
-      float* tl = th + kN * 8;
+      // row `lane` of the B operand of MMA batch m, slot m % kRS. That slot was last read by the
+      // MMAs of batch m - kRS, which completed before the consumers finished its batches, whose
+      // geometry slot release this warp waited for.
+      float* th = rbase + static_cast<size_t>(m % kRS) * (2 * kNM * 8);
+      float* tl = th + kNM * 8;
       *reinterpret_cast<float4*>(th + canon(lane, 0)) = make_float4(hh[0], hh[1], hh[2], hh[3]);
       *reinterpret_cast<float4*>(th + canon(lane, 4)) = make_float4(hh[4], hh[5], hh[6], hh[7]);
       *reinterpret_cast<float4*>(tl + canon(lane, 0)) = make_float4(ll[0], ll[1], ll[2], ll[3]);
@@ -416,19 +480,56 @@ __device__ __forceinline__ bool setup(const Args& a, unsigned char* smem, Bars* 
     }
     fence_proxy_async();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars->sfull[sl]);
+    if (lane == 0) {
+      mbar_arrive(&bars->sfull[(2 * m) % kGS]);
+      if (2 * m + 1 < nb) mbar_arrive(&bars->sfull[(2 * m + 1) % kGS]);
+    }
   }
   return ok;
 }
 
+// ---------------------------------------------------------------- sender-row loader
+
+// One bulk copy per edge (the sender's whole row, dim floats) into the batch's slot, completion on
+// xfull; a slot is refilled once every consumer has read it (xfree).
+__device__ __forceinline__ bool load_rows(const Args& a, unsigned char* smem, Bars* bars, int nb, int off_x) {
+  const int lane = threadIdx.x & 31;
+  volatile int* abort_flag = &bars->abort_flag;
+  float* xbase = reinterpret_cast<float*>(smem + off_x);
+  const int e_beg = bars->e_beg, e_end = bars->e_end;
+  const uint32_t row_bytes = static_cast<uint32_t>(a.dim) * 4u;
+  auto load_j = [&](int k) {
+    const int e = e_beg + k * kN + lane;
+    return (lane < kN && k < nb && e < e_end) ? __ldg(a.sender + e) : -1;
+  };
+  int nj = load_j(0);
+  for (int k = 0; k < nb; ++k) {
+    const int xl = k % kXS;
+    const int j = nj;
+    nj = load_j(k + 1);
+    if (k >= kXS && !warp_wait_lazy(&bars->xfree[xl], ((k / kXS) - 1) & 1, abort_flag, a.err, 41)) return false;
+    const unsigned valid = __ballot_sync(0xffffffffu, j >= 0);
+    if (lane == 0) {
+      mbar_expect_tx(&bars->xfull[xl], static_cast<uint32_t>(__popc(valid)) * row_bytes);
+      bars->x_last[xl] = k;   // a slot is reused only after xfree, so these writes are ordered
+    }
+    __syncwarp();
+    if (j >= 0)
+      bulk_g2s(xbase + static_cast<size_t>(xl * kN + lane) * a.dim, a.x + static_cast<size_t>(j) * a.dim, row_bytes,
+               &bars->xfull[xl]);
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------- MMA thread
 
-// Issues batch after batch; returns the number of batches whose MMAs were committed.
+// Issues MMA batch after MMA batch (kNM edges: setup batches 2 m and 2 m + 1); returns the number of
+// MMA batches committed.
 template <int L>
 __device__ __forceinline__ int issue_mma(const Args& a, unsigned char* smem, Bars* bars, uint32_t tmem, int nb) {
   using G = Cfg<L>;
   constexpr int NB = G::NB;
-  constexpr uint32_t idesc = idesc_tf32(kN);
+  constexpr uint32_t idesc = idesc_tf32(kNM);
   volatile int* abort_flag = &bars->abort_flag;
   const float* wa = reinterpret_cast<const float*>(smem + G::OFF_WA);
   const float* rbase = reinterpret_cast<const float*>(smem + G::OFF_RB);
@@ -438,26 +539,30 @@ __device__ __forceinline__ int issue_mma(const Args& a, unsigned char* smem, Bar
     wdesc[2 * b] = smem_desc(sptr(wa + b * 2048));
     wdesc[2 * b + 1] = smem_desc(sptr(wa + b * 2048 + 1024));
   }
+  const int nbm = (nb + 1) / 2;
   int issued = 0;
-  for (int k = 0; k < nb; ++k) {
-    const int sl = k % kSB, ts = k & 1;
-    if (!mbar_wait(&bars->sfull[sl], (k / kSB) & 1, abort_flag, a.err, 35)) break;
-    if (k >= 2 && !mbar_wait(&bars->tempty[ts], ((k >> 1) - 1) & 1, abort_flag, a.err, 36)) break;
+  for (int m = 0; m < nbm; ++m) {
+    const int ts = m & 1;
+    bool ok = true;
+    for (int k = 2 * m; k < 2 * m + 2 && k < nb && ok; ++k)
+      ok = mbar_wait(&bars->sfull[k % kGS], (k / kGS) & 1, abort_flag, a.err, 35);
+    if (ok && m >= 2) ok = mbar_wait(&bars->tempty[ts], ((m >> 1) - 1) & 1, abort_flag, a.err, 36);
+    if (!ok) break;
     tc_fence_after();
-    const float* rb = rbase + static_cast<size_t>(sl) * (2 * kN * 8);
+    const float* rb = rbase + static_cast<size_t>(m % kRS) * (2 * kNM * 8);
     const uint64_t bh = smem_desc(sptr(rb));
-    const uint64_t bl = smem_desc(sptr(rb + kN * 8));
+    const uint64_t bl = smem_desc(sptr(rb + kNM * 8));
     const uint32_t d0 = tmem + ts * G::SLOTC;
     // the three products of the tf32 split accumulate into the same columns: issued pass by pass
-    // over the blocks, so consecutive MMAs are independent and the tensor core can overlap them
+    // over the blocks (measured faster than block by block)
 #pragma unroll
-    for (int b = 0; b < NB; ++b) mma_tf32(d0 + b * kN, wdesc[2 * b], bh, idesc, 0u);
+    for (int b = 0; b < NB; ++b) mma_tf32(d0 + b * kNM, wdesc[2 * b], bh, idesc, 0u);
 #pragma unroll
-    for (int b = 0; b < NB; ++b) mma_tf32(d0 + b * kN, wdesc[2 * b], bl, idesc, 1u);
+    for (int b = 0; b < NB; ++b) mma_tf32(d0 + b * kNM, wdesc[2 * b], bl, idesc, 1u);
 #pragma unroll
-    for (int b = 0; b < NB; ++b) mma_tf32(d0 + b * kN, wdesc[2 * b + 1], bh, idesc, 1u);
+    for (int b = 0; b < NB; ++b) mma_tf32(d0 + b * kNM, wdesc[2 * b + 1], bh, idesc, 1u);
     mma_commit(&bars->tfull[ts]);
-    issued = k + 1;
+    issued = m + 1;
   }
   return issued;
 }
@@ -568,10 +673,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_cx(Args a) {
       mbar_init(&bars->tfull[i], 1);
       mbar_init(&bars->tempty[i], kCons);
     }
-    for (int i = 0; i < kSB; ++i) {
+    for (int i = 0; i < kGS; ++i) {
       mbar_init(&bars->sfull[i], 1);
       mbar_init(&bars->sfree[i], kCons);
+    }
+    for (int i = 0; i < kXS; ++i) {
       mbar_init(&bars->xfull[i], 1);
+      mbar_init(&bars->xfree[i], kCons);
     }
     for (int i = 0; i < kNR; ++i) {
       mbar_init(&bars->rfull[i], kCons);
@@ -579,7 +687,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_cx(Args a) {
     }
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
-    for (int i = 0; i < kSB; ++i) bars->x_last[i] = -1;
+    for (int i = 0; i < kXS; ++i) bars->x_last[i] = -1;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   // the CTA's edge range and the receivers it owes: three independent binary searches over
@@ -639,14 +747,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_cx(Args a) {
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const uint32_t tmem = bars->tmem_holder;
   if (threadIdx.x == 0) {
     const int last = bars->e_beg, after = bars->e_end;
     bars->r_end = after > last ? after : last;
     bars->e_beg = eb;
     bars->e_end = ee;
   }
+  tc_fence_before();
   __syncthreads();
-  const uint32_t tmem = bars->tmem_holder;
+  tc_fence_after();
   const int nb = (ee - eb + kN - 1) / kN;
   bool drained = true;
 
@@ -670,6 +780,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_cx(Args a) {
     drained = __shfl_sync(kFull, drained ? 1 : 0, 0) != 0;
   } else if (warp == kCombWarp) {
     combine<L>(a, smem, bars);
+  } else if (warp == kLoadWarp) {
+    load_rows(a, smem, bars, nb, G::OFF_X);
   }
 
   // teardown: every thread reaches this barrier exactly once. Then the sender-row copies that may
@@ -678,9 +790,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_cx(Args a) {
   // batch issued into each slot can be outstanding.
   __syncthreads();
   if (warp == kCombWarp && lane == 0) {
-    for (int sl = 0; sl < kSB; ++sl) {
+    for (int sl = 0; sl < kXS; ++sl) {
       const int k = bars->x_last[sl];
-      if (k >= 0 && !mbar_wait_drain(&bars->xfull[sl], (k / kSB) & 1)) {
+      if (k >= 0 && !mbar_wait_drain(&bars->xfull[sl], (k / kXS) & 1)) {
         tc::report_code(a.err, 40);
         break;
       }

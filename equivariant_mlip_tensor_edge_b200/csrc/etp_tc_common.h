@@ -54,6 +54,21 @@ __device__ __forceinline__ void report_code(int* err, int code) {
   __threadfence_system();
 }
 
+// try_wait with a suspend-time hint: a thread whose phase is not complete sleeps in hardware until
+// the phase completes or about `ns` nanoseconds pass, instead of spinning on issue slots that the
+// working warps of its scheduler need.
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t* b, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(sptr(b)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on the phase of the given parity. Returns false (and raises the CTA abort flag and
 // records the error code) when the limit is exceeded or another thread has aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile int* abort_flag, int* err,
@@ -61,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity, volatile
   if (mbar_test(b, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_test(b, parity)) return true;
+    if (mbar_test_sleep(b, parity, 20000u)) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitCycles) {
       report_code(err, code);

@@ -650,7 +650,73 @@ def emit_cx(out, lmax):
         out.append("    }")
         out.append("  }")
         out.append(f"  static constexpr int FMA = {fma};   // FP32 instructions per edge and channel")
+        emit_cx_pair(out, sub, paths, ent, emap, nc, xi, oi)
         out.append("};")
+
+
+def emit_cx_pair(out, sub, paths, ent, emap, nc, xi, oi):
+    """The same contraction for two edges of one receiver at once, in packed FP32 (f32x2) arithmetic:
+    component .x belongs to the first edge, .y to the second. The coefficient row holds the two
+    edges' coefficients interleaved (coefficient k of edge t at float 2 k + t). A coefficient used
+    with a minus sign multiplies the negated x (exact), so each component sees exactly the roundings
+    of the one-edge code."""
+    nx, npth, no = len(xi), len(sub), len(oi)
+    body, neg = [], set()
+    for pi, p in enumerate(sub):
+        l1, l2, l3 = paths[p]
+        e = ent[p]
+        body.append(f"    {{ // path {p}: ({l1},{l2},{l3})")
+        if l2 == 0:
+            for m3, m1, terms in e:
+                o, xx = oi[idx(l3, m3 - l3)], xi[idx(l1, m1 - l1)]
+                body.append(f"      acc[{o}] = __ffma2_rn(w[{pi}], x[{xx}], acc[{o}]);")
+        elif (2 * l1 + 1) < (2 * l3 + 1):
+            sgn = {}
+            for m3, m1, _ in e:
+                ci, sg = emap[(p, m3, m1)]
+                sgn.setdefault(m1, set()).add(sg)
+            for m1 in range(2 * l1 + 1):
+                xx = xi[idx(l1, m1 - l1)]
+                if 1 in sgn.get(m1, ()):
+                    body.append(f"      const float2 xs{m1} = __fmul2_rn(w[{pi}], x[{xx}]);")
+                if -1 in sgn.get(m1, ()):
+                    neg.add(xx)
+                    body.append(f"      const float2 xn{m1} = __fmul2_rn(w[{pi}], xm[{xx}]);")
+            for m3, m1, _ in e:
+                ci, sg = emap[(p, m3, m1)]
+                o = oi[idx(l3, m3 - l3)]
+                src = f"xs{m1}" if sg > 0 else f"xn{m1}"
+                body.append(f"      acc[{o}] = __ffma2_rn(cv[{ci}], {src}, acc[{o}]);")
+        else:
+            for m3 in range(2 * l3 + 1):
+                row = [(a, m1) for (a, m1, _) in e if a == m3]
+                if not row:
+                    continue
+                o = oi[idx(l3, m3 - l3)]
+                for j, (a, m1) in enumerate(row):
+                    ci, sg = emap[(p, a, m1)]
+                    xx = xi[idx(l1, m1 - l1)]
+                    if sg < 0:
+                        neg.add(xx)
+                    xv = f"x[{xx}]" if sg > 0 else f"xm[{xx}]"
+                    if j == 0:
+                        body.append(f"      float2 s{m3} = __fmul2_rn(cv[{ci}], {xv});")
+                    else:
+                        body.append(f"      s{m3} = __ffma2_rn(cv[{ci}], {xv}, s{m3});")
+                body.append(f"      acc[{o}] = __ffma2_rn(w[{pi}], s{m3}, acc[{o}]);")
+        body.append("    }")
+    out.append(f"  __device__ __forceinline__ static void fwd2(const float4* __restrict__ cf, const float2 (&x)[{nx}],")
+    out.append(f"      const float2 (&w)[{npth}], float2 (&acc)[{no}]) {{")
+    for q in range(nc // 2):
+        out.append(f"    const float4 c4_{q} = cf[{q}];")
+    out.append(f"    const float2 cv[{nc}] = {{" + ", ".join(
+        f"make_float2(c4_{k // 2}.{'x' if k % 2 == 0 else 'z'}, c4_{k // 2}.{'y' if k % 2 == 0 else 'w'})" for k in range(nc)) + "};")
+    if neg:
+        out.append(f"    float2 xm[{nx}];")
+        for xx in sorted(neg):
+            out.append(f"    xm[{xx}] = __fmul2_rn(x[{xx}], make_float2(-1.0f, -1.0f));")
+    out.extend(body)
+    out.append("  }")
 
 
 # ---------------------------------------------------------------- general irreps
