@@ -4,6 +4,7 @@
 #include <cub/cub.cuh>
 
 #include <cmath>
+#include <cstdlib>
 #include <string>
 
 #include "etp_internal.h"
@@ -171,6 +172,205 @@ __global__ void k_nbr_emit(const float* __restrict__ pos, int n, int n_chunks, C
   }
 }
 
+// ------------------------------------------------------------------ cell binning
+// The binned search finds the same edge set as the all-pairs scan above: it only narrows the
+// candidates (j, S) that reach pair_test. Atoms are binned by fractional coordinate
+// f = pos inv(cell) (Cartesian coordinates when there is no cell). Periodic axis a: nb_a bins of
+// width 1 / nb_a in f, i.e. at least r_cut (1 + 1e-6) along the plane normal; an atom's bin is
+// floor((f - floor f) nb_a) and its wrap count floor f. Non-periodic axis: bins of width
+// r_cut (1 + 1e-6) / spacing_a in f, bin floor(f / width). Two points within r_cut differ by less
+// than r_cut / spacing_a in f_a, so their bins differ by at most K_a on every axis; the candidates
+// of receiver i are the atoms of the bins b_i + d, |d_a| <= K_a, with image S_a = q_a + w_i - w_j
+// (q_a: the wrap of b_i + d on a periodic axis, 0 otherwise), kept iff |S_a| <= n_a and the exact
+// pair_test passes. Each kept pair then goes to its rank by (sender, S) within the row, which is
+// the canonical order.
+struct BinParams {
+  double inv[9];     // f_a = sum_k pos_k inv[3 k + a]
+  int periodic[3];
+  int nb[3];         // periodic axes: bins per axis
+  double width[3];   // non-periodic axes: bin width in f
+  int K[3];          // bin offsets scanned per axis: d_a in [-K_a, K_a]
+  int n_off;         // (2 K0 + 1)(2 K1 + 1)(2 K2 + 1)
+  long long n_s;     // images per sender: (2 n0 + 1)(2 n1 + 1)(2 n2 + 1)
+};
+
+constexpr int kBinBias = 1 << 20;           // bin coordinates are stored biased, in 21 bits
+constexpr unsigned long long kBinMask = (1ull << 21) - 1;
+
+__device__ __forceinline__ unsigned long long bin_key(int b0, int b1, int b2) {
+  return (static_cast<unsigned long long>(b0 + kBinBias) << 42) |
+         (static_cast<unsigned long long>(b1 + kBinBias) << 21) | static_cast<unsigned long long>(b2 + kBinBias);
+}
+
+__device__ __forceinline__ int key_coord(unsigned long long key, int a) {
+  return static_cast<int>((key >> (21 * (2 - a))) & kBinMask) - kBinBias;
+}
+
+// Per atom: its bin key (this unsorted array also serves the receiver side), the atom id, its wrap
+// counts.
+// flag bit 0: a coordinate outside the representable bin range (the caller then scans all pairs).
+__global__ void k_bin_atoms(const float* __restrict__ pos, int n, BinParams bp, unsigned long long* __restrict__ key,
+                            int* __restrict__ atom, int* __restrict__ wrap, int* __restrict__ flag) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const double p[3] = {static_cast<double>(pos[3 * i]), static_cast<double>(pos[3 * i + 1]),
+                         static_cast<double>(pos[3 * i + 2])};
+    int b[3];
+    for (int a = 0; a < 3; ++a) {
+      const double f = (p[0] * bp.inv[a] + p[1] * bp.inv[3 + a]) + p[2] * bp.inv[6 + a];
+      int w = 0, bb;
+      if (bp.periodic[a]) {
+        const double fl = floor(f);
+        const bool fits = fabs(fl) < 1.0e8;   // wrap counts and their differences stay ints
+        if (!fits) atomicOr(flag, 1);
+        w = fits ? static_cast<int>(fl) : 0;
+        bb = static_cast<int>(floor((f - fl) * bp.nb[a]));
+        bb = bb < 0 ? 0 : (bb >= bp.nb[a] ? bp.nb[a] - 1 : bb);
+      } else {
+        const double q = floor(f / bp.width[a]);
+        if (!(fabs(q) < static_cast<double>(kBinBias - 4))) {
+          atomicOr(flag, 1);
+          bb = 0;
+        } else {
+          bb = static_cast<int>(q);
+        }
+      }
+      b[a] = bb;
+      wrap[3 * i + a] = w;
+    }
+    const unsigned long long k = bin_key(b[0], b[1], b[2]);
+    key[i] = k;
+    atom[i] = i;
+  }
+}
+
+__device__ __forceinline__ int lower_bound_u64(const unsigned long long* __restrict__ v, int n, unsigned long long x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (v[mid] < x) lo = mid + 1; else hi = mid;
+  }
+  return lo;
+}
+
+// One warp per receiver. EMIT = false: counts[i] = kept pairs. EMIT = true: the row's keys
+// (sender * n_s + image index) are first written in bin order to the row's slots of `ekey`; then
+// every key goes to its canonical place, base + (number of smaller keys in the row), where its
+// sender, image and r (recomputed by the same pair_test) are stored, with the receiver.
+template <bool EMIT>
+__global__ void k_bin_pairs(const float* __restrict__ pos, int n, CellParams cp, BinParams bp,
+                            const unsigned long long* __restrict__ skey, const int* __restrict__ satom,
+                            const unsigned long long* __restrict__ akey, const int* __restrict__ wrap,
+                            int* __restrict__ counts, const int* __restrict__ row_ptr,
+                            unsigned long long* __restrict__ ekey, int* __restrict__ receiver,
+                            int* __restrict__ sender, float* __restrict__ edge_vec, int* __restrict__ shift) {
+  const int lane = threadIdx.x & 31;
+  const int stride = gridDim.x * (blockDim.x >> 5);
+  for (int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); i < n; i += stride) {
+    const float3 pi = load_pos(pos, i);
+    const unsigned long long ki = akey[i];
+    const int bi[3] = {key_coord(ki, 0), key_coord(ki, 1), key_coord(ki, 2)};
+    const int wi[3] = {wrap[3 * i], wrap[3 * i + 1], wrap[3 * i + 2]};
+    int count = 0;
+    const int base = EMIT ? row_ptr[i] : 0;
+    const int row_end = EMIT ? row_ptr[i + 1] : 0;   // the count pass kept exactly this many
+    for (int o0 = 0; o0 < bp.n_off; o0 += 32) {
+      // lane o: the bin b_i + d of offset index o0 + lane, its atom range and wrap
+      const int o = o0 + lane;
+      bool have = o < bp.n_off;
+      int lo = 0, hi = 0, q[3] = {0, 0, 0};
+      if (have) {
+        int rem = o, bb[3];
+        for (int a = 2; a >= 0; --a) {
+          const int span = 2 * bp.K[a] + 1;
+          const int d = rem % span - bp.K[a];
+          rem /= span;
+          int u = bi[a] + d;
+          if (bp.periodic[a]) {
+            const int nb = bp.nb[a];
+            const int qq = u >= 0 ? u / nb : -((-u + nb - 1) / nb);
+            q[a] = qq;
+            u -= qq * nb;
+          } else if (u <= -kBinBias || u >= kBinBias) {
+            have = false;
+          }
+          bb[a] = u;
+        }
+        if (have) {
+          const unsigned long long kb = bin_key(bb[0], bb[1], bb[2]);
+          lo = lower_bound_u64(skey, n, kb);
+          hi = lower_bound_u64(skey, n, kb + 1);
+        }
+      }
+      for (int src = 0; src < 32; ++src) {
+        const int blo = __shfl_sync(0xffffffffu, lo, src);
+        const int bhi = __shfl_sync(0xffffffffu, hi, src);
+        const int q0 = __shfl_sync(0xffffffffu, q[0], src);
+        const int q1 = __shfl_sync(0xffffffffu, q[1], src);
+        const int q2 = __shfl_sync(0xffffffffu, q[2], src);
+        for (int t = blo; t < bhi; t += 32) {
+          const int idx = t + lane;
+          bool keep = false;
+          int j = 0, s0 = 0, s1 = 0, s2 = 0;
+          if (idx < bhi) {
+            j = satom[idx];
+            s0 = bp.periodic[0] ? q0 + wi[0] - wrap[3 * j] : 0;
+            s1 = bp.periodic[1] ? q1 + wi[1] - wrap[3 * j + 1] : 0;
+            s2 = bp.periodic[2] ? q2 + wi[2] - wrap[3 * j + 2] : 0;
+            keep = abs(s0) <= cp.n[0] && abs(s1) <= cp.n[1] && abs(s2) <= cp.n[2] &&
+                   !(j == i && s0 == 0 && s1 == 0 && s2 == 0);
+            if (keep) {
+              double rx, ry, rz;
+              keep = pair_test(pi, load_pos(pos, j), s0, s1, s2, cp, &rx, &ry, &rz);
+            }
+          }
+          const unsigned m = __ballot_sync(0xffffffffu, keep);
+          const int at = base + count + __popc(m & ((1u << lane) - 1u));
+          if (EMIT && keep && at < row_end) {
+            const long long sidx =
+                (static_cast<long long>(s0 + cp.n[0]) * (2 * cp.n[1] + 1) + (s1 + cp.n[1])) * (2 * cp.n[2] + 1) +
+                (s2 + cp.n[2]);
+            ekey[at] = static_cast<unsigned long long>(j) * static_cast<unsigned long long>(bp.n_s) +
+                       static_cast<unsigned long long>(sidx);
+          }
+          count += __popc(m);
+        }
+      }
+    }
+    if (!EMIT) {
+      if (lane == 0) counts[i] = count;
+      continue;
+    }
+    __syncwarp();   // the row's keys, written by every lane, are visible to the whole warp
+    const int len = row_end - base;
+    const int w2 = 2 * cp.n[2] + 1, w1 = 2 * cp.n[1] + 1;
+    for (int t = lane; t < len; t += 32) {
+      const unsigned long long key = ekey[base + t];
+      int rank = 0;
+      for (int u = 0; u < len; ++u) rank += ekey[base + u] < key ? 1 : 0;   // keys are distinct
+      const int j = static_cast<int>(key / static_cast<unsigned long long>(bp.n_s));
+      long long sidx = static_cast<long long>(key % static_cast<unsigned long long>(bp.n_s));
+      const int s2 = static_cast<int>(sidx % w2) - cp.n[2];
+      sidx /= w2;
+      const int s1 = static_cast<int>(sidx % w1) - cp.n[1];
+      const int s0 = static_cast<int>(sidx / w1) - cp.n[0];
+      if (j < 0 || j >= n) continue;   // never taken: both passes keep the same pairs
+      double rx, ry, rz;
+      pair_test(pi, load_pos(pos, j), s0, s1, s2, cp, &rx, &ry, &rz);
+      const int at = base + rank;
+      sender[at] = j;
+      receiver[at] = i;
+      edge_vec[3 * at + 0] = static_cast<float>(rx);
+      edge_vec[3 * at + 1] = static_cast<float>(ry);
+      edge_vec[3 * at + 2] = static_cast<float>(rz);
+      if (shift) {
+        shift[3 * at + 0] = s0;
+        shift[3 * at + 1] = s1;
+        shift[3 * at + 2] = s2;
+      }
+    }
+  }
+}
+
 // Nearest-image lists are symmetric with at most one image per pair, and the image of j <- i is
 // minus that of i <- j (rint and the clamp are odd functions). So the transposed order needs no
 // sort: the edges j sends, in receiver order, are the reverses of row j's edges in sender order,
@@ -248,6 +448,12 @@ struct GraphWs {
   int* vb;
   int* pm;
   int* flag;
+  // binned search: per-atom bin keys (sorted and in atom order), atom ids, wrap counts
+  unsigned long long* bkey;
+  unsigned long long* bkey_sorted;
+  int* batom;
+  int* batom_sorted;
+  int* wrap;
   void* cub_tmp;
   size_t cub_bytes;
 };
@@ -261,7 +467,18 @@ size_t cub_temp_bytes(int n_nodes, int max_edges) {
                                   static_cast<int*>(nullptr), static_cast<const int*>(nullptr),
                                   static_cast<int*>(nullptr), max_edges > 0 ? max_edges : 1, 0,
                                   key_bits(n_nodes));
-  return scan_b > sort_b ? scan_b : sort_b;
+  size_t bin_b = 0;
+  cub::DeviceRadixSort::SortPairs(nullptr, bin_b, static_cast<const unsigned long long*>(nullptr),
+                                  static_cast<unsigned long long*>(nullptr), static_cast<const int*>(nullptr),
+                                  static_cast<int*>(nullptr), n_nodes > 0 ? n_nodes : 1, 0, 63);
+  const size_t m = scan_b > sort_b ? scan_b : sort_b;
+  return m > bin_b ? m : bin_b;
+}
+
+// bytes of the binned search's per-atom arrays
+size_t bin_bytes(int n_nodes) {
+  const size_t n = static_cast<size_t>(n_nodes > 0 ? n_nodes : 1);
+  return 2 * align256(8 * n) + 2 * align256(4 * n) + align256(12 * n);
 }
 
 GraphWs carve(void* ws, int n_nodes, int max_edges) {
@@ -279,6 +496,12 @@ GraphWs carve(void* ws, int n_nodes, int max_edges) {
   g.vb = reinterpret_cast<int*>(p); p += eb;
   g.pm = reinterpret_cast<int*>(p); p += eb;
   g.flag = reinterpret_cast<int*>(p); p += 256;
+  const size_t n = static_cast<size_t>(n_nodes > 0 ? n_nodes : 1);
+  g.bkey = reinterpret_cast<unsigned long long*>(p); p += align256(8 * n);
+  g.bkey_sorted = reinterpret_cast<unsigned long long*>(p); p += align256(8 * n);
+  g.batom = reinterpret_cast<int*>(p); p += align256(4 * n);
+  g.batom_sorted = reinterpret_cast<int*>(p); p += align256(4 * n);
+  g.wrap = reinterpret_cast<int*>(p); p += align256(12 * n);
   g.cub_tmp = p;
   g.cub_bytes = cub_temp_bytes(n_nodes, max_edges);
   return g;
@@ -306,12 +529,163 @@ etp_status transpose(int n_nodes, int n_edges, const int* sender, int* t_row_ptr
   return cuda_status(cudaGetLastError(), "transpose");
 }
 
+
+enum class NbrMode { kAuto, kAllPairs, kBins };
+
+// ETP_NEIGHBORS = "bins" or "all-pairs" forces a search; unset, empty or "default" chooses.
+NbrMode nbr_mode() {
+  const char* v = std::getenv("ETP_NEIGHBORS");
+  if (!v || !*v) return NbrMode::kAuto;
+  const std::string m(v);
+  if (m == "bins") return NbrMode::kBins;
+  if (m == "all-pairs") return NbrMode::kAllPairs;
+  return NbrMode::kAuto;
+}
+
+// The bin layout (see BinParams). Returns whether binning is worth it by default: at least 2048
+// atoms, and on a fully periodic cell at least 4 x 4 x 4 bins (with fewer, every receiver scans
+// nearly every atom anyway). bp->n_off = 0 when no layout can be built.
+bool plan_bins(const double* cell, const int* pbc, double rc, int n_nodes, const CellParams& cp, BinParams* bp) {
+  bp->n_off = 0;
+  bp->n_s = static_cast<long long>(2 * cp.n[0] + 1) * (2 * cp.n[1] + 1) * (2 * cp.n[2] + 1);
+  if (!(rc > 0.0) || !std::isfinite(rc)) return false;
+  const double rcm = rc * (1.0 + 1e-6);
+  double spacing[3] = {1.0, 1.0, 1.0};
+  for (int k = 0; k < 9; ++k) bp->inv[k] = (k % 4 == 0) ? 1.0 : 0.0;
+  if (cell) {
+    const double* c = cell;
+    const double det = c[0] * (c[4] * c[8] - c[5] * c[7]) - c[1] * (c[3] * c[8] - c[5] * c[6]) +
+                       c[2] * (c[3] * c[7] - c[4] * c[6]);
+    if (!(std::fabs(det) > 0.0)) return false;
+    // inverse by cofactors: inv[3 k + a] = cof(a, k) / det
+    bp->inv[0] = (c[4] * c[8] - c[5] * c[7]) / det;
+    bp->inv[1] = (c[2] * c[7] - c[1] * c[8]) / det;
+    bp->inv[2] = (c[1] * c[5] - c[2] * c[4]) / det;
+    bp->inv[3] = (c[5] * c[6] - c[3] * c[8]) / det;
+    bp->inv[4] = (c[0] * c[8] - c[2] * c[6]) / det;
+    bp->inv[5] = (c[2] * c[3] - c[0] * c[5]) / det;
+    bp->inv[6] = (c[3] * c[7] - c[4] * c[6]) / det;
+    bp->inv[7] = (c[1] * c[6] - c[0] * c[7]) / det;
+    bp->inv[8] = (c[0] * c[4] - c[1] * c[3]) / det;
+    for (int a = 0; a < 3; ++a) {
+      const double* u = c + 3 * ((a + 1) % 3);
+      const double* w = c + 3 * ((a + 2) % 3);
+      const double cx = u[1] * w[2] - u[2] * w[1], cy = u[2] * w[0] - u[0] * w[2], cz = u[0] * w[1] - u[1] * w[0];
+      spacing[a] = std::fabs(det) / std::sqrt(cx * cx + cy * cy + cz * cz);
+      if (!(spacing[a] > 0.0)) return false;
+    }
+  }
+  long long periodic_bins = 1;
+  bool all_periodic = true;
+  bp->n_off = 1;
+  for (int a = 0; a < 3; ++a) {
+    bp->periodic[a] = (cell && pbc && pbc[a]) ? 1 : 0;
+    if (bp->periodic[a]) {
+      const double per = std::floor(spacing[a] / rcm);
+      bp->nb[a] = per >= 1.0 ? (per < 1e6 ? static_cast<int>(per) : 1000000) : 1;
+      bp->K[a] = static_cast<int>(std::ceil(rcm * bp->nb[a] / spacing[a]));
+      if (bp->K[a] < 1) bp->K[a] = 1;
+      bp->width[a] = 1.0 / bp->nb[a];
+      periodic_bins *= bp->nb[a];
+    } else {
+      all_periodic = false;
+      bp->nb[a] = 1;
+      bp->K[a] = 1;
+      bp->width[a] = rcm / spacing[a];
+    }
+    if (bp->K[a] > 8) {   // a cell far thinner than r_cut: nothing to gain from bins
+      bp->n_off = 0;
+      return false;
+    }
+    bp->n_off *= 2 * bp->K[a] + 1;
+  }
+  if (n_nodes < 2048) return false;
+  return !(all_periodic && periodic_bins < 64);
+}
+
+// All-pairs search: row_ptr, sender, edge_vec, shift and the receiver of every edge (g.ka).
+etp_status neighbors_all_pairs(const float* pos, int n_nodes, const CellParams& cp, int max_edges, int* n_edges,
+                               int* row_ptr, int* sender, float* edge_vec, int* shift, GraphWs& g, cudaStream_t s) {
+  cudaError_t e;
+  const int n_chunks = n_chunks_of(n_nodes);
+  const long long n_tasks = static_cast<long long>(n_nodes) * n_chunks;
+  const int task_blocks = grid_for(n_tasks * 32, 256);
+  if (n_nodes > 0) {
+    k_nbr_count<<<task_blocks, 256, 0, s>>>(pos, n_nodes, n_chunks, cp, g.counts);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour count");
+    size_t tb = g.cub_bytes;
+    e = cub::DeviceScan::InclusiveSum(g.cub_tmp, tb, g.counts, g.incl, static_cast<int>(n_tasks), s);
+    if (e != cudaSuccess) return cuda_status(e, "neighbour scan");
+  }
+  k_row_ptr_chunks<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.incl, n_nodes, n_chunks, row_ptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "row pointers");
+  int total = 0;
+  if ((e = cudaMemcpyAsync(&total, row_ptr + n_nodes, sizeof(int), cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_status(e, "read edge count");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_status(e, "neighbour count sync");
+  *n_edges = total;
+  if (total > max_edges) {
+    set_error("etp_neighbors: " + std::to_string(total) + " edges exceed max_edges");
+    return ETP_ERR_CAPACITY;
+  }
+  if (n_nodes > 0 && total > 0) {
+    k_nbr_emit<<<task_blocks, 256, 0, s>>>(pos, n_nodes, n_chunks, cp, g.counts, g.incl, sender, edge_vec, shift,
+                                           g.ka);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour emit");
+  }
+  return ETP_OK;
+}
+
+// Binned search, same outputs. *done = false (nothing written that the all-pairs search does not
+// rewrite) when a coordinate falls outside the representable bin range.
+etp_status neighbors_binned(const float* pos, int n_nodes, const CellParams& cp, const BinParams& bp, int max_edges,
+                            int* n_edges, int* row_ptr, int* sender, float* edge_vec, int* shift, GraphWs& g,
+                            cudaStream_t s, bool* done) {
+  *done = false;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(g.flag, 0, sizeof(int), s)) != cudaSuccess) return cuda_status(e, "memset");
+  k_bin_atoms<<<grid_for(n_nodes, 256), 256, 0, s>>>(pos, n_nodes, bp, g.bkey, g.batom, g.wrap, g.flag);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "bin atoms");
+  size_t tb = g.cub_bytes;
+  e = cub::DeviceRadixSort::SortPairs(g.cub_tmp, tb, g.bkey, g.bkey_sorted, g.batom, g.batom_sorted, n_nodes, 0, 63,
+                                      s);
+  if (e != cudaSuccess) return cuda_status(e, "bin sort");
+  const int warp_blocks = grid_for(static_cast<long long>(n_nodes) * 32, 256);
+  k_bin_pairs<false><<<warp_blocks, 256, 0, s>>>(pos, n_nodes, cp, bp, g.bkey_sorted, g.batom_sorted, g.bkey, g.wrap,
+                                                 g.counts, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "binned count");
+  tb = g.cub_bytes;
+  e = cub::DeviceScan::InclusiveSum(g.cub_tmp, tb, g.counts, g.incl, n_nodes, s);
+  if (e != cudaSuccess) return cuda_status(e, "binned scan");
+  k_row_ptr_chunks<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.incl, n_nodes, 1, row_ptr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "row pointers");
+  int total = 0, flag = 0;
+  if ((e = cudaMemcpyAsync(&total, row_ptr + n_nodes, sizeof(int), cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_status(e, "read edge count");
+  if ((e = cudaMemcpyAsync(&flag, g.flag, sizeof(int), cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+    return cuda_status(e, "read bin flag");
+  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_status(e, "neighbour count sync");
+  if (flag) return ETP_OK;   // coordinates beyond the bin range: the caller scans all pairs
+  *done = true;
+  *n_edges = total;
+  if (total > max_edges) {
+    set_error("etp_neighbors: " + std::to_string(total) + " edges exceed max_edges");
+    return ETP_ERR_CAPACITY;
+  }
+  if (total == 0) return ETP_OK;
+  // the rows' edge keys (sender * n_s + image index), in bin order, in [kb, va)
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(g.kb);
+  k_bin_pairs<true><<<warp_blocks, 256, 0, s>>>(pos, n_nodes, cp, bp, g.bkey_sorted, g.batom_sorted, g.bkey, g.wrap,
+                                                nullptr, row_ptr, keys, g.ka, sender, edge_vec, shift);
+  return cuda_status(cudaGetLastError(), "binned emit");
+}
+
 }  // namespace
 
 size_t graph_workspace_bytes(int n_nodes, int max_edges) {
   const size_t eb = align256(sizeof(int) * static_cast<size_t>(max_edges > 0 ? max_edges : 1));
   const size_t cb = align256(sizeof(int) * (static_cast<size_t>(n_nodes) * n_chunks_of(n_nodes) + 1));
-  return 2 * cb + 5 * eb + 256 + align256(cub_temp_bytes(n_nodes, max_edges));
+  return 2 * cb + 5 * eb + 256 + bin_bytes(n_nodes) + align256(cub_temp_bytes(n_nodes, max_edges));
 }
 
 etp_status neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,
@@ -356,33 +730,23 @@ etp_status neighbors(const float* pos, int n_nodes, const double* cell, const in
     cp.n[0] = cp.n[1] = cp.n[2] = 0;
   }
   GraphWs g = carve(ws, n_nodes, max_edges);
+  BinParams bp;
+  const NbrMode mode = nbr_mode();
+  const bool bins_help = plan_bins(cell, pbc, rc, n_nodes, cp, &bp);
+  const bool use_bins = n_nodes > 0 && cp.rc2 > 0.0 && mode != NbrMode::kAllPairs &&
+                        (mode == NbrMode::kBins ? bp.n_off > 0 : bins_help);
+  etp_status st = ETP_OK;
+  bool done = false;
+  if (use_bins) {
+    st = neighbors_binned(pos, n_nodes, cp, bp, max_edges, n_edges, row_ptr, sender, edge_vec, shift, g, s, &done);
+    if (st != ETP_OK) return st;
+  }
+  if (!done) {
+    st = neighbors_all_pairs(pos, n_nodes, cp, max_edges, n_edges, row_ptr, sender, edge_vec, shift, g, s);
+    if (st != ETP_OK) return st;
+  }
+  const int total = *n_edges;
   cudaError_t e;
-  const int n_chunks = n_chunks_of(n_nodes);
-  const long long n_tasks = static_cast<long long>(n_nodes) * n_chunks;
-  const int task_blocks = grid_for(n_tasks * 32, 256);
-  if (n_nodes > 0) {
-    k_nbr_count<<<task_blocks, 256, 0, s>>>(pos, n_nodes, n_chunks, cp, g.counts);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour count");
-    size_t tb = g.cub_bytes;
-    e = cub::DeviceScan::InclusiveSum(g.cub_tmp, tb, g.counts, g.incl, static_cast<int>(n_tasks), s);
-    if (e != cudaSuccess) return cuda_status(e, "neighbour scan");
-  }
-  k_row_ptr_chunks<<<grid_for(n_nodes + 1, 256), 256, 0, s>>>(g.incl, n_nodes, n_chunks, row_ptr);
-  if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "row pointers");
-  int total = 0;
-  if ((e = cudaMemcpyAsync(&total, row_ptr + n_nodes, sizeof(int), cudaMemcpyDeviceToHost, s)) != cudaSuccess)
-    return cuda_status(e, "read edge count");
-  if ((e = cudaStreamSynchronize(s)) != cudaSuccess) return cuda_status(e, "neighbour count sync");
-  *n_edges = total;
-  if (total > max_edges) {
-    set_error("etp_neighbors: " + std::to_string(total) + " edges exceed max_edges");
-    return ETP_ERR_CAPACITY;
-  }
-  if (n_nodes > 0 && total > 0) {
-    k_nbr_emit<<<task_blocks, 256, 0, s>>>(pos, n_nodes, n_chunks, cp, g.counts, g.incl, sender, edge_vec, shift,
-                                           g.ka);
-    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "neighbour emit");
-  }
   if (cp.min_image) {
     e = cudaMemcpyAsync(t_row_ptr, row_ptr, sizeof(int) * (static_cast<size_t>(n_nodes) + 1),
                         cudaMemcpyDeviceToDevice, s);

@@ -251,7 +251,9 @@ etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, 
 etp_status etp_forces(int n_nodes, int n_edges, const int* row_ptr, const int* t_row_ptr,
                       const int* t_perm, const float* grad_edge_vec, float* forces, void* stream);
 
-/* ---- graph construction (integer outputs are bit-exact against a float64 brute force) ---- */
+/* ---- graph construction (integer outputs are bit-exact against a float64 brute force) ----
+ * Defined by the pages' force workloads, which build the neighbour graph of periodic cells with
+ * ghost images ("Fast and Accurate Foundation Models...", section V). */
 
 /* Device workspace for etp_neighbors / etp_build_csr with up to max_edges edges. */
 size_t etp_graph_workspace_bytes(int n_nodes, int max_edges);
@@ -264,8 +266,14 @@ size_t etp_graph_workspace_bytes(int n_nodes, int max_edges);
  * scanning every image with |S_a| <= ceil(r_cut / plane spacing_a) on periodic axes.
  * Outputs (device, capacity max_edges): row_ptr, sender, edge_vec (= float32(r)), shift
  * [max_edges][3] (may be NULL), t_row_ptr, t_perm. *n_edges (HOST) receives the edge count;
- * this call synchronises `stream` once to read it. If the count exceeds max_edges the call
- * returns ETP_ERR_CAPACITY after filling row_ptr only. */
+ * this call synchronises `stream` once to read it (twice if it falls back, below). If the count
+ * exceeds max_edges the call returns ETP_ERR_CAPACITY after filling row_ptr only.
+ * Search: from 2048 atoms (and, on a fully periodic cell, at least 4 x 4 x 4 bins of width >=
+ * r_cut), atoms are binned by fractional coordinate and each receiver tests only the atoms of its
+ * neighbouring bins; otherwise every pair is tested. Both apply the test above to the same
+ * candidate images and produce identical outputs. Environment variable ETP_NEIGHBORS = "bins" or
+ * "all-pairs" forces one; coordinates beyond about 1e8 cell lengths (or 1e6 r_cut on a
+ * non-periodic axis) fall back to all pairs. */
 etp_status etp_neighbors(const float* pos, int n_nodes, const double* cell, const int* pbc,
                          float r_cut, int max_edges, int* n_edges, int* row_ptr, int* sender,
                          float* edge_vec, int* shift, int* t_row_ptr, int* t_perm,

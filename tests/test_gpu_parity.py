@@ -65,8 +65,10 @@ def _gpu_receivers(g):
 
 # ------------------------------------------------------------------ graph
 
+@pytest.mark.parametrize("search", ["default", "bins", "all-pairs"])
 @pytest.mark.parametrize("name", ["tiny", "diamond1k"])
-def test_neighbors_bit_exact_full(wls, name):
+def test_neighbors_bit_exact_full(wls, name, search, monkeypatch):
+    monkeypatch.setenv("ETP_NEIGHBORS", search)
     wl = wls(name)
     ref = full_graph(wl)
     g = _gpu_graph(wl)
@@ -92,10 +94,13 @@ class _Cell:
         self.n_nodes = n
 
 
+@pytest.mark.parametrize("search", ["bins", "all-pairs"])
 @pytest.mark.parametrize("case", ["orthorhombic_small", "triclinic", "slab"])
-def test_neighbors_bit_exact_image_scan(case):
+def test_neighbors_bit_exact_image_scan(case, search, monkeypatch):
     """Cells where the nearest-image shortcut does not apply: a periodic length below 2 r_cut
-    (several images of one pair), a sheared cell, and a slab periodic in two axes only."""
+    (several images of one pair), a sheared cell, and a slab periodic in two axes only; both the
+    binned and the all-pairs search against the oracle."""
+    monkeypatch.setenv("ETP_NEIGHBORS", search)
     if case == "orthorhombic_small":
         sysm = _Cell(np.diag([7.1, 7.6, 8.3]), 40, seed=21)
     elif case == "triclinic":
@@ -112,6 +117,36 @@ def test_neighbors_bit_exact_image_scan(case):
     assert np.array_equal(_np(g.edge_vec).view(np.uint32), ref["edge_vec"].view(np.uint32))
     assert np.array_equal(_np(g.t_row_ptr), ref["t_row_ptr"])
     assert np.array_equal(_np(g.t_perm), ref["t_perm"])
+
+
+def _graph_arrays(g):
+    return [_np(a) for a in (g.row_ptr, g.sender, g.shift, g.edge_vec.view(torch.int32), g.t_row_ptr, g.t_perm)]
+
+
+def _uniform_positions(n, seed, box):
+    return (np.random.default_rng(seed).random((n, 3)) * np.asarray(box)).astype(np.float32)
+
+
+@pytest.mark.parametrize("case", ["diamond8k", "melt32k", "cluster", "slab"])
+def test_neighbors_binned_equals_all_pairs(wls, case, monkeypatch):
+    """Large systems where the default search bins the atoms: every output of the binned search is
+    bit for bit the all-pairs search's (which the oracle pins on the small cells above)."""
+    if case in ("diamond8k", "melt32k"):
+        wl = wls(case)
+        pos, rc, cell, pbc = wl.pos, float(wl.r_cut), wl.cell, wl.pbc
+    elif case == "cluster":   # no cell at all
+        pos, rc, cell, pbc = _uniform_positions(3000, 31, 40.0), 5.0, None, (False, False, False)
+    else:                     # periodic in x and y only, 4000 atoms in a 36 x 36 x 40 slab
+        pos, rc, cell, pbc = _uniform_positions(4000, 32, (36.0, 36.0, 40.0)), 5.0, np.diag([36.0, 36.0, 60.0]), \
+            (True, True, False)
+    pd = torch.from_numpy(np.asarray(pos, np.float32)).to(DEV)
+    res = {}
+    for search in ("default", "bins", "all-pairs"):
+        monkeypatch.setenv("ETP_NEIGHBORS", search)
+        res[search] = _graph_arrays(etp.neighbors(pd, rc, cell=cell, pbc=pbc))
+    for search in ("default", "bins"):
+        for a, b, what in zip(res[search], res["all-pairs"], ("row_ptr", "sender", "shift", "edge_vec", "t_row_ptr", "t_perm")):
+            assert np.array_equal(a, b), f"{case}: {search} search differs from all-pairs in {what}"
 
 
 @pytest.mark.parametrize("name", ["diamond8k", "melt32k"])
@@ -797,8 +832,10 @@ def test_general_irreps_weight_grad_parity(wls, irin, sh, irout):
 
 
 def test_general_irreps_weight_grad_full_size(wls):
-    """NequIP-L channel counts on the 1000-atom diamond cell: dL/dW against <dW, dW'> = directional
-    derivative of <grad_out, out> (exact: the output is linear in W), through the forward kernel."""
+    """NequIP-L channel counts on the 1000-atom diamond cell: dL/dW against the oracle's weight VJP
+    over the whole graph; as an extra, <dW, V> against the directional derivative <grad_out, F(V)>
+    (exact: the output is linear in W), through the forward kernel."""
+    from oracle.conv import conv_vjp_weights
     wl = wls("diamond1k")
     irr = "128x0e+64x1o+32x2e+32x3o"
     conv = etp.EdgeConv(irr, 3, irr, 8, float(wl.r_cut))
@@ -807,6 +844,9 @@ def test_general_irreps_weight_grad_full_size(wls):
     g = _gpu_graph(wl)
     xd, Wd, gd = (torch.from_numpy(a).to(DEV) for a in (x, W, gout))
     dW = conv.backward_weights(g, xd, gd).double()
+    ref_g = full_graph(wl)
+    ref = conv_vjp_weights(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, gout)
+    assert_close_rel(_np(dW).reshape(ref.shape), ref, "NequIP-L diamond1k dL/dW vs oracle")
     dir_ = torch.from_numpy(np.random.default_rng(5).standard_normal(W.shape).astype(np.float32)).to(DEV)
     lhs = float((dW * dir_.double()).sum())
     rhs = float((conv.forward(g, xd, dir_).double() * gd.double()).sum())

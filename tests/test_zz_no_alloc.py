@@ -12,6 +12,7 @@ import pytest
 import equivariant_mlip_tensor_edge_b200 as etp
 import workloads
 from tests._oracle_side import assert_blocks_close
+from oracle.conv import ConvSpec, conv_forward
 
 ETP_ERR_CAPACITY = 6
 
@@ -26,17 +27,24 @@ def _noalloc(conv, g, x, W, out, stream):
                                    _ptr(g.edge_vec), _ptr(x), _ptr(W), _ptr(out), ctypes.c_void_p(stream))
 
 
-def _check_two_calls(conv, g, x, W, channels, lmax, what):
+def _check_two_calls(conv, g, x, W, channels, lmax, what, oracle_ref=None):
+    """Two no-alloc calls in a row against etp_forward and, when given, against the oracle."""
     import torch
     ref = conv.forward(g, x, W)
+    if oracle_ref is not None:
+        assert_blocks_close(ref.cpu().numpy().astype(np.float64), oracle_ref, channels, lmax,
+                            f"{what}: etp_forward vs oracle")
     stream = torch.cuda.current_stream().cuda_stream
     for call in range(2):
         out = torch.full_like(ref, float("nan"))
         st = _noalloc(conv, g, x, W, out, stream)
         assert st == 0, etp.load_library().etp_last_error().decode()
         torch.cuda.synchronize()
-        assert_blocks_close(out.cpu().numpy().astype(np.float64), ref.cpu().numpy().astype(np.float64),
-                            channels, lmax, f"{what}: no-alloc call {call + 1} vs etp_forward")
+        got = out.cpu().numpy().astype(np.float64)
+        assert_blocks_close(got, ref.cpu().numpy().astype(np.float64), channels, lmax,
+                            f"{what}: no-alloc call {call + 1} vs etp_forward")
+        if oracle_ref is not None:
+            assert_blocks_close(got, oracle_ref, channels, lmax, f"{what}: no-alloc call {call + 1} vs oracle")
 
 
 @pytest.mark.gpu
@@ -53,7 +61,8 @@ def test_noalloc_forward_matches_workspace_forward(name):
 
 @pytest.mark.gpu
 def test_noalloc_forward_lmax3_largest_accepted_channels():
-    """lmax 3 with 160 channels: the largest scratch that fits the fixed array."""
+    """lmax 3 with 160 channels: the largest scratch that fits the fixed array. Both etp_forward and
+    the no-alloc entry are compared with the oracle on this ragged graph (degrees 0..69)."""
     import torch
     c, lmax, n = 160, 3, 40
     irr = "+".join(f"{c}x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
@@ -68,7 +77,10 @@ def test_noalloc_forward_lmax3_largest_accepted_channels():
                       torch.from_numpy(vec).to("cuda"))
     x = torch.from_numpy(rng.standard_normal((n, conv.info["dim_in"])).astype(np.float32)).to("cuda")
     W = torch.from_numpy((rng.standard_normal((8, conv.n_paths, c)) / np.sqrt(8)).astype(np.float32)).to("cuda")
-    _check_two_calls(conv, g, x, W, c, lmax, "lmax3 C160")
+    spec = ConvSpec(irr, lmax, irr, 8, 5.0)
+    row_ptr = np.concatenate([[0], np.cumsum(degrees)])
+    oracle_ref = conv_forward(spec, row_ptr, send, vec, x.cpu().numpy(), W.cpu().numpy())
+    _check_two_calls(conv, g, x, W, c, lmax, "lmax3 C160", oracle_ref=oracle_ref)
 
 
 def test_noalloc_forward_refuses_scratch_beyond_the_fixed_array():
