@@ -97,7 +97,7 @@ def algorithmic_counts(info, n_nodes, n_edges):
 # ---------------------------------------------------------------- recorded DRAM traffic
 
 CSRC = os.path.join(ROOT, "equivariant_mlip_tensor_edge_b200", "csrc")
-FWD_KERNEL = "k_fwd_cx"     # the default forward for l_max <= 2, C <= 128
+FWD_KERNEL = "k_fwd_cx"     # the default forward for l_max <= 2 and 4 <= C <= 64 (C % 4 == 0)
 KERNEL_SOURCES = {
     "k_fwd_cx": ["etp_fwd_cx.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_fwd_tc": ["etp_fwd_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
