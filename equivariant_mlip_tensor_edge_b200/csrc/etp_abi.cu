@@ -474,26 +474,22 @@ size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges) {
   const size_t f = tc::forward_tc_workspace_bytes(h->c, n_nodes);
   const size_t b = tc::backward_tc_workspace_bytes(h->c, n_edges);
   const size_t w = weight_grad_workspace_bytes(h->c, n_edges);
-  const size_t cmw = cm::workspace_bytes(h->c);
   const size_t cxw = cx::workspace_bytes(h->c);
   size_t m = f > b ? f : b;
   m = m > w ? m : w;
-  m = m > cmw ? m : cmw;
   return ws_tc_offset(n_edges) + (m > cxw ? m : cxw);
 }
 
 // Forward kernels. By default the channel-major path-subset kernel (etp_fwd_cx.cu) where it
-// applies (l_max <= 2, C <= 128), else the edge-major tensor-core kernel. ETP_FORWARD=edge selects
-// the edge-major kernel, ETP_FORWARD=channel the single-subset channel-major kernel (l_max <= 2,
-// C in {32, 64, 128}) and ETP_FORWARD=generic the all-FP32 one. Every kernel is tested.
+// applies (l_max <= 2, 4 <= C <= 64, C % 4 == 0), else the edge-major tensor-core kernel.
+// ETP_FORWARD=edge selects the edge-major kernel and ETP_FORWARD=generic the all-FP32 one. Every
+// kernel is tested.
 static bool forward_env_is(const char* name) {
   const char* v = std::getenv("ETP_FORWARD");
   return v && std::strcmp(v, name) == 0;
 }
 
 static bool use_tc_forward() { return !forward_env_is("generic"); }
-
-static bool use_cm_forward(const Ctx& c) { return cm::supported(c) && forward_env_is("channel"); }
 
 static bool use_cx_forward(const Ctx& c) {
   const char* v = std::getenv("ETP_FORWARD");
@@ -569,11 +565,6 @@ etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_pt
     if (use_cx_forward(h->c)) {
       st = cx::launch(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);
       if (st == ETP_OK && validate_requested()) st = cx::status(h->c, tcws, s);
-      return st;
-    }
-    if (use_cm_forward(h->c)) {
-      st = cm::launch(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);
-      if (st == ETP_OK && validate_requested()) st = cm::status(h->c, tcws, s);
       return st;
     }
     st = tc::launch_forward_tc(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s);

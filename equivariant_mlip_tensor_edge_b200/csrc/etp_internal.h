@@ -117,16 +117,7 @@ etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int*
                               cudaStream_t s, const uint32_t* path_mask = nullptr);
 }  // namespace tc
 
-// ---- channel-major forward (etp_fwd_cm.cu): l_max <= 2 and C in {32, 64, 128}
-namespace cm {
-bool supported(const Ctx& c);
-size_t workspace_bytes(const Ctx& c);
-etp_status launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, const int* sender,
-                  const float* edge_vec, const float* x, const float* W, float* out, void* ws, cudaStream_t s);
-etp_status status(const Ctx& c, const void* ws, cudaStream_t s);
-}  // namespace cm
-
-// ---- channel-major forward with path subsets (etp_fwd_cx.cu): l_max <= 2, C <= 128
+// ---- channel-major forward with path subsets (etp_fwd_cx.cu): l_max <= 2, 4 <= C <= 64, C % 4 == 0
 namespace cx {
 bool supported(const Ctx& c);
 size_t workspace_bytes(const Ctx& c);

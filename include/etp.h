@@ -154,12 +154,12 @@ size_t etp_workspace_bytes(etp_handle h, int n_nodes, int n_edges);
  * Spherical harmonics, radial basis, radial projection, Clebsch-Gordan contraction and the
  * per-receiver segmented sum run in one kernel pass; receivers without edges get zero rows.
  * Edges with d >= r_cut contribute zero (u = 0). workspace may be NULL when
- * etp_workspace_bytes returns 0. Kernel: for uniform handles with L <= 2 and C <= 128 the
+ * etp_workspace_bytes returns 0. Kernel: for uniform handles with L <= 2 and 4 <= C <= 64 the
  * channel-major path-subset kernel (the CTAs take equal contiguous ranges of canonical edges;
  * a receiver whose edges cross a range boundary is summed by the CTA that adds its last part,
  * in CTA order, so the result is still bitwise reproducible), else the edge-major tensor-core
- * kernel; the environment variable ETP_FORWARD=edge, channel or generic selects another
- * kernel (all agree with the float64 reference within the same tolerance). */
+ * kernel; the environment variable ETP_FORWARD=edge or generic selects another kernel (all
+ * agree with the float64 reference within the same tolerance). */
 etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_ptr,
                        const int* sender, const float* edge_vec, const float* x, const float* W,
                        float* out, void* workspace, size_t workspace_bytes, void* stream);

@@ -403,7 +403,7 @@ def test_no_cpu_fallback():
 
 # ------------------------------------------------------------------ forward kernels: both implementations
 
-@pytest.mark.parametrize("impl", ["default", "edge", "channel", "generic"])
+@pytest.mark.parametrize("impl", ["default", "edge", "generic"])
 @pytest.mark.parametrize("name", ["tiny", "diamond1k"])
 def test_forward_both_kernels(wls, name, impl, monkeypatch):
     if impl != "default":
@@ -601,41 +601,7 @@ def test_weight_grad_empty_graph_and_autograd(wls):
     assert torch.equal(Wt.grad, conv.backward_weights(g, xt, gout))
 
 
-# ------------------------------------------------------------------ channel-major forward
-
-@pytest.mark.parametrize("lmax,c", [(1, 32), (1, 64), (1, 128), (2, 32), (2, 64), (2, 128)])
-def test_forward_channel_major_ragged(lmax, c, monkeypatch):
-    """The channel-major kernel (l_max <= 2, C in {32, 64, 128}): empty rows at both ends and in
-    between, degrees up to several batches, receiver boundaries inside MMA batches; compared with
-    the oracle and with the edge-major kernel, and bitwise reproducible."""
-    from oracle.conv import ConvSpec
-    monkeypatch.setenv("ETP_VALIDATE", "1")
-    monkeypatch.setenv("ETP_FORWARD", "channel")
-    irr = "+".join(f"{c}x{l}{'eo'[l % 2]}" for l in range(lmax + 1))
-    degrees = np.array([0, 0, 1, 31, 32, 33, 0, 127, 128, 129, 300, 5, 0, 64, 97, 15, 17, 0])
-    n = len(degrees)
-    recv, send, vec = _random_graph(n, degrees, seed=40 + lmax + c)
-    conv = etp.EdgeConv(irr, lmax, irr, 8, 5.0)
-    spec = ConvSpec(irr, lmax, irr, 8, 5.0)
-    rng = np.random.default_rng(500 + lmax + c)
-    x = rng.standard_normal((n, spec.dim_in)).astype(np.float32)
-    W = (rng.standard_normal((8, len(spec.paths), c)) / np.sqrt(8)).astype(np.float32)
-    g = etp.build_csr(n, torch.from_numpy(recv).to(DEV), torch.from_numpy(send).to(DEV),
-                      torch.from_numpy(vec).to(DEV))
-    xd, Wd = torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)
-    out = conv.forward(g, xd, Wd)
-    again = conv.forward(g, xd, Wd)
-    assert torch.equal(out, again), "channel-major forward is not bitwise deterministic"
-    order = np.lexsort((send, recv))
-    rp = np.concatenate([[0], np.cumsum(degrees)])
-    ref = conv_forward(spec, rp, send[order], vec[order], x, W)
-    o = _np(out)
-    assert np.all(o[degrees == 0] == 0.0)
-    assert_blocks_close(o, ref, c, lmax, f"channel-major forward lmax={lmax} C={c}")
-    monkeypatch.delenv("ETP_FORWARD")
-    edge = _np(conv.forward(g, xd, Wd))
-    assert_blocks_close(o, edge.astype(np.float64), c, lmax, f"channel-major vs edge-major lmax={lmax} C={c}")
-
+# ------------------------------------------------------------------ path-subset forward
 
 @pytest.mark.parametrize("lmax,c", [(1, 8), (1, 32), (1, 64), (2, 8), (2, 20), (2, 36), (2, 64)])
 def test_forward_path_subset_kernel_ragged(lmax, c, monkeypatch):
