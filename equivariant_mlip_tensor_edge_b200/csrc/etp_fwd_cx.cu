@@ -75,7 +75,6 @@ constexpr int kNR = 2;                   // receiver ring (partial messages)
 constexpr int kN = 16;                   // edges per setup / consumer batch
 constexpr int kNM = 2 * kN;              // edges per MMA batch (MMA N): two consecutive batches
 constexpr int kEPW = kN / kH;            // edges per consumer warp and batch
-constexpr int kRW = 4;                   // edges per TMEM load round (the slow path selects among 4)
 constexpr int kMaxC = 64;                // channels: two 32-lane slices
 constexpr int kMinEdgesPerCta = 64;
 
@@ -178,14 +177,11 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
                : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld4(uint32_t taddr, float (&v)[4]) {
-  uint32_t r[4];
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(taddr)
-               : "memory");
-#pragma unroll
-  for (int i = 0; i < 4; ++i) v[i] = __uint_as_float(r[i]);
+__device__ __forceinline__ void tmem_ld2(uint32_t taddr, float (&v)[2]) {
+  uint32_t r[2];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr) : "memory");
+  v[0] = __uint_as_float(r[0]);
+  v[1] = __uint_as_float(r[1]);
 }
 
 // Bounded wait for the roles whose latency is hidden (setup, loader, combine): only lane 0 polls,
@@ -306,71 +302,57 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
     const float* xs = xbase + static_cast<size_t>(xl * kN + h * kEPW) * dim;
     const uint32_t tb = tmem + (static_cast<uint32_t>(32 * q) << 16) + ts * G::SLOTC + (k & 1) * kN + h * kEPW;
     const bool last_of_mma = (k & 1) || k == nb - 1;   // the MMA batch's columns are all read after this
+    // the batch half pair by pair: w of the pair's two columns per path item, then one packed
+    // contraction when both edges are valid and belong to the current receiver; otherwise the
+    // pair is taken edge by edge with the other edge masked (w = x = 0), flushing in between
 #pragma unroll 1
-    for (int rr = 0; rr < kEPW / kRW && ok; ++rr) {
-      float wv[NP][kRW];
+    for (int pr = 0; pr < kEPW / 2 && ok; ++pr) {
+      const int i = 2 * pr;
+      float wv[NP][2];
 #pragma unroll
-      for (int b = 0; b < NP; ++b) tmem_ld4(tb + b * kNM + rr * kRW, wv[b]);
+      for (int b = 0; b < NP; ++b) tmem_ld2(tb + b * kNM + i, wv[b]);
       tc::tmem_wait_ld();
-      if (rr == kEPW / kRW - 1 && last_of_mma) {   // every column of the slot this warp needs is read
+      if (pr == kEPW / 2 - 1 && last_of_mma) {   // every column of the slot this warp needs is read
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars->tempty[ts]);
       }
-      const int r0 = rr * kRW;
-      const int nv = nval - r0 < kRW ? nval - r0 : kRW;   // valid edges of the round (may be <= 0)
-      if (nv == kRW && base + r0 + kRW - 1 < nxt) {
-        // common case: four valid edges of the current receiver, two pairs in straight-line code
+      const int nv = nval - i;   // valid edges from this pair on (may be <= 0)
+      if (nv <= 0) continue;
+      const bool vb = nv >= 2;
+      const float* xa = xs + static_cast<size_t>(i) * dim;
+      const float* xb = xa + dim;
+      const float4* cf = reinterpret_cast<const float4*>(cfs + pr * PW);
+      if (vb && base + i + 1 < nxt) {
+        float2 xv[NX];
 #pragma unroll
-        for (int pr = 0; pr < kRW / 2; ++pr) {
-          const int i = r0 + 2 * pr;
-          const float* xa = xs + static_cast<size_t>(i) * dim;
-          const float* xb = xa + dim;
-          float2 xv[NX];
+        for (int c = 0; c < NX; ++c) xv[c] = chv ? make_float2(xa[xoff[c]], xb[xoff[c]]) : make_float2(0.0f, 0.0f);
+        float2 w[NP];
 #pragma unroll
-          for (int c = 0; c < NX; ++c) xv[c] = chv ? make_float2(xa[xoff[c]], xb[xoff[c]]) : make_float2(0.0f, 0.0f);
-          float2 w[NP];
-#pragma unroll
-          for (int pi = 0; pi < NP; ++pi) w[pi] = make_float2(wv[pi][2 * pr], wv[pi][2 * pr + 1]);
-          SUB::fwd2(reinterpret_cast<const float4*>(cfs + (i >> 1) * PW), xv, w, acc);
+        for (int pi = 0; pi < NP; ++pi) w[pi] = make_float2(wv[pi][0], wv[pi][1]);
+        SUB::fwd2(cf, xv, w, acc);
+        continue;
+      }
+      const int want = vb ? 3 : 1;
+      int done = 0;   // bit t: edge t of the pair accumulated
+      while (done != want) {
+        const int first = done & 1;   // the next edge still to take
+        while (base + i + first >= nxt) {
+          ok = flush();
+          if (!ok) break;
         }
-      } else {
-        // a receiver boundary or the end of the range inside the round: pair by pair; an edge of
-        // the pair that is invalid or belongs to a later receiver is masked (w = x = 0) and taken
-        // in a second step after the flush
-#pragma unroll 1
-        for (int pr = 0; pr < kRW / 2 && ok; ++pr) {
-          const int i = r0 + 2 * pr;
-          if (2 * pr >= nv) break;
-          const bool vb = 2 * pr + 1 < nv;
-          const int want = vb ? 3 : 1;
-          int done = 0;   // bit t: edge t of the pair accumulated
-          while (done != want) {
-            const int first = done & 1;   // the next edge still to take
-            while (base + i + first >= nxt) {
-              ok = flush();
-              if (!ok) break;
-            }
-            if (!ok) break;
-            const bool m0 = first == 0;
-            const bool m1 = vb && base + i + 1 < nxt;
-            const float* xa = xs + static_cast<size_t>(i) * dim;
-            const float* xb = xa + dim;
-            float2 xv[NX];
+        if (!ok) break;
+        const bool m0 = first == 0;
+        const bool m1 = vb && base + i + 1 < nxt;
+        float2 xv[NX];
 #pragma unroll
-            for (int c = 0; c < NX; ++c)
-              xv[c] = make_float2(chv && m0 ? xa[xoff[c]] : 0.0f, chv && m1 ? xb[xoff[c]] : 0.0f);
-            float2 w[NP];
+        for (int c = 0; c < NX; ++c)
+          xv[c] = make_float2(chv && m0 ? xa[xoff[c]] : 0.0f, chv && m1 ? xb[xoff[c]] : 0.0f);
+        float2 w[NP];
 #pragma unroll
-            for (int pi = 0; pi < NP; ++pi) {
-              const float wa = pr == 0 ? wv[pi][0] : wv[pi][2];
-              const float wb = pr == 0 ? wv[pi][1] : wv[pi][3];
-              w[pi] = make_float2(m0 ? wa : 0.0f, m1 ? wb : 0.0f);
-            }
-            SUB::fwd2(reinterpret_cast<const float4*>(cfs + (i >> 1) * PW), xv, w, acc);
-            done |= (m0 ? 1 : 0) | (m1 ? 2 : 0);
-          }
-        }
+        for (int pi = 0; pi < NP; ++pi) w[pi] = make_float2(m0 ? wv[pi][0] : 0.0f, m1 ? wv[pi][1] : 0.0f);
+        SUB::fwd2(cf, xv, w, acc);
+        done |= (m0 ? 1 : 0) | (m1 ? 2 : 0);
       }
     }
     if (!ok) break;

@@ -651,6 +651,7 @@ def emit_cx(out, lmax):
         out.append("  }")
         out.append(f"  static constexpr int FMA = {fma};   // FP32 instructions per edge and channel")
         emit_cx_pair(out, sub, paths, ent, emap, nc, xi, oi)
+        emit_cx_gw_pair(out, sub, paths, ent, emap, nc, xi, oi)
         out.append("};")
 
 
@@ -715,6 +716,94 @@ def emit_cx_pair(out, sub, paths, ent, emap, nc, xi, oi):
         out.append(f"    float2 xm[{nx}];")
         for xx in sorted(neg):
             out.append(f"    xm[{xx}] = __fmul2_rn(x[{xx}], make_float2(-1.0f, -1.0f));")
+    out.extend(body)
+    out.append("  }")
+
+
+def emit_cx_gw_pair(out, sub, paths, ent, emap, nc, xi, oi):
+    """Weight-gradient factor of the subset's paths for two edges at once (f32x2: .x the first edge,
+    .y the second): gw_p = sum_{m1,m3} x[l1 m1] M_p[m3][m1] g[l3 m3], with M_p[m3][m1] = sum_m2 C Y
+    from the pair-interleaved coefficient row. Each path contracts M with the longer side first
+    (v = M^T g then x . v, or s = M x then g . s). A coefficient used with a minus sign multiplies
+    the negated x or g (exact). sink(IC<p>{}, gw) receives path p (global path index)."""
+    nx, no = len(xi), len(oi)
+    body, negx, negg = [], set(), set()
+    for pi, p in enumerate(sub):
+        l1, l2, l3 = paths[p]
+        e = ent[p]
+        body.append(f"    {{ // path {p}: ({l1},{l2},{l3})")
+        if l2 == 0:
+            for j, (m3, m1, terms) in enumerate(e):
+                o, xx = oi[idx(l3, m3 - l3)], xi[idx(l1, m1 - l1)]
+                if j == 0:
+                    body.append(f"      float2 t = __fmul2_rn(x[{xx}], g[{o}]);")
+                else:
+                    body.append(f"      t = __ffma2_rn(x[{xx}], g[{o}], t);")
+            body.append(f"      sink(IC<{p}>{{}}, t);")
+        elif (2 * l1 + 1) <= (2 * l3 + 1):
+            # v[m1] = sum_m3 M[m3][m1] g[m3], then gw = sum_m1 x[m1] v[m1]
+            first = True
+            for m1 in range(2 * l1 + 1):
+                col = [(m3, b) for (m3, b, _) in e if b == m1]
+                if not col:
+                    continue
+                for j, (m3, _) in enumerate(col):
+                    ci, sg = emap[(p, m3, m1)]
+                    o = oi[idx(l3, m3 - l3)]
+                    if sg < 0:
+                        negg.add(o)
+                    gv = f"g[{o}]" if sg > 0 else f"gm[{o}]"
+                    if j == 0:
+                        body.append(f"      float2 v{m1} = __fmul2_rn(cv[{ci}], {gv});")
+                    else:
+                        body.append(f"      v{m1} = __ffma2_rn(cv[{ci}], {gv}, v{m1});")
+                xx = xi[idx(l1, m1 - l1)]
+                if first:
+                    body.append(f"      float2 t = __fmul2_rn(x[{xx}], v{m1});")
+                    first = False
+                else:
+                    body.append(f"      t = __ffma2_rn(x[{xx}], v{m1}, t);")
+            body.append(f"      sink(IC<{p}>{{}}, t);")
+        else:
+            # s[m3] = sum_m1 M[m3][m1] x[m1], then gw = sum_m3 g[m3] s[m3]
+            first = True
+            for m3 in range(2 * l3 + 1):
+                row = [(a, m1) for (a, m1, _) in e if a == m3]
+                if not row:
+                    continue
+                for j, (a, m1) in enumerate(row):
+                    ci, sg = emap[(p, a, m1)]
+                    xx = xi[idx(l1, m1 - l1)]
+                    if sg < 0:
+                        negx.add(xx)
+                    xv = f"x[{xx}]" if sg > 0 else f"xm[{xx}]"
+                    if j == 0:
+                        body.append(f"      float2 s{m3} = __fmul2_rn(cv[{ci}], {xv});")
+                    else:
+                        body.append(f"      s{m3} = __ffma2_rn(cv[{ci}], {xv}, s{m3});")
+                o = oi[idx(l3, m3 - l3)]
+                if first:
+                    body.append(f"      float2 t = __fmul2_rn(g[{o}], s{m3});")
+                    first = False
+                else:
+                    body.append(f"      t = __ffma2_rn(g[{o}], s{m3}, t);")
+            body.append(f"      sink(IC<{p}>{{}}, t);")
+        body.append("    }")
+    out.append("  template <class SINK>")
+    out.append(f"  __device__ __forceinline__ static void gw2(const float4* __restrict__ cf, const float2 (&x)[{nx}],")
+    out.append(f"      const float2 (&g)[{no}], SINK&& sink) {{")
+    for q in range(nc // 2):
+        out.append(f"    const float4 c4_{q} = cf[{q}];")
+    out.append(f"    const float2 cv[{nc}] = {{" + ", ".join(
+        f"make_float2(c4_{k // 2}.{'x' if k % 2 == 0 else 'z'}, c4_{k // 2}.{'y' if k % 2 == 0 else 'w'})" for k in range(nc)) + "};")
+    if negx:
+        out.append(f"    float2 xm[{nx}];")
+        for xx in sorted(negx):
+            out.append(f"    xm[{xx}] = __fmul2_rn(x[{xx}], make_float2(-1.0f, -1.0f));")
+    if negg:
+        out.append(f"    float2 gm[{no}];")
+        for o in sorted(negg):
+            out.append(f"    gm[{o}] = __fmul2_rn(g[{o}], make_float2(-1.0f, -1.0f));")
     out.extend(body)
     out.append("  }")
 

@@ -662,7 +662,10 @@ def test_path_mask_forward_backward_parity(wls, name, monkeypatch):
     assert_close_rel(_np(gv), rgv, f"{name} masked grad_edge_vec")
 
 
-def test_path_mask_all_ones_and_zero(wls):
+def test_path_mask_all_ones_and_zero(wls, monkeypatch):
+    """All bits set is the unmasked call of the same (edge-major) kernels, bit for bit; no bits set
+    gives zeros. Masked calls run the edge-major kernels, so the unmasked forward is pinned to it."""
+    monkeypatch.setenv("ETP_FORWARD", "edge")
     wl = wls("diamond1k")
     conv = _conv(wl)
     x, W = _inputs(wl, conv)
