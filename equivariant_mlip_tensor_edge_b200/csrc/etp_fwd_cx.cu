@@ -312,6 +312,8 @@ __device__ __forceinline__ bool consume(const Args& a, unsigned char* smem, Bars
 #pragma unroll
       for (int b = 0; b < NP; ++b) tmem_ld2(tb + b * kNM + i, wv[b]);
       tc::tmem_wait_ld();
+#pragma unroll
+      for (int b = 0; b < NP; ++b) asm volatile("" : "+f"(wv[b][0]), "+f"(wv[b][1]));   // no read above the wait
       if (pr == kEPW / 2 - 1 && last_of_mma) {   // every column of the slot this warp needs is read
         tc_fence_before();
         __syncwarp();
