@@ -184,8 +184,10 @@ __global__ void k_bprep(const float* __restrict__ W, int C, int n_units, float* 
   }
 }
 
-// receiver of every canonical edge
+// receiver of every canonical edge. A kernel launched as its programmatic dependent may start at once
+// and waits for this grid (griddepcontrol.wait) before reading recv.
 __global__ void k_recv_of_edge(const int* __restrict__ row_ptr, int n_nodes, int n_edges, int* __restrict__ recv) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < n_edges; e += gridDim.x * blockDim.x) {
     int lo = 0, hi = n_nodes - 1;   // last r with row_ptr[r] <= e
     while (lo < hi) {
@@ -272,6 +274,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_tc(BArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   bool drained = true;   // false: issued tensor-core work did not finish; TMEM is then not released
+  // launched as a programmatic dependent of k_recv_of_edge: the setup above overlaps it, the work
+  // below reads its output (the pre-split weights come from k_bprep, complete before it began)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == kQuads) {
     // ---------------------------------------------------------------- producer
@@ -684,9 +689,17 @@ etp_status blaunch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, c
   const long long min_grid = (n_rg + G::MAXRG - 3) / (G::MAXRG - 2);
   if (grid < min_grid) grid = min_grid;
   if (grid > a.n_groups) grid = a.n_groups;
-  if (mask) k_bwd_tc<L, true><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
-  else k_bwd_tc<L, false><<<static_cast<int>(grid), kThreads, G::SMEM, s>>>(a);
-  e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = G::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = mask ? cudaLaunchKernelEx(&cfg, k_bwd_tc<L, true>, a) : cudaLaunchKernelEx(&cfg, k_bwd_tc<L, false>, a);
   if (e != cudaSuccess) return cuda_status(e, "tc backward launch");
   if (grad_vec && n_units > 1 && n_edges > 0) {
     long long blocks = (3LL * n_edges + 255) / 256;

@@ -201,6 +201,8 @@ __global__ void __launch_bounds__(32 * kPairWarps) k_dw_pair(int n_edges, int C,
     for (int p = 0; p < P; ++p) acc[b][p] = make_float2(0.0f, 0.0f);
   float2 gp[D];   // cotangent rows of the current pair's receivers (.x first edge, .y second)
   int gi0 = -1, gi1 = -1;
+  // launched as a programmatic dependent of k_recv_of_edge, whose output (recv) is read below
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   auto node = [&](const float* a, int i, int c) { return cu ? __ldg(a + static_cast<size_t>(i) * dim + c * C + u) : 0.0f; };
 
   for (int e0 = e_beg; e0 < e_end; e0 += 32) {
@@ -369,10 +371,19 @@ etp_status dw_launch(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr,
   const int n_tasks = n_ranges * n_slices;
   if (L <= 2) {
     const int pblocks = (n_tasks + kPairWarps - 1) / kPairWarps;
-    k_dw_pair<L <= 2 ? L : 2><<<pblocks, 32 * kPairWarps, 0, s>>>(n_edges, c.channels, c.dim, 1.0f / c.r_cut, chunk,
-                                                                  n_slices, n_tasks, recv, sender, edge_vec, x, g,
-                                                                  part);
-    cudaError_t e = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pblocks);
+    cfg.blockDim = dim3(32 * kPairWarps);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, k_dw_pair<L <= 2 ? L : 2>, n_edges, c.channels, c.dim, 1.0f / c.r_cut,
+                                       chunk, n_slices, n_tasks, static_cast<const int*>(recv), sender, edge_vec, x,
+                                       g, part);
     if (e != cudaSuccess) return cuda_status(e, "weight gradient launch");
     k_dw_sum<<<(n_out + 31) / 32, 256, 0, s>>>(part, n_ranges, n_out, dW);
     return cuda_status(cudaGetLastError(), "weight gradient sum launch");

@@ -159,24 +159,6 @@ __device__ __forceinline__ int recv_of_warp(const int* __restrict__ row_ptr, int
   return first - 1;
 }
 
-// D (TMEM) = A (TMEM, M = 128 lanes x K = 8 columns of tf32) x B (shared memory descriptor)
-__device__ __forceinline__ void mma_tf32_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float (&v)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),
-               "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-               "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-               "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
-               : "memory");
-}
-
 __device__ __forceinline__ void tmem_ld2(uint32_t taddr, float (&v)[2]) {
   uint32_t r[2];
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr) : "memory");
@@ -564,6 +546,8 @@ __device__ __forceinline__ bool combine(const Args& a, unsigned char* smem, Bars
   const float* part = reinterpret_cast<const float*>(smem + G::OFF_PT);
   const int r_begin = bars->r_begin, r_end = bars->r_end;
   const long long E = a.n_edges;
+  // the counters are zeroed by the preceding prep kernel (this kernel may start before it ends)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (int kr = 0; kr <= r_end - r_begin; ++kr) {
     const int slot = kr % kNR;
     if (!warp_wait_lazy(&bars->rfull[slot], (kr / kNR) & 1, abort_flag, a.err, 37)) return false;
@@ -790,8 +774,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_fwd_cx(Args a) {
   }
 }
 
-// Per call: zero the spanning-receiver counters.
+// Per call: zero the spanning-receiver counters. The forward kernel is launched as its programmatic
+// dependent, so its prologue overlaps this kernel; only its combine warp, the one user of the
+// counters, waits for this grid's completion (griddepcontrol.wait) before touching them.
 __global__ void k_cx_prep(int* __restrict__ cnt, int n) {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   for (int i = threadIdx.x; i < n; i += blockDim.x) cnt[i] = 0;
 }
 
@@ -847,8 +834,17 @@ etp_status launch_t(const Ctx& c, int n_nodes, int n_edges, const int* row_ptr, 
   a.gpart = gpart_ptr(ws);
   a.cnt = cnt;
   a.err = c.status_dev;
-  k_fwd_cx<L, CT><<<grid, kThreads, G::SMEM, s>>>(a);
-  return cuda_status(cudaGetLastError(), "cx forward launch");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = G::SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, k_fwd_cx<L, CT>, a), "cx forward launch");
 }
 
 }  // namespace
