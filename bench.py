@@ -388,29 +388,38 @@ def run_gpu(args, rank, world, local_rank):
     out_h = torch.empty_like(bufs["out"], device="cpu").pin_memory()
     f_h = torch.empty((n, 3), dtype=torch.float32).pin_memory()
 
-    # the copies run on a second stream where the data flow allows: x, W and the cotangent travel
-    # while the neighbour list is built from the positions, and the forward output travels back
-    # while the backward runs
-    copy_stream = torch.cuda.Stream(device=dev)
+    # the copies overlap the compute where the data flow allows: x and W travel (upload stream)
+    # while the neighbour list is built from the positions, the cotangent while the forward runs,
+    # and the forward output comes back (download stream) while the backward runs
+    up_stream = torch.cuda.Stream(device=dev)
+    down_stream = torch.cuda.Stream(device=dev)
+    ev_xw = torch.cuda.Event()
+    ev_g = torch.cuda.Event()
     in_d = [torch.empty_like(t, device=dev) for t in (pos_h, x_h, W_h, g_h)]
 
     def e2e_step():
         main = torch.cuda.current_stream(dev)
-        copy_stream.wait_stream(main)                  # the previous step is done with the buffers
+        up_stream.wait_stream(main)                    # the previous step is done with the buffers
+        down_stream.wait_stream(main)
         in_d[0].copy_(pos_h, non_blocking=True)
-        with torch.cuda.stream(copy_stream):
-            for d_, h_ in zip(in_d[1:], (x_h, W_h, g_h)):
-                d_.copy_(h_, non_blocking=True)
+        with torch.cuda.stream(up_stream):
+            in_d[1].copy_(x_h, non_blocking=True)
+            in_d[2].copy_(W_h, non_blocking=True)
+            ev_xw.record(up_stream)
+            in_d[3].copy_(g_h, non_blocking=True)
+            ev_g.record(up_stream)
         gr_ = graph_step(in_d[0])
-        main.wait_stream(copy_stream)
+        main.wait_event(ev_xw)
         conv_fwd(gr_, in_d[1], in_d[2])
-        copy_stream.wait_stream(main)
-        with torch.cuda.stream(copy_stream):
+        down_stream.wait_stream(main)
+        with torch.cuda.stream(down_stream):
             out_h.copy_(bufs["out"], non_blocking=True)
+        main.wait_event(ev_g)
         conv_bwd(gr_, in_d[1], in_d[2], in_d[3])
         etp.forces(gr_, bufs["gv"][:gr_.n_edges], out=bufs["f"])
         f_h.copy_(bufs["f"], non_blocking=True)
-        main.wait_stream(copy_stream)
+        main.wait_stream(down_stream)
+        main.wait_stream(up_stream)
 
     for _ in range(2):
         e2e_step()
