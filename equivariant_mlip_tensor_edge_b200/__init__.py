@@ -49,6 +49,9 @@ SIGNATURES = {
                                  _vp]),
     "etp_radial_weights": (_i, [_vp, _i, _vp, _vp, _vp, _vp]),
     "etp_node_ladder": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp]),
+    "etp_node_ladder_full_step_floats": (_sz, [_i, _i]),
+    "etp_node_ladder_full_workspace_bytes": (_sz, [_i, _i, _i]),
+    "etp_node_ladder_full": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "etp_forces": (_i, [_i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "etp_graph_workspace_bytes": (_sz, [_i, _i]),
     "etp_neighbors": (_i, [_vp, _i, _dp, _ip, _f, _i, _ip, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
@@ -355,6 +358,36 @@ def node_ladder(A, Ws, lmax, out=None):
         out = torch.empty_like(A)
     _check(load_library().etp_node_ladder(int(lmax), c, n, nu, _ptr(A), _ptr(Ws) if nu > 1 else None, _ptr(out),
                                           _stream(A.device)), "etp_node_ladder")
+    return out
+
+
+def node_ladder_full_step_floats(lmax, channels):
+    """Floats of one step of full-ladder weights (the per-rank matrices [C][P_l3 C], l3 = 0..lmax)."""
+    return int(load_library().etp_node_ladder_full_step_floats(int(lmax), int(channels)))
+
+
+def node_ladder_full(A, Ws, lmax, out=None, workspace=None):
+    """The full product ladder: out = B_1 + ... + B_nu, B_1 = A, and each step the per-path products
+    of B_q and A compressed by that step's per-rank matrices (paths and channels mixed; the mixing
+    runs on the tensor cores).
+
+    A: [N, C (lmax+1)^2] float32 CUDA tensor (node-row layout, C in 32, 64, 96, 128);
+    Ws: [nu - 1, node_ladder_full_step_floats(lmax, C)] (nu - 1 may be 0). Returns out like A.
+    """
+    torch = _torch()
+    _need_cuda(A, Ws)
+    A, Ws = _f32(A), _f32(Ws)
+    n, dim = A.shape
+    c = dim // ((lmax + 1) ** 2)
+    nu = Ws.shape[0] + 1
+    lib = load_library()
+    if out is None:
+        out = torch.empty_like(A)
+    need = int(lib.etp_node_ladder_full_workspace_bytes(int(lmax), c, n))
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=A.device)
+    _check(lib.etp_node_ladder_full(int(lmax), c, n, nu, _ptr(A), _ptr(Ws) if nu > 1 else None, _ptr(out),
+                                    _ptr(workspace), workspace.numel(), _stream(A.device)), "etp_node_ladder_full")
     return out
 
 

@@ -768,6 +768,58 @@ etp_status etp_node_ladder(int lmax, int channels, int n_nodes, int nu, const fl
   return launch_node_ladder(lmax, channels, n_nodes, nu, A, W, out, static_cast<cudaStream_t>(stream));
 }
 
+size_t etp_node_ladder_full_step_floats(int lmax, int channels) {
+  return lad::supported(lmax, channels) ? lad::step_weight_floats(lmax, channels) : 0;
+}
+
+size_t etp_node_ladder_full_workspace_bytes(int lmax, int channels, int n_nodes) {
+  return lad::workspace_bytes(lmax, channels, n_nodes);
+}
+
+etp_status etp_node_ladder_full(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,
+                                float* out, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!lad::supported(lmax, channels)) {
+    set_error("etp_node_ladder_full: lmax must be 1, 2 or 3 and channels 32, 64, 96 or 128");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  if (n_nodes < 0 || nu < 1 || nu > 8) {
+    set_error("etp_node_ladder_full: n_nodes >= 0 and 1 <= nu <= 8");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (static_cast<long long>(n_nodes) * 99 * channels >= (1LL << 40)) {
+    set_error("etp_node_ladder_full: too many nodes");
+    return ETP_ERR_UNSUPPORTED;
+  }
+  if (n_nodes > 0 && (!A || !out || (nu > 1 && !W))) {
+    set_error("etp_node_ladder_full: NULL array");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if ((A && !aligned16(A)) || (out && !aligned16(out)) || (W && !aligned16(W))) {
+    set_error("etp_node_ladder_full: A, W and out must be 16-byte aligned");
+    return ETP_ERR_INVALID_ARG;
+  }
+  if (n_nodes == 0) return ETP_OK;
+  if (!workspace || workspace_bytes < lad::workspace_bytes(lmax, channels, n_nodes) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) {
+    set_error("etp_node_ladder_full: workspace missing, misaligned or smaller than "
+              "etp_node_ladder_full_workspace_bytes()");
+    return ETP_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int* status = nullptr;
+  etp_status st = lad::launch(lmax, channels, nu, n_nodes, A, W, out, workspace, s, &status);
+  if (st != ETP_OK || !validate_requested()) return st;
+  int code = 0;
+  cudaError_t e = cudaMemcpyAsync(&code, status, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_status(e, "etp_node_ladder_full status");
+  if (code != 0) {
+    set_error("etp_node_ladder_full: a tensor-core pipeline wait gave up (code " + std::to_string(code) + ")");
+    return ETP_ERR_CUDA;
+  }
+  return ETP_OK;
+}
+
 etp_status etp_radial_weights(etp_handle h, int n_edges, const float* edge_vec, const float* W,
                               float* w_out, void* stream) {
   if (!h || n_edges < 0 || (n_edges > 0 && (!edge_vec || !W || !w_out))) {

@@ -117,6 +117,15 @@ etp_status launch_backward_tc(const Ctx& c, int n_nodes, int n_edges, const int*
                               cudaStream_t s, const uint32_t* path_mask = nullptr);
 }  // namespace tc
 
+// ---- the full product ladder (etp_ladder_full.cu)
+namespace lad {
+bool supported(int lmax, int channels);
+size_t workspace_bytes(int lmax, int channels, int n_nodes);
+size_t step_weight_floats(int lmax, int channels);
+etp_status launch(int lmax, int channels, int order, int n_nodes, const float* A, const float* W, float* out,
+                  void* ws, cudaStream_t s, int** status_dev);
+}  // namespace lad
+
 // ---- channel-major forward with path subsets (etp_fwd_cx.cu): l_max <= 2, 4 <= C <= 64, C % 4 == 0
 namespace cx {
 bool supported(const Ctx& c);

@@ -1,0 +1,409 @@
+// The full node-local product ladder ("FlashCart", Fig. 3b dashed curves; Fig. E1 (b)): every step
+// keeps the unweighted "uvu" product of each retained coupling path and compresses the paths of each
+// output rank with one matrix that mixes paths and channels,
+//
+//   T_p[m3, u]      = sum_{m1, m2} C^{l1 l2 l3}_{m1 m2 m3} B[l1 m1 u] A[l2 m2 u]
+//   B'[l3, m3, v]   = sum_{p of rank l3} sum_u W_l3[v, p' C + u] T_p[m3, u]
+//   B_1 = A, B_{q+1} = step(B_q, A; W_q), out = sum_{q = 1..nu} B_q.
+//
+// The compression is a dense GEMM per output component (l3, m3): rows = nodes, K = P_l3 C (the
+// paths of rank l3 times the channels), N = C. It runs on the tensor cores:
+//   k_ladder_t:   CUDA cores, one warp per (node, 32-channel slice): the NT per-path products of the
+//                 node for the lane's channel, written as the rows of the GEMM operands T_l3.
+//   k_ladder_mix: one CTA per (128-node tile, component). Four loader warps stream K-chunks of 32
+//                 columns of T (the node rows) and of W_l3 (the output-channel rows) into shared
+//                 memory as tf32 hi/lo tiles in the canonical K-major layout; one thread issues
+//                 three kind::tf32 MMAs per 8 columns (hi*hi + hi*lo + lo*hi) into a TMEM
+//                 accumulator [128 nodes x C]; the loader warps then read it back (tcgen05.ld) and
+//                 store the component of B_{q+1} and add it into out.
+// Every output element is written by one thread per step: the result is bitwise reproducible.
+// Every mbarrier wait is bounded; a timeout records a code in the status word and the CTA drains
+// the MMAs it issued before it releases TMEM.
+#include <cstdint>
+#include <string>
+
+#include "etp_device.h"
+#include "etp_internal.h"
+#include "etp_tc_common.h"
+
+namespace etp {
+namespace lad {
+namespace {
+
+using tc::canon;
+using tc::fence_proxy_async;
+using tc::idesc_tf32;
+using tc::mbar_arrive;
+using tc::mbar_init;
+using tc::mbar_wait;
+using tc::mbar_wait_drain;
+using tc::mma_commit;
+using tc::mma_tf32;
+using tc::smem_desc;
+using tc::split_tf32;
+using tc::sptr;
+using tc::tc_fence_after;
+using tc::tc_fence_before;
+
+constexpr int kRows = 128;                 // nodes per tile (MMA M)
+constexpr int kChunk = 32;                 // K columns per pipeline stage (4 MMA K-steps of 8)
+constexpr int kLoadWarps = 4;              // loaders, later the epilogue (TMEM lane quadrant = warp)
+constexpr int kMmaWarp = kLoadWarps;
+constexpr int kThreads = 32 * (kLoadWarps + 1);
+constexpr int kStages = 3;
+constexpr int kMaxC = 128;
+
+template <int L>
+struct LadderGen;
+template <>
+struct LadderGen<1> {
+  using S = etp_gen::LadderShape<1>;
+  static __device__ __forceinline__ void t(const float (&b)[4], const float (&a)[4], float (&t)[S::NT]) {
+    etp_gen::ladder_t_1(b, a, t);
+  }
+};
+template <>
+struct LadderGen<2> {
+  using S = etp_gen::LadderShape<2>;
+  static __device__ __forceinline__ void t(const float (&b)[9], const float (&a)[9], float (&t)[S::NT]) {
+    etp_gen::ladder_t_2(b, a, t);
+  }
+};
+template <>
+struct LadderGen<3> {
+  using S = etp_gen::LadderShape<3>;
+  static __device__ __forceinline__ void t(const float (&b)[16], const float (&a)[16], float (&t)[S::NT]) {
+    etp_gen::ladder_t_3(b, a, t);
+  }
+};
+
+// Shared memory of k_ladder_mix for C channels: barriers, then kStages stages of
+// [A hi | A lo | B hi | B lo], each part 4 sub-tiles [rows x 8] in the canonical layout.
+struct Smem {
+  static constexpr int kBar = 1024;
+  static __host__ __device__ constexpr int a_part() { return 4 * kRows * 8 * 4; }
+  static __host__ __device__ constexpr int b_part(int C) { return 4 * C * 8 * 4; }
+  static __host__ __device__ constexpr int stage(int C) { return 2 * a_part() + 2 * b_part(C); }
+  static __host__ __device__ constexpr int bytes(int C) { return kBar + kStages * stage(C); }
+};
+
+// ---------------------------------------------------------------- per-path products
+
+// Task t: node t / n_slices, channel slice t % n_slices (32 channels). T_l3 is laid out
+// [node][m3][p' C + u] after the blocks of the lower ranks (block l3 starts at N C off(l3)).
+template <int L>
+__global__ void __launch_bounds__(256) k_ladder_t(int n_nodes, int C, const float* __restrict__ B,
+                                                  const float* __restrict__ A, float* __restrict__ T) {
+  using S = typename LadderGen<L>::S;
+  constexpr int D = (L + 1) * (L + 1);
+  const int lane = threadIdx.x & 31;
+  const int n_slices = C / 32;
+  const long long n_tasks = static_cast<long long>(n_nodes) * n_slices;
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long task = blockIdx.x * static_cast<long long>(blockDim.x >> 5) + (threadIdx.x >> 5); task < n_tasks;
+       task += stride) {
+    const int node = static_cast<int>(task / n_slices);
+    const int u = static_cast<int>(task % n_slices) * 32 + lane;
+    const size_t row = static_cast<size_t>(node) * D * C;
+    float b[D], a[D];
+#pragma unroll
+    for (int c = 0; c < D; ++c) {
+      b[c] = __ldg(B + row + static_cast<size_t>(c) * C + u);
+      a[c] = __ldg(A + row + static_cast<size_t>(c) * C + u);
+    }
+    float t[S::NT];
+    LadderGen<L>::t(b, a, t);
+#pragma unroll
+    for (int l3 = 0; l3 <= L; ++l3) {
+      const int P = S::P(l3);
+      float* dst = T + static_cast<size_t>(n_nodes) * C * S::off(l3) +
+                   static_cast<size_t>(node) * (2 * l3 + 1) * P * C + u;
+#pragma unroll
+      for (int i = 0; i < (2 * l3 + 1) * P; ++i) dst[static_cast<size_t>(i) * C] = t[S::off(l3) + i];
+    }
+  }
+}
+
+// ---------------------------------------------------------------- the compression GEMM
+
+struct MixArgs {
+  int n_nodes;
+  int C;
+  const float* T;      // the step's products (k_ladder_t layout)
+  const float* W;      // the step's matrices: rank blocks one after another, each [C][P_l3 C]
+  float* b_next;       // B_{q+1} [N][D C], or null on the last step
+  float* out;          // out [N][D C], += B_{q+1}
+  int* err;
+};
+
+struct Bars {
+  uint64_t full[kStages];    // a stage's tiles written (kLoadWarps arrivals)
+  uint64_t empty[kStages];   // a stage's MMAs complete (one commit)
+  uint64_t done;             // every MMA of the tile complete
+  uint64_t drain;
+  uint32_t tmem_holder;
+  int abort_flag;
+};
+
+// One row of a tile: columns [k0, k0 + 32) of row `row` (tile-local) of a row-major matrix whose
+// tile starts at src (leading dimension ld floats), split into tf32 hi/lo and stored in 4
+// sub-tiles [rows x 8] (one per MMA K-step) of the canonical K-major layout. An invalid row (past
+// the last node) is stored as zeros.
+__device__ __forceinline__ void load_row_split(const float* __restrict__ src, size_t ld, int row, bool valid, int k0,
+                                               int rows, float* hi, float* lo) {
+  const float4* p = reinterpret_cast<const float4*>(src + static_cast<size_t>(row) * ld + k0);
+#pragma unroll
+  for (int c4 = 0; c4 < kChunk / 4; ++c4) {
+    const float4 v = valid ? __ldg(p + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    float4 h, l;
+    split_tf32(v.x, &h.x, &l.x);
+    split_tf32(v.y, &h.y, &l.y);
+    split_tf32(v.z, &h.z, &l.z);
+    split_tf32(v.w, &h.w, &l.w);
+    const int off = (c4 >> 1) * rows * 8 + canon(row, (c4 & 1) * 4);   // K-step c4 / 2, columns 4 (c4 & 1)..
+    *reinterpret_cast<float4*>(hi + off) = h;
+    *reinterpret_cast<float4*>(lo + off) = l;
+  }
+}
+
+// Grid: x = 128-node tiles, y = output component (l3, m3) in (l, m) order.
+template <int L>
+__global__ void __launch_bounds__(kThreads, 1) k_ladder_mix(MixArgs a) {
+  using S = typename LadderGen<L>::S;
+  constexpr int D = (L + 1) * (L + 1);
+  extern __shared__ __align__(1024) unsigned char smem[];
+  Bars* bars = reinterpret_cast<Bars*>(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int C = a.C;
+  const int comp = blockIdx.y;
+  int l3 = 0;
+  while ((l3 + 1) * (l3 + 1) <= comp) ++l3;
+  const int m3 = comp - l3 * l3;
+  const int P = S::P(l3);
+  const int K = P * C;                       // GEMM K: the paths of rank l3 times the channels
+  const int n_chunks = K / kChunk;
+  const int node0 = blockIdx.x * kRows;
+  // the tile's operand rows: T_l3 row (node, m3) has K columns; W_l3 row v has K columns
+  const float* Tt = a.T + static_cast<size_t>(a.n_nodes) * C * S::off(l3) +
+                    (static_cast<size_t>(node0) * (2 * l3 + 1) + m3) * K;
+  const size_t t_ld = static_cast<size_t>(2 * l3 + 1) * K;
+  size_t w_off = 0;
+  for (int l = 0; l < l3; ++l) w_off += static_cast<size_t>(S::P(l)) * C * C;
+  const float* Wl = a.W + w_off;
+  volatile int* abort_flag = &bars->abort_flag;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars->full[s], kLoadWarps);
+      mbar_init(&bars->empty[s], 1);
+    }
+    mbar_init(&bars->done, 1);
+    mbar_init(&bars->drain, 1);
+    bars->abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const uint32_t cols = C <= 32 ? 32u : (C <= 64 ? 64u : 128u);   // TMEM allocation: a power of two >= C
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sptr(&bars->tmem_holder)),
+                 "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_holder;
+  unsigned char* stages = smem + Smem::kBar;
+  bool drained = true;
+
+  if (warp < kLoadWarps) {
+    // ---------------------------------------------------------------- loaders, then the epilogue
+    const int t = threadIdx.x;   // 0..127: node row t of the tile, and output-channel row t of W
+    bool ok = true;
+    for (int c = 0; c < n_chunks && ok; ++c) {
+      const int st = c % kStages;
+      if (c >= kStages) ok = tc::warp_wait(&bars->empty[st], ((c / kStages) - 1) & 1, abort_flag, a.err, 61);
+      if (!ok) break;
+      float* base = reinterpret_cast<float*>(stages + static_cast<size_t>(st) * Smem::stage(C));
+      float* ahi = base;
+      float* alo = ahi + Smem::a_part() / 4;
+      float* bhi = alo + Smem::a_part() / 4;
+      float* blo = bhi + Smem::b_part(C) / 4;
+      load_row_split(Tt, t_ld, t, node0 + t < a.n_nodes, c * kChunk, kRows, ahi, alo);
+      if (t < C) load_row_split(Wl, static_cast<size_t>(K), t, true, c * kChunk, C, bhi, blo);
+      fence_proxy_async();   // generic-proxy stores, read next by the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->full[st]);
+    }
+    if (ok) ok = tc::warp_wait(&bars->done, 0, abort_flag, a.err, 62);
+    if (ok) {
+      tc_fence_after();
+      const int node = node0 + t;
+      const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+      for (int v0 = 0; v0 < C; v0 += 32) {
+        float d[32];
+        tc::tmem_ld32(trow + v0, d);
+        tc::tmem_wait_ld();
+        if (node < a.n_nodes) {
+          const size_t off = static_cast<size_t>(node) * D * C + static_cast<size_t>(comp) * C + v0;
+          float4* o = reinterpret_cast<float4*>(a.out + off);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            float4 s = o[i];
+            s.x += d[4 * i];
+            s.y += d[4 * i + 1];
+            s.z += d[4 * i + 2];
+            s.w += d[4 * i + 3];
+            o[i] = s;
+          }
+          if (a.b_next) {
+            float4* bn = reinterpret_cast<float4*>(a.b_next + off);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bn[i] = make_float4(d[4 * i], d[4 * i + 1], d[4 * i + 2], d[4 * i + 3]);
+          }
+        }
+      }
+    }
+  } else if (lane == 0) {
+    // ---------------------------------------------------------------- MMA thread
+    const uint32_t idesc = idesc_tf32(C);
+    bool ok = true;
+    for (int c = 0; c < n_chunks && ok; ++c) {
+      const int st = c % kStages;
+      ok = mbar_wait(&bars->full[st], (c / kStages) & 1, abort_flag, a.err, 63);
+      if (!ok) break;
+      tc_fence_after();
+      const float* base = reinterpret_cast<const float*>(stages + static_cast<size_t>(st) * Smem::stage(C));
+      const float* ahi = base;
+      const float* alo = ahi + Smem::a_part() / 4;
+      const float* bhi = alo + Smem::a_part() / 4;
+      const float* blo = bhi + Smem::b_part(C) / 4;
+#pragma unroll
+      for (int s = 0; s < kChunk / 8; ++s) {
+        const uint64_t dah = smem_desc(sptr(ahi + s * kRows * 8)), dal = smem_desc(sptr(alo + s * kRows * 8));
+        const uint64_t dbh = smem_desc(sptr(bhi + s * C * 8)), dbl = smem_desc(sptr(blo + s * C * 8));
+        mma_tf32(tmem, dah, dbh, idesc, (c > 0 || s > 0) ? 1u : 0u);
+        mma_tf32(tmem, dah, dbl, idesc, 1u);
+        mma_tf32(tmem, dal, dbh, idesc, 1u);
+      }
+      mma_commit(&bars->empty[st]);
+    }
+    if (ok) mma_commit(&bars->done);
+    // drain, ignoring the abort flag: one more commit tracks every MMA issued so far
+    mma_commit(&bars->drain);
+    if (!mbar_wait_drain(&bars->drain, 0)) {
+      tc::report_code(a.err, 64);
+      bars->abort_flag = 1;
+      drained = false;
+    }
+  }
+  if (warp == kMmaWarp) drained = __shfl_sync(0xffffffffu, drained ? 1 : 0, 0) != 0;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp && drained) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(cols) : "memory");
+  }
+}
+
+bool supported_shape(int lmax, int C) {
+  return lmax >= 1 && lmax <= 3 && C >= 32 && C <= kMaxC && C % 32 == 0;
+}
+
+template <int L>
+size_t t_floats(int n_nodes, int C) {
+  return static_cast<size_t>(n_nodes) * C * LadderGen<L>::S::NT;
+}
+
+size_t t_floats_rt(int lmax, int n_nodes, int C) {
+  switch (lmax) {
+    case 1: return t_floats<1>(n_nodes, C);
+    case 2: return t_floats<2>(n_nodes, C);
+    default: return t_floats<3>(n_nodes, C);
+  }
+}
+
+template <int L>
+size_t step_weights(int C) {
+  using S = typename LadderGen<L>::S;
+  size_t w = 0;
+  for (int l = 0; l <= L; ++l) w += static_cast<size_t>(S::P(l)) * C * C;
+  return w;
+}
+
+template <int L>
+etp_status run(int C, int order, int n_nodes, const float* A, const float* W, float* out, float* bufs, float* T,
+               int* status, cudaStream_t s) {
+  constexpr int D = (L + 1) * (L + 1);
+  const size_t row = static_cast<size_t>(D) * C;
+  cudaError_t e = cudaMemcpyAsync(out, A, sizeof(float) * row * n_nodes, cudaMemcpyDeviceToDevice, s);
+  if (e != cudaSuccess) return cuda_status(e, "full ladder: out = A");
+  if (order <= 1 || n_nodes == 0) return ETP_OK;
+  e = cudaFuncSetAttribute(k_ladder_mix<L>, cudaFuncAttributeMaxDynamicSharedMemorySize, Smem::bytes(C));
+  if (e != cudaSuccess) return cuda_status(e, "full ladder smem attribute");
+  const float* b_cur = A;
+  const size_t wstep = step_weights<L>(C);
+  const long long tasks = static_cast<long long>(n_nodes) * (C / 32);
+  long long tblocks = (tasks + 7) / 8;
+  if (tblocks > 148LL * 16) tblocks = 148LL * 16;
+  for (int q = 1; q < order; ++q) {
+    float* b_next = q + 1 < order ? bufs + static_cast<size_t>(q & 1) * row * n_nodes : nullptr;
+    k_ladder_t<L><<<static_cast<int>(tblocks), 256, 0, s>>>(n_nodes, C, b_cur, A, T);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "full ladder products");
+    MixArgs m;
+    m.n_nodes = n_nodes;
+    m.C = C;
+    m.T = T;
+    m.W = W + static_cast<size_t>(q - 1) * wstep;
+    m.b_next = b_next;
+    m.out = out;
+    m.err = status;
+    dim3 grid((n_nodes + kRows - 1) / kRows, D);
+    k_ladder_mix<L><<<grid, kThreads, Smem::bytes(C), s>>>(m);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "full ladder mixing");
+    b_cur = b_next;
+  }
+  return ETP_OK;
+}
+
+}  // namespace
+
+size_t workspace_bytes(int lmax, int channels, int n_nodes) {
+  if (!supported_shape(lmax, channels) || n_nodes < 0) return 0;
+  const size_t row = static_cast<size_t>((lmax + 1) * (lmax + 1)) * channels;
+  return align256(sizeof(int)) + 2 * align256(sizeof(float) * row * n_nodes) +
+         align256(sizeof(float) * t_floats_rt(lmax, n_nodes, channels));
+}
+
+size_t step_weight_floats(int lmax, int channels) {
+  switch (lmax) {
+    case 1: return step_weights<1>(channels);
+    case 2: return step_weights<2>(channels);
+    default: return step_weights<3>(channels);
+  }
+}
+
+bool supported(int lmax, int channels) { return supported_shape(lmax, channels); }
+
+etp_status launch(int lmax, int channels, int order, int n_nodes, const float* A, const float* W, float* out,
+                  void* ws, cudaStream_t s, int** status_dev) {
+  char* p = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(p);
+  p += align256(sizeof(int));
+  const size_t row = static_cast<size_t>((lmax + 1) * (lmax + 1)) * channels;
+  float* bufs = reinterpret_cast<float*>(p);
+  p += 2 * align256(sizeof(float) * row * n_nodes);
+  float* T = reinterpret_cast<float*>(p);
+  *status_dev = status;
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
+  if (e != cudaSuccess) return cuda_status(e, "full ladder status");
+  switch (lmax) {
+    case 1: return run<1>(channels, order, n_nodes, A, W, out, bufs, T, status, s);
+    case 2: return run<2>(channels, order, n_nodes, A, W, out, bufs, T, status, s);
+    default: return run<3>(channels, order, n_nodes, A, W, out, bufs, T, status, s);
+  }
+}
+
+}  // namespace lad
+}  // namespace etp

@@ -393,15 +393,50 @@ def emit_node(out, lmax):
     out.append("}")
 
 
-# ---------------------------------------------------------------- channel-major forward
-# Lanes hold channels; the paths are dealt to G warps that share a 32-channel slice (G = 128 / C
-# for C in {32, 64, 128}), so each warp evaluates a subset of the paths for every edge. The
-# per-edge coefficients M_p[m3][m1] = sum_m2 C Y[l2 m2] are computed once per edge and stored in
-# a row laid out subset by subset (each subset's block starts on a float4 boundary).
+# ---------------------------------------------------------------- full product ladder
+def emit_ladder_t(out, lmax):
+    """The unweighted per-path products of the full ladder for one channel (FlashCart Fig. E1 (b)):
+    t[kLadderOff[l3] + m3 * kLadderP[l3] + j] = sum_{m1,m2} C[m1,m2,m3] b[l1 m1] a[l2 m2], j = the
+    path's index among the paths of output rank l3 (path order). Each (l3, m3) row of j values is
+    the K dimension of that output component's mixing matrix."""
+    paths = paths_for(lmax)
+    D = (lmax + 1) ** 2
+    ent = path_m_entries(lmax)
+    by_rank = [[p for p, (_, _, c) in enumerate(paths) if c == l3] for l3 in range(lmax + 1)]
+    offs, nt = [], 0
+    for l3 in range(lmax + 1):
+        offs.append(nt)
+        nt += (2 * l3 + 1) * len(by_rank[l3])
+    out.append(f"template <> struct LadderShape<{lmax}> {{")
+    out.append(f"  static constexpr int NT = {nt};   // products per node and channel")
+    out.append(f"  __host__ __device__ static constexpr int P(int l3) {{ constexpr int t[{lmax + 1}] = {{{', '.join(str(len(r)) for r in by_rank)}}}; return t[l3]; }}")
+    out.append(f"  __host__ __device__ static constexpr int off(int l3) {{ constexpr int t[{lmax + 1}] = {{{', '.join(map(str, offs))}}}; return t[l3]; }}")
+    out.append("};")
+    out.append(f"__device__ __forceinline__ void ladder_t_{lmax}(const float (&b)[{D}], const float (&a)[{D}], float (&t)[{nt}]) {{")
+    for l3 in range(lmax + 1):
+        for j, p in enumerate(by_rank[l3]):
+            l1, l2, _ = paths[p]
+            out.append(f"  {{ // path {p}: ({l1},{l2},{l3})")
+            for m3 in range(2 * l3 + 1):
+                row = [(m1, terms) for (a3, m1, terms) in ent[p] if a3 == m3]
+                dst = f"t[{offs[l3] + m3 * len(by_rank[l3]) + j}]"
+                if not row:
+                    out.append(f"    {dst} = 0.0f;")
+                    continue
+                first = True
+                for m1, terms in row:
+                    mexpr = " + ".join(f"{repr_f32(np.float32(v))}*a[{i}]" for v, i in terms)
+                    if first:
+                        out.append(f"    float s{m3} = ({mexpr}) * b[{idx(l1, m1 - l1)}];")
+                        first = False
+                    else:
+                        out.append(f"    s{m3} = fmaf({mexpr}, b[{idx(l1, m1 - l1)}], s{m3});")
+                out.append(f"    {dst} = s{m3};")
+            out.append("  }")
+    out.append("}")
 
-CM_LMAX = (1, 2)
-CM_GROUPS = (1, 2, 4)
 
+# ---------------------------------------------------------------- per-path M entries
 
 def path_m_entries(lmax):
     """Per path: the (m3, m1, terms) nonzeros of M in the order the code generator uses."""
@@ -416,117 +451,6 @@ def path_m_entries(lmax):
                     ent.append((m3, m1, terms))
         out.append(ent)
     return out
-
-
-def cm_split(lmax, G):
-    """Deal the paths to G subsets of equal size (padded with -1), balancing the per-channel cost
-    (M nonzeros + the shorter of 2 l1 + 1 and 2 l3 + 1), largest first."""
-    paths = paths_for(lmax)
-    ent = path_m_entries(lmax)
-    cost = [len(ent[p]) + min(2 * paths[p][0] + 1, 2 * paths[p][2] + 1) for p in range(len(paths))]
-    nblk = -(-len(paths) // G)
-    subsets = [[] for _ in range(G)]
-    load = [0] * G
-    for p in sorted(range(len(paths)), key=lambda q: (-cost[q], q)):
-        open_ = [g for g in range(G) if len(subsets[g]) < nblk]
-        g = min(open_, key=lambda h: (load[h], h))
-        subsets[g].append(p)
-        load[g] += cost[p]
-    for g in range(G):
-        subsets[g].sort()
-        subsets[g] += [-1] * (nblk - len(subsets[g]))
-    return subsets, nblk, load
-
-
-def emit_cm(out, lmax):
-    paths = paths_for(lmax)
-    D = (lmax + 1) ** 2
-    ent = path_m_entries(lmax)
-    for G in CM_GROUPS:
-        subsets, nblk, load = cm_split(lmax, G)
-        # row layout: subset blocks, each a multiple of 4 floats; total width MW with MW / 4 odd
-        offs, widths, pos = [], [], 0
-        moff = {}
-        for g in range(G):
-            offs.append(pos)
-            n = 0
-            for p in subsets[g]:
-                if p >= 0:
-                    moff[p] = pos + n
-                    n += len(ent[p])
-            w4 = -(-n // 4) * 4
-            widths.append(w4 if w4 > 0 else 4)
-            pos += widths[-1]
-        mw = pos
-        if (mw // 4) % 2 == 0:
-            mw += 4
-        name = f"{lmax}_{G}"
-        out.append(f"// ---- channel-major forward, l_max = {lmax}, {G} path subset(s); per-channel cost {load}")
-        out.append(f"template <> struct CmLayout<{lmax}, {G}> {{")
-        out.append(f"  static constexpr int NBLK = {nblk};   // paths per subset (MMA blocks)")
-        out.append(f"  static constexpr int MW = {mw};       // coefficient row width (floats)")
-        rows = ", ".join("{" + ", ".join(str(p) for p in subsets[g]) + "}" for g in range(G))
-        out.append(f"  static constexpr int path[{G}][{nblk}] = {{{rows}}};")
-        out.append(f"  static constexpr int off[{G}] = {{{', '.join(str(o) for o in offs)}}};")
-        out.append(f"  static constexpr int width[{G}] = {{{', '.join(str(w) for w in widths)}}};")
-        out.append("  // the same tables for indices known only at run time (device code)")
-        out.append("  __host__ __device__ static constexpr int path_at(int g, int b) {")
-        out.append(f"    constexpr int t[{G}][{nblk}] = {{{rows}}};")
-        out.append("    return t[g][b];")
-        out.append("  }")
-        out.append("  __host__ __device__ static constexpr int off_at(int g) {")
-        out.append(f"    constexpr int t[{G}] = {{{', '.join(str(o) for o in offs)}}};")
-        out.append("    return t[g];")
-        out.append("  }")
-        out.append("  __host__ __device__ static constexpr int width_at(int g) {")
-        out.append(f"    constexpr int t[{G}] = {{{', '.join(str(w) for w in widths)}}};")
-        out.append("    return t[g];")
-        out.append("  }")
-        out.append("};")
-        # coefficient row (setup side)
-        out.append(f"__device__ __forceinline__ void cm_coef_{name}(const float* Y, float (&row)[{mw}]) {{")
-        out.append(f"  #pragma unroll")
-        out.append(f"  for (int i = 0; i < {mw}; ++i) row[i] = 0.0f;")
-        for p, e in enumerate(ent):
-            for n, (m3, m1, terms) in enumerate(e):
-                l2 = paths[p][1]
-                if l2 == 0:
-                    expr = repr_f32(np.float32(terms[0][0]))
-                else:
-                    expr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
-                out.append(f"  row[{moff[p] + n}] = {expr};")
-        out.append("}")
-        # consumer side, one function per subset: acc[l3 m3] += w_p (sum_m1 M x[l1 m1]), one channel
-        for g in range(G):
-            out.append("template <class WF>")
-            out.append(f"__device__ __forceinline__ void cm_fwd_{name}_{g}(const float* mv, WF&& wfetch,")
-            out.append(f"    const float (&x)[{D}], float (&acc)[{D}]) {{")
-            for slot, p in enumerate(subsets[g]):
-                if p < 0:
-                    continue
-                l1, l2, l3 = paths[p]
-                base = moff[p] - offs[g]
-                e = ent[p]
-                out.append(f"  {{ // path {p}: ({l1},{l2},{l3}), block {slot}")
-                out.append(f"    const float wp = wfetch(IC<{slot}>{{}});")
-                scale_x = (2 * l1 + 1) < (2 * l3 + 1)
-                if scale_x:
-                    for m1 in range(2 * l1 + 1):
-                        out.append(f"    const float xs{m1} = wp * x[{idx(l1, m1 - l1)}];")
-                    for n, (m3, m1, _) in enumerate(e):
-                        out.append(f"    acc[{idx(l3, m3 - l3)}] = fmaf(mv[{base + n}], xs{m1}, acc[{idx(l3, m3 - l3)}]);")
-                else:
-                    for m3 in range(2 * l3 + 1):
-                        row = [(n, m1) for n, (a, m1, _) in enumerate(e) if a == m3]
-                        if not row:
-                            continue
-                        n0, b0 = row[0]
-                        out.append(f"    float s{m3} = mv[{base + n0}] * x[{idx(l1, b0 - l1)}];")
-                        for n, b in row[1:]:
-                            out.append(f"    s{m3} = fmaf(mv[{base + n}], x[{idx(l1, b - l1)}], s{m3});")
-                        out.append(f"    acc[{idx(l3, m3 - l3)}] = fmaf(wp, s{m3}, acc[{idx(l3, m3 - l3)}]);")
-                out.append("  }")
-            out.append("}")
 
 
 # ---------------------------------------------------------------- channel-major forward, path subsets
@@ -993,17 +917,16 @@ def generate():
            "  }",
            "}",
            "template <int L> struct PathSet;",
-           "template <int L, int G> struct CmLayout;",
-           "template <int L, int S> struct CxSub;"]
+           "template <int L, int S> struct CxSub;",
+           "template <int L> struct LadderShape;"]
     for lmax in LMAX_SUPPORTED:
         emit_sh(out, lmax)
         emit_paths(out, lmax)
-    for lmax in CM_LMAX:
-        emit_cm(out, lmax)
     for lmax in CX_LMAX:
         emit_cx(out, lmax)
     for lmax in LMAX_SUPPORTED:
         emit_node(out, lmax)
+        emit_ladder_t(out, lmax)
     emit_sh(out, GEN_LMAX)
     emit_general(out)
     out.append("}  // namespace etp_gen")

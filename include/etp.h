@@ -210,6 +210,26 @@ etp_status etp_backward(etp_handle h, int n_nodes, int n_edges, const int* row_p
 etp_status etp_node_ladder(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,
                            float* out, void* stream);
 
+/* The full node-local product ladder of correlation order nu (FlashCart Fig. 3b dashed curves and
+ * Fig. E1 (b): the products of the retained coupling paths are compressed by W^(q) to the channel
+ * width per retained rank, mixing paths and channels):
+ *   T_p[m3, u] = sum_{m1,m2} C B_q[l1, m1, u] A[l2, m2, u]   for every path p = (l1, l2, l3),
+ *   B_{q+1}[l3, m3, v] = sum_{p of rank l3} sum_u W_q,l3[v][p' C + u] T_p[m3, u],
+ *   B_1 = A,  out = B_1 + ... + B_nu,
+ * p' = the index of p among the paths of rank l3 in path order (the order of etp_node_ladder).
+ * W: the nu - 1 steps one after another; a step holds the matrices W_q,l3 for l3 = 0..lmax one
+ * after another, each [C][P_l3 C] row-major (P_l3 = the number of paths of rank l3; a step has
+ * etp_node_ladder_full_step_floats(lmax, channels) floats). The mixing runs on the tensor cores
+ * (3xTF32, fp32 accumulation): one GEMM per output component, rows = nodes, K = P_l3 C, N = C.
+ * lmax 1..3; channels 32, 64, 96 or 128; 1 <= nu <= 8. A, W, out: device pointers, 16-byte
+ * aligned; workspace: etp_node_ladder_full_workspace_bytes(lmax, channels, n_nodes) bytes, 256-byte
+ * aligned. Asynchronous on stream; with ETP_VALIDATE=1 the call synchronises and returns
+ * ETP_ERR_CUDA if a bounded pipeline wait gave up. */
+size_t etp_node_ladder_full_step_floats(int lmax, int channels);
+size_t etp_node_ladder_full_workspace_bytes(int lmax, int channels, int n_nodes);
+etp_status etp_node_ladder_full(int lmax, int channels, int n_nodes, int nu, const float* A, const float* W,
+                                float* out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Per-edge path selection (adaptive computation: an edge may use only some of the paths).
  * path_mask[n_edges] (device, canonical edge order): bit p set = path p contributes for that edge;
  * a clear bit is the same as w_{e,p,u} = 0 for every u. Paths that no edge of a 32-edge tile needs

@@ -216,3 +216,17 @@ def test_status_word_gates_calls_until_get_status_clears_it(lib):
         conv.check_status()
     assert ei.value.status == 5 and "code 12" in str(ei.value)
     conv.check_status()
+
+
+def test_node_ladder_full_refuses_unsupported_shapes_before_device_work():
+    """Widths other than 32, 64, 96, 128, ranks outside 1..3, orders outside 1..8 and a missing
+    workspace are refused by the host checks, before any device pointer is touched."""
+    import equivariant_mlip_tensor_edge_b200 as etp
+    lib = etp.load_library()
+    fake = ctypes.c_void_p(256)
+    assert lib.etp_node_ladder_full(2, 16, 10, 2, fake, fake, fake, fake, 1 << 30, None) == 3   # ETP_ERR_UNSUPPORTED
+    assert lib.etp_node_ladder_full(4, 32, 10, 2, fake, fake, fake, fake, 1 << 30, None) == 3
+    assert lib.etp_node_ladder_full(2, 32, 10, 9, fake, fake, fake, fake, 1 << 30, None) == 1   # ETP_ERR_INVALID_ARG
+    assert lib.etp_node_ladder_full(2, 32, 10, 2, fake, fake, fake, None, 0, None) == 1
+    assert lib.etp_node_ladder_full_step_floats(2, 32) == 11 * 32 * 32
+    assert lib.etp_node_ladder_full_workspace_bytes(2, 16, 10) == 0

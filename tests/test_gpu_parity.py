@@ -884,3 +884,53 @@ def test_general_irreps_autograd_function(wls):
     gx, gv = conv.backward(g, xt.detach(), Wt.detach(), gd)
     assert torch.equal(xt.grad, gx) and torch.equal(vt.grad, gv)
     assert torch.equal(Wt.grad, conv.backward_weights(g, xt.detach(), gd).reshape(Wt.shape))
+
+
+# ------------------------------------------------------------------ full product ladder
+
+@pytest.mark.parametrize("lmax,c,n,nu", [(2, 128, 4096, 3), (1, 32, 37, 2), (2, 64, 300, 3), (3, 32, 130, 2),
+                                        (3, 96, 129, 3), (2, 128, 128, 1), (1, 128, 257, 4)])
+def test_node_ladder_full_parity(lmax, c, n, nu):
+    """The full ladder (per-rank path- and channel-mixing matrices on the tensor cores) against the
+    oracle: the pages' 4096-node x 128-channel case and ragged tiles (node counts not a multiple of
+    the 128-node tile), every rank and channel width; bitwise reproducible."""
+    from oracle.product import full_step_sizes, node_ladder_full
+    rng = np.random.default_rng(700 + 10 * lmax + nu + c)
+    dim = (lmax + 1) ** 2 * c
+    A = rng.standard_normal((n, dim)).astype(np.float32)
+    steps = sum(full_step_sizes(lmax, c))
+    assert etp.node_ladder_full_step_floats(lmax, c) == steps
+    Ws = (rng.standard_normal((nu - 1, steps)) / np.sqrt(4 * c)).astype(np.float32)
+    ref = node_ladder_full(lmax, c, A, list(Ws))
+    Ad, Wd = torch.from_numpy(A).to(DEV), torch.from_numpy(Ws).to(DEV)
+    out = etp.node_ladder_full(Ad, Wd, lmax)
+    assert_blocks_close(_np(out), ref, c, lmax, f"full ladder lmax={lmax} C={c} N={n} nu={nu}")
+    assert torch.equal(out, etp.node_ladder_full(Ad, Wd, lmax)), "full ladder is not bitwise deterministic"
+
+
+def test_node_ladder_full_with_diagonal_matrices_matches_the_path_reduced_kernel():
+    """Channel-diagonal matrices make the full ladder the path-reduced one: the two kernels agree."""
+    from oracle.product import paths_of_rank
+    lmax, c, n, nu = 2, 64, 500, 3
+    rng = np.random.default_rng(77)
+    A = rng.standard_normal((n, 9 * c)).astype(np.float32)
+    wr = (rng.standard_normal((nu - 1, len(product_paths_of(lmax)), c)) / 2).astype(np.float32)
+    full = []
+    for q in range(nu - 1):
+        blocks = []
+        for l3 in range(lmax + 1):
+            ps = paths_of_rank(lmax, l3)
+            m = np.zeros((c, len(ps) * c), np.float32)
+            for j, p in enumerate(ps):
+                m[np.arange(c), j * c + np.arange(c)] = wr[q, p]
+            blocks.append(m.ravel())
+        full.append(np.concatenate(blocks))
+    Ad = torch.from_numpy(A).to(DEV)
+    got = etp.node_ladder_full(Ad, torch.from_numpy(np.stack(full)).to(DEV), lmax)
+    red = etp.node_ladder(Ad, torch.from_numpy(wr).to(DEV), lmax)
+    assert_blocks_close(_np(got), _np(red).astype(np.float64), c, lmax, "full ladder with diagonal matrices")
+
+
+def product_paths_of(lmax):
+    from oracle.product import product_paths
+    return product_paths(lmax)
