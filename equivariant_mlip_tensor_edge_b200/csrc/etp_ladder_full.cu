@@ -10,12 +10,16 @@
 // paths of rank l3 times the channels), N = C. It runs on the tensor cores:
 //   k_ladder_t:   CUDA cores, one warp per (node, 32-channel slice): the NT per-path products of the
 //                 node for the lane's channel, written as the rows of the GEMM operands T_l3.
-//   k_ladder_mix: one CTA per (128-node tile, component). Four loader warps stream K-chunks of 32
-//                 columns of T (the node rows) and of W_l3 (the output-channel rows) into shared
-//                 memory as tf32 hi/lo tiles in the canonical K-major layout; one thread issues
-//                 three kind::tf32 MMAs per 8 columns (hi*hi + hi*lo + lo*hi) into a TMEM
-//                 accumulator [128 nodes x C]; the loader warps then read it back (tcgen05.ld) and
-//                 store the component of B_{q+1} and add it into out.
+//   k_ladder_wprep: once per call, every step's W_l3 split into tf32 hi/lo and laid out as the
+//                 MMA B operand tiles (canonical K-major), 32 columns of K per contiguous chunk.
+//   k_ladder_mix: one CTA per (128-node tile, component). Per K-chunk of 32 columns, each of four
+//                 loader warps loads its 32 node rows of T (thread = row = TMEM lane), splits them
+//                 into tf32 hi/lo and writes them straight into TMEM (tcgen05.st): the MMA A operand
+//                 never touches shared memory. The chunk's W tiles arrive by one cp.async.bulk.
+//                 One thread issues three kind::tf32 MMAs per 8 columns (hi*hi + hi*lo + lo*hi,
+//                 A from TMEM, B from shared memory) into a TMEM accumulator [128 nodes x C]; the
+//                 loader warps then read it back (tcgen05.ld), store the component of B_{q+1} and
+//                 add it into out.
 // Every output element is written by one thread per step: the result is bitwise reproducible.
 // Every mbarrier wait is bounded; a timeout records a code in the status word and the CTA drains
 // the MMAs it issued before it releases TMEM.
@@ -77,15 +81,28 @@ struct LadderGen<3> {
   }
 };
 
-// Shared memory of k_ladder_mix for C channels: barriers, then kStages stages of
-// [A hi | A lo | B hi | B lo], each part 4 sub-tiles [rows x 8] in the canonical layout.
+// Shared memory of k_ladder_mix for C channels: barriers; kStages stages of the B operand of a
+// K-chunk, [K-step 0..3][hi, lo][C x 8] (the layout k_ladder_wprep writes); kRaw stages of raw T
+// rows, [128 rows][kRawLd floats] (each loader thread copies and reads back only its own row; the
+// padding keeps the 16-byte reads of 8 consecutive rows on distinct banks).
+constexpr int kRaw = 4;                    // raw T stages: kRaw - 1 chunks requested ahead
+constexpr int kRawLd = kChunk + 4;
 struct Smem {
   static constexpr int kBar = 1024;
-  static __host__ __device__ constexpr int a_part() { return 4 * kRows * 8 * 4; }
-  static __host__ __device__ constexpr int b_part(int C) { return 4 * C * 8 * 4; }
-  static __host__ __device__ constexpr int stage(int C) { return 2 * a_part() + 2 * b_part(C); }
-  static __host__ __device__ constexpr int bytes(int C) { return kBar + kStages * stage(C); }
+  static __host__ __device__ constexpr int stage(int C) { return 4 * 2 * C * 8 * 4; }
+  static __host__ __device__ constexpr int raw_stage() { return kRows * kRawLd * 4; }
+  static __host__ __device__ constexpr int raw_off(int C) { return kBar + kStages * stage(C); }
+  // above half an SM, so that one CTA holds the SM and its 512 TMEM columns
+  static __host__ __device__ constexpr int bytes(int C) {
+    return raw_off(C) + kRaw * raw_stage() > 118 * 1024 ? raw_off(C) + kRaw * raw_stage() : 118 * 1024;
+  }
 };
+
+// TMEM columns of k_ladder_mix: the accumulator [0, 128), then per stage the A operand of a
+// K-chunk: [K-step 0..3][hi, lo][8 columns].
+constexpr uint32_t kTmemAlloc = 512;
+constexpr uint32_t kAccCols = 128;
+constexpr uint32_t kAStageCols = 64;
 
 // ---------------------------------------------------------------- per-path products
 
@@ -130,41 +147,75 @@ struct MixArgs {
   int n_nodes;
   int C;
   const float* T;      // the step's products (k_ladder_t layout)
-  const float* W;      // the step's matrices: rank blocks one after another, each [C][P_l3 C]
+  const float* Wt;     // the step's B operand tiles (k_ladder_wprep layout)
   float* b_next;       // B_{q+1} [N][D C], or null on the last step
   float* out;          // out [N][D C], += B_{q+1}
   int* err;
 };
 
 struct Bars {
-  uint64_t full[kStages];    // a stage's tiles written (kLoadWarps arrivals)
+  uint64_t full[kStages];    // a stage's A columns written to TMEM (kLoadWarps arrivals)
+  uint64_t bfull[kStages];   // a stage's B tiles landed (transaction bytes)
   uint64_t empty[kStages];   // a stage's MMAs complete (one commit)
   uint64_t done;             // every MMA of the tile complete
   uint64_t drain;
   uint32_t tmem_holder;
   int abort_flag;
+  int b_last[kStages];       // per stage: the last chunk whose B copy was issued into it
 };
 
-// One row of a tile: columns [k0, k0 + 32) of row `row` (tile-local) of a row-major matrix whose
-// tile starts at src (leading dimension ld floats), split into tf32 hi/lo and stored in 4
-// sub-tiles [rows x 8] (one per MMA K-step) of the canonical K-major layout. An invalid row (past
-// the last node) is stored as zeros.
-__device__ __forceinline__ void load_row_split(const float* __restrict__ src, size_t ld, int row, bool valid, int k0,
-                                               int rows, float* hi, float* lo) {
-  const float4* p = reinterpret_cast<const float4*>(src + static_cast<size_t>(row) * ld + k0);
-#pragma unroll
-  for (int c4 = 0; c4 < kChunk / 4; ++c4) {
-    const float4 v = valid ? __ldg(p + c4) : make_float4(0.f, 0.f, 0.f, 0.f);
-    float4 h, l;
-    split_tf32(v.x, &h.x, &l.x);
-    split_tf32(v.y, &h.y, &l.y);
-    split_tf32(v.z, &h.z, &l.z);
-    split_tf32(v.w, &h.w, &l.w);
-    const int off = (c4 >> 1) * rows * 8 + canon(row, (c4 & 1) * 4);   // K-step c4 / 2, columns 4 (c4 & 1)..
-    *reinterpret_cast<float4*>(hi + off) = h;
-    *reinterpret_cast<float4*>(lo + off) = l;
+// W of one step as B operand tiles: rank blocks one after another; block l3 holds, per K-chunk c of
+// 32 columns, [K-step s][hi, lo][C x 8] in the canonical K-major layout, so one chunk's tiles are
+// 8 C 8 contiguous floats.
+template <int L>
+__global__ void k_ladder_wprep(int C, int steps, const float* __restrict__ W, float* __restrict__ Wt) {
+  using S = typename LadderGen<L>::S;
+  size_t per_step = 0;
+  for (int l = 0; l <= L; ++l) per_step += static_cast<size_t>(S::P(l)) * C * C;
+  const size_t total = per_step * steps;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const size_t q = i / per_step;
+    size_t r = i - q * per_step;
+    int l3 = 0;
+    size_t blk = 0;
+    while (r >= blk + static_cast<size_t>(S::P(l3)) * C * C) {
+      blk += static_cast<size_t>(S::P(l3)) * C * C;
+      ++l3;
+    }
+    r -= blk;
+    const int K = S::P(l3) * C;
+    const int v = static_cast<int>(r / K), k = static_cast<int>(r % K);
+    float hi, lo;
+    split_tf32(W[i], &hi, &lo);
+    float* dst = Wt + 2 * (q * per_step + blk) + (static_cast<size_t>(k / kChunk) * 8 + ((k % kChunk) / 8) * 2) * C * 8;
+    dst[canon(v, k % 8)] = hi;
+    dst[C * 8 + canon(v, k % 8)] = lo;
   }
 }
+
+// D (TMEM) += A (TMEM: 128 lanes x 8 columns of tf32) x B (shared memory descriptor)
+__device__ __forceinline__ void mma_tf32_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]),
+      "f"(v[19]), "f"(v[20]), "f"(v[21]), "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]),
+      "f"(v[28]), "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Grid: x = 128-node tiles, y = output component (l3, m3) in (l, m) order.
 template <int L>
@@ -180,33 +231,34 @@ __global__ void __launch_bounds__(kThreads, 1) k_ladder_mix(MixArgs a) {
   int l3 = 0;
   while ((l3 + 1) * (l3 + 1) <= comp) ++l3;
   const int m3 = comp - l3 * l3;
-  const int P = S::P(l3);
-  const int K = P * C;                       // GEMM K: the paths of rank l3 times the channels
+  const int K = S::P(l3) * C;                 // GEMM K: the paths of rank l3 times the channels
   const int n_chunks = K / kChunk;
   const int node0 = blockIdx.x * kRows;
-  // the tile's operand rows: T_l3 row (node, m3) has K columns; W_l3 row v has K columns
+  // T_l3 row (node, m3) has K columns
   const float* Tt = a.T + static_cast<size_t>(a.n_nodes) * C * S::off(l3) +
                     (static_cast<size_t>(node0) * (2 * l3 + 1) + m3) * K;
   const size_t t_ld = static_cast<size_t>(2 * l3 + 1) * K;
   size_t w_off = 0;
   for (int l = 0; l < l3; ++l) w_off += static_cast<size_t>(S::P(l)) * C * C;
-  const float* Wl = a.W + w_off;
+  const float* Wl = a.Wt + 2 * w_off;        // the rank's B tiles: 64 C floats per chunk
+  const uint32_t b_bytes = static_cast<uint32_t>(Smem::stage(C));
   volatile int* abort_flag = &bars->abort_flag;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bars->full[s], kLoadWarps);
+      mbar_init(&bars->bfull[s], 1);
       mbar_init(&bars->empty[s], 1);
+      bars->b_last[s] = -1;
     }
     mbar_init(&bars->done, 1);
     mbar_init(&bars->drain, 1);
     bars->abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  const uint32_t cols = C <= 32 ? 32u : (C <= 64 ? 64u : 128u);   // TMEM allocation: a power of two >= C
   if (warp == kMmaWarp) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sptr(&bars->tmem_holder)),
-                 "r"(cols)
+                 "r"(kTmemAlloc)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
@@ -219,33 +271,68 @@ __global__ void __launch_bounds__(kThreads, 1) k_ladder_mix(MixArgs a) {
 
   if (warp < kLoadWarps) {
     // ---------------------------------------------------------------- loaders, then the epilogue
-    const int t = threadIdx.x;   // 0..127: node row t of the tile, and output-channel row t of W
+    const int t = threadIdx.x;                                         // tile row = TMEM lane
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    const bool valid = node0 + t < a.n_nodes;
+    const float* src = Tt + static_cast<size_t>(valid ? t : 0) * t_ld;
+    float* raw = reinterpret_cast<float*>(smem + Smem::raw_off(C)) + t * kRawLd;
+    // this thread's row of chunk k into raw stage k % kRaw (zero-filled past the last node); one
+    // commit group per chunk, so chunk k's copies are complete once at most kRaw - 2 later groups
+    // are pending
+    auto request = [&](int k) {
+      if (k < n_chunks) {
+        float* dst = raw + (k % kRaw) * (kRows * kRawLd);
+#pragma unroll
+        for (int i = 0; i < kChunk / 4; ++i) tc::cp_async16(dst + 4 * i, src + k * kChunk + 4 * i, valid ? 16u : 0u);
+      }
+      tc::cp_async_commit();
+    };
+    for (int k = 0; k < kRaw - 1; ++k) request(k);
     bool ok = true;
     for (int c = 0; c < n_chunks && ok; ++c) {
+      request(c + kRaw - 1);
+      tc::cp_async_wait<kRaw - 1>();
       const int st = c % kStages;
       if (c >= kStages) ok = tc::warp_wait(&bars->empty[st], ((c / kStages) - 1) & 1, abort_flag, a.err, 61);
       if (!ok) break;
-      float* base = reinterpret_cast<float*>(stages + static_cast<size_t>(st) * Smem::stage(C));
-      float* ahi = base;
-      float* alo = ahi + Smem::a_part() / 4;
-      float* bhi = alo + Smem::a_part() / 4;
-      float* blo = bhi + Smem::b_part(C) / 4;
-      load_row_split(Tt, t_ld, t, node0 + t < a.n_nodes, c * kChunk, kRows, ahi, alo);
-      if (t < C) load_row_split(Wl, static_cast<size_t>(K), t, true, c * kChunk, C, bhi, blo);
-      fence_proxy_async();   // generic-proxy stores, read next by the tensor core
+      if (warp == 0 && lane == 0) {   // the chunk's B tiles: one bulk copy (the stage's MMAs are done)
+        tc::mbar_expect_tx(&bars->bfull[st], b_bytes);
+        bars->b_last[st] = c;
+        tc::bulk_g2s(stages + static_cast<size_t>(st) * Smem::stage(C), Wl + static_cast<size_t>(c) * 64 * C,
+                     b_bytes, &bars->bfull[st]);
+      }
+      float4 v[kChunk / 4];
+      const float4* rrow = reinterpret_cast<const float4*>(raw + (c % kRaw) * (kRows * kRawLd));
+#pragma unroll
+      for (int i = 0; i < kChunk / 4; ++i) v[i] = rrow[i];
+      // [K-step s][hi, lo][8]: 64 TMEM columns
+      float hl[64];
+#pragma unroll
+      for (int i = 0; i < kChunk / 4; ++i) {
+        const int s = i >> 1, kk = (i & 1) * 4;
+        split_tf32(v[i].x, &hl[s * 16 + kk + 0], &hl[s * 16 + 8 + kk + 0]);
+        split_tf32(v[i].y, &hl[s * 16 + kk + 1], &hl[s * 16 + 8 + kk + 1]);
+        split_tf32(v[i].z, &hl[s * 16 + kk + 2], &hl[s * 16 + 8 + kk + 2]);
+        split_tf32(v[i].w, &hl[s * 16 + kk + 3], &hl[s * 16 + 8 + kk + 3]);
+      }
+      const uint32_t acol = trow + kAccCols + st * kAStageCols;
+      tmem_st32(acol, *reinterpret_cast<const float(*)[32]>(&hl[0]));
+      tmem_st32(acol + 32, *reinterpret_cast<const float(*)[32]>(&hl[32]));
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars->full[st]);
     }
+    tc::cp_async_wait<0>();   // no copy into this CTA's shared memory outlives the loop
     if (ok) ok = tc::warp_wait(&bars->done, 0, abort_flag, a.err, 62);
     if (ok) {
       tc_fence_after();
       const int node = node0 + t;
-      const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
       for (int v0 = 0; v0 < C; v0 += 32) {
         float d[32];
         tc::tmem_ld32(trow + v0, d);
         tc::tmem_wait_ld();
-        if (node < a.n_nodes) {
+        if (valid) {
           const size_t off = static_cast<size_t>(node) * D * C + static_cast<size_t>(comp) * C + v0;
           float4* o = reinterpret_cast<float4*>(a.out + off);
 #pragma unroll
@@ -272,20 +359,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_ladder_mix(MixArgs a) {
     for (int c = 0; c < n_chunks && ok; ++c) {
       const int st = c % kStages;
       ok = mbar_wait(&bars->full[st], (c / kStages) & 1, abort_flag, a.err, 63);
+      if (ok) ok = mbar_wait(&bars->bfull[st], (c / kStages) & 1, abort_flag, a.err, 65);
       if (!ok) break;
       tc_fence_after();
-      const float* base = reinterpret_cast<const float*>(stages + static_cast<size_t>(st) * Smem::stage(C));
-      const float* ahi = base;
-      const float* alo = ahi + Smem::a_part() / 4;
-      const float* bhi = alo + Smem::a_part() / 4;
-      const float* blo = bhi + Smem::b_part(C) / 4;
+      const float* bst = reinterpret_cast<const float*>(stages + static_cast<size_t>(st) * Smem::stage(C));
+      const uint32_t acol = tmem + kAccCols + st * kAStageCols;
 #pragma unroll
       for (int s = 0; s < kChunk / 8; ++s) {
-        const uint64_t dah = smem_desc(sptr(ahi + s * kRows * 8)), dal = smem_desc(sptr(alo + s * kRows * 8));
-        const uint64_t dbh = smem_desc(sptr(bhi + s * C * 8)), dbl = smem_desc(sptr(blo + s * C * 8));
-        mma_tf32(tmem, dah, dbh, idesc, (c > 0 || s > 0) ? 1u : 0u);
-        mma_tf32(tmem, dah, dbl, idesc, 1u);
-        mma_tf32(tmem, dal, dbh, idesc, 1u);
+        const uint64_t dbh = smem_desc(sptr(bst + (2 * s) * C * 8));
+        const uint64_t dbl = smem_desc(sptr(bst + (2 * s + 1) * C * 8));
+        const uint32_t ah = acol + s * 16, al = ah + 8;
+        mma_tf32_ta(tmem, ah, dbh, idesc, (c > 0 || s > 0) ? 1u : 0u);
+        mma_tf32_ta(tmem, ah, dbl, idesc, 1u);
+        mma_tf32_ta(tmem, al, dbh, idesc, 1u);
       }
       mma_commit(&bars->empty[st]);
     }
@@ -299,11 +385,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_ladder_mix(MixArgs a) {
     }
   }
   if (warp == kMmaWarp) drained = __shfl_sync(0xffffffffu, drained ? 1 : 0, 0) != 0;
+  __syncthreads();
+  // B copies still in flight (on abort no MMA waited for them) are drained before the CTA exits: a
+  // stage is refilled only after its MMAs completed, which waited for its previous copy.
+  if (threadIdx.x == 0) {
+    for (int st = 0; st < kStages; ++st) {
+      const int c = bars->b_last[st];
+      if (c >= 0 && !mbar_wait_drain(&bars->bfull[st], (c / kStages) & 1)) {
+        tc::report_code(a.err, 66);
+        break;
+      }
+    }
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp && drained) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(cols) : "memory");
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemAlloc) : "memory");
   }
 }
 
@@ -334,7 +432,7 @@ size_t step_weights(int C) {
 
 template <int L>
 etp_status run(int C, int order, int n_nodes, const float* A, const float* W, float* out, float* bufs, float* T,
-               int* status, cudaStream_t s) {
+               float* Wt, int* status, cudaStream_t s) {
   constexpr int D = (L + 1) * (L + 1);
   const size_t row = static_cast<size_t>(D) * C;
   cudaError_t e = cudaMemcpyAsync(out, A, sizeof(float) * row * n_nodes, cudaMemcpyDeviceToDevice, s);
@@ -351,11 +449,14 @@ etp_status run(int C, int order, int n_nodes, const float* A, const float* W, fl
     float* b_next = q + 1 < order ? bufs + static_cast<size_t>(q & 1) * row * n_nodes : nullptr;
     k_ladder_t<L><<<static_cast<int>(tblocks), 256, 0, s>>>(n_nodes, C, b_cur, A, T);
     if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "full ladder products");
+    k_ladder_wprep<L><<<static_cast<int>((wstep + 255) / 256 < 4096 ? (wstep + 255) / 256 : 4096), 256, 0, s>>>(
+        C, 1, W + static_cast<size_t>(q - 1) * wstep, Wt);
+    if ((e = cudaGetLastError()) != cudaSuccess) return cuda_status(e, "full ladder weight tiles");
     MixArgs m;
     m.n_nodes = n_nodes;
     m.C = C;
     m.T = T;
-    m.W = W + static_cast<size_t>(q - 1) * wstep;
+    m.Wt = Wt;
     m.b_next = b_next;
     m.out = out;
     m.err = status;
@@ -369,11 +470,15 @@ etp_status run(int C, int order, int n_nodes, const float* A, const float* W, fl
 
 }  // namespace
 
+size_t step_weight_floats(int lmax, int channels);
+
+// [status][B ping-pong: 2 x N x dim][T][one step of B operand tiles: 2 x step floats]
 size_t workspace_bytes(int lmax, int channels, int n_nodes) {
   if (!supported_shape(lmax, channels) || n_nodes < 0) return 0;
   const size_t row = static_cast<size_t>((lmax + 1) * (lmax + 1)) * channels;
   return align256(sizeof(int)) + 2 * align256(sizeof(float) * row * n_nodes) +
-         align256(sizeof(float) * t_floats_rt(lmax, n_nodes, channels));
+         align256(sizeof(float) * t_floats_rt(lmax, n_nodes, channels)) +
+         align256(sizeof(float) * 2 * step_weight_floats(lmax, channels));
 }
 
 size_t step_weight_floats(int lmax, int channels) {
@@ -395,13 +500,15 @@ etp_status launch(int lmax, int channels, int order, int n_nodes, const float* A
   float* bufs = reinterpret_cast<float*>(p);
   p += 2 * align256(sizeof(float) * row * n_nodes);
   float* T = reinterpret_cast<float*>(p);
+  p += align256(sizeof(float) * t_floats_rt(lmax, n_nodes, channels));
+  float* Wt = reinterpret_cast<float*>(p);
   *status_dev = status;
   cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int), s);
   if (e != cudaSuccess) return cuda_status(e, "full ladder status");
   switch (lmax) {
-    case 1: return run<1>(channels, order, n_nodes, A, W, out, bufs, T, status, s);
-    case 2: return run<2>(channels, order, n_nodes, A, W, out, bufs, T, status, s);
-    default: return run<3>(channels, order, n_nodes, A, W, out, bufs, T, status, s);
+    case 1: return run<1>(channels, order, n_nodes, A, W, out, bufs, T, Wt, status, s);
+    case 2: return run<2>(channels, order, n_nodes, A, W, out, bufs, T, Wt, status, s);
+    default: return run<3>(channels, order, n_nodes, A, W, out, bufs, T, Wt, status, s);
   }
 }
 
