@@ -31,6 +31,7 @@ METRIC = "edges/sec for TP conv fwd and fwd+bwd (fp32), % of HBM/FP32 roofline"
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 KERNEL_WARMUP = 20
 KERNEL_REPS = 200
 
@@ -352,6 +353,15 @@ def run_gpu(args, rank, world, local_rank):
     for _ in range(3):
         etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out)
     ms_ladder = kernel_ms(lambda: etp.node_ladder(lad_A, lad_W, lad["lmax"], out=lad_out))
+    # the full ladder (per-rank path- and channel-mixing matrices on the tensor cores), same size
+    lf_W = (torch.randn((lad["nu"] - 1, etp.node_ladder_full_step_floats(lad["lmax"], lad["c"])), generator=gen) /
+            (4 * lad["c"]) ** 0.5).to(dev)
+    lf_out = torch.empty_like(lad_A)
+    lf_ws = torch.empty(etp.load_library().etp_node_ladder_full_workspace_bytes(lad["lmax"], lad["c"], lad["n"]),
+                        dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        etp.node_ladder_full(lad_A, lf_W, lad["lmax"], out=lf_out, workspace=lf_ws)
+    ms_ladder_full = kernel_ms(lambda: etp.node_ladder_full(lad_A, lf_W, lad["lmax"], out=lf_out, workspace=lf_ws))
     # general irreps: NequIP-L channel counts on the same graph (table-driven kernels)
     gen_irreps = "128x0e+64x1o+32x2e+32x3o"
     gconv = etp.EdgeConv(gen_irreps, 3, gen_irreps, wl.n_basis, float(wl.r_cut))
@@ -429,8 +439,10 @@ def run_gpu(args, rank, world, local_rank):
     d2h = out_h.numel() * 4 + f_h.numel() * 4
 
     e = gr.n_edges
-    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd, ms_gen_dw), total_edges = \
-        combine_ranks([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_gen_fwd, ms_gen_bwd, ms_gen_dw],
+    (ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_ladder_full, ms_gen_fwd, ms_gen_bwd,
+     ms_gen_dw), total_edges = \
+        combine_ranks([ms_step, ms_e2e, ms_fwd, ms_bwd, ms_graph, ms_dw, ms_ladder, ms_ladder_full, ms_gen_fwd,
+                       ms_gen_bwd, ms_gen_dw],
                       e, world, dev)
     if rank != 0:
         return None
@@ -474,6 +486,26 @@ def run_gpu(args, rank, world, local_rank):
                 "alu_frac": round(flop / (ms * 1e-3) / 1e12 / fp32_peak, 4),
                 "hbm_frac_of_" + peak_kind: round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
 
+    def ladder_full_roof(ms):
+        """The full ladder's dominant work is the mixing GEMM, 2 K C flop per (node, component) and
+        step (K = paths of the component's rank x C); bound: the tensor cores at the TF32 rate (the
+        measured bf16 rate x the nominal TF32/bf16 ratio 1.1/2.25). The mixing runs as three TF32
+        products (hi*hi + hi*lo + lo*hi) for fp32 accuracy, so the ceiling of this kernel is a third
+        of that rate; fp32_frac compares with the FP32 CUDA-core peak an fp32 GEMM would otherwise
+        run on."""
+        L, c = lad["lmax"], lad["c"]
+        paths = [(a, b, d) for a in range(L + 1) for b in range(L + 1) for d in range(L + 1)
+                 if abs(a - b) <= d <= a + b and (a + b + d) % 2 == 0]
+        per_node = sum((2 * d + 1) * sum(1 for p in paths if p[2] == d) * c * c * 2 for d in range(L + 1))
+        flop = float(per_node) * lad["n"] * (lad["nu"] - 1)
+        tf32 = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS)) * 1.1 / 2.25
+        ach = flop / (ms * 1e-3) / 1e12
+        return {"workload": f"{lad['n']} nodes x {c} channels, lmax {L}, order {lad['nu']}, full ladder",
+                "kernel": "k_ladder_mix", "ms_per_launch": round(ms, 5), "bound": "tensor",
+                "achieved": round(ach, 3), "peak": round(tf32, 2), "unit": "TFLOP/s", "frac": round(ach / tf32, 4),
+                "peak_source": f"{peak_kind} bf16 x 1.1/2.25 (TF32)", "traffic": None,
+                "fp32_frac": round(ach / fp32_peak, 4), "mixing_gflop": round(flop / 1e9, 3)}
+
     def general_roof(ms, kind):
         # the weight gradient's per-path factor costs what the forward contraction does, plus the
         # edge reduction sum_e R_b gw (2 n_basis cols flop per edge)
@@ -511,6 +543,7 @@ def run_gpu(args, rank, world, local_rank):
         "ms_weight_grad": round(ms_dw, 5),
         "roofline_weight_grad": roof("dw", ms_dw),
         "node_ladder": ladder_roof(ms_ladder),
+        "node_ladder_full": ladder_full_roof(ms_ladder_full),
         "general_irreps_fwd": general_roof(ms_gen_fwd, "fwd"),
         "general_irreps_bwd": general_roof(ms_gen_bwd, "bwd"),
         "general_irreps_dw": general_roof(ms_gen_dw, "dw"),
