@@ -118,17 +118,19 @@ KERNEL_SOURCES = {
     "k_gen_fwd": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
     "k_gen_bwd": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
     "k_gen_dw": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
+    "k_ladder_mix": ["etp_ladder_full.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
 }
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised in
 # profiles/<kernel>_<workload>.md, keyed by a hash of the kernel's sources at capture time.
 RECORDED_TRAFFIC = {
-    ("k_fwd_cx", "diamond1k"): (3838720 + 0, "8a4b160400164a98"),
-    ("k_bwd_tc", "diamond1k"): (6547456 + 0, "acdaf5bd61983e18"),
-    ("k_dw_pair", "diamond1k"): (6419072 + 0, "ad7bbc9fed014daf"),
-    ("k_node_ladder", "ladder4096_l2"): (18898432 + 0, "3a9fc533f0a02650"),
-    ("k_gen_fwd", "nequipl_diamond1k"): (4371968 + 0, "b245e3ee8de0307d"),
-    ("k_gen_bwd", "nequipl_diamond1k"): (7540736 + 0, "b245e3ee8de0307d"),
-    ("k_gen_dw", "nequipl_diamond1k"): (7535104 + 0, "b245e3ee8de0307d"),
+    ("k_fwd_cx", "diamond1k"): (3838976 + 0, "53d21688231dedef"),
+    ("k_bwd_tc", "diamond1k"): (6546688 + 0, "63325d2c4afb1ec5"),
+    ("k_dw_pair", "diamond1k"): (6419072 + 0, "00a89d774a2c119d"),
+    ("k_node_ladder", "ladder4096_l2"): (18898176 + 0, "66f8b4ce79f9935b"),
+    ("k_gen_fwd", "nequipl_diamond1k"): (4371712 + 0, "dfd2b891a353c1c8"),
+    ("k_gen_bwd", "nequipl_diamond1k"): (7540224 + 0, "dfd2b891a353c1c8"),
+    ("k_gen_dw", "nequipl_diamond1k"): (7535616 + 0, "dfd2b891a353c1c8"),
+    ("k_ladder_mix", "ladder_full4096_l2"): (93743488 + 429184, "39ca551a22249767"),
 }
 
 
@@ -503,7 +505,8 @@ def run_gpu(args, rank, world, local_rank):
         return {"workload": f"{lad['n']} nodes x {c} channels, lmax {L}, order {lad['nu']}, full ladder",
                 "kernel": "k_ladder_mix", "ms_per_launch": round(ms, 5), "bound": "tensor",
                 "achieved": round(ach, 3), "peak": round(tf32, 2), "unit": "TFLOP/s", "frac": round(ach / tf32, 4),
-                "peak_source": f"{peak_kind} bf16 x 1.1/2.25 (TF32)", "traffic": None,
+                "peak_source": f"{peak_kind} bf16 x 1.1/2.25 (TF32)",
+                "traffic": recorded_traffic("k_ladder_mix", f"ladder_full4096_l{L}"),
                 "fp32_frac": round(ach / fp32_peak, 4), "mixing_gflop": round(flop / 1e9, 3)}
 
     def general_roof(ms, kind):
