@@ -15,7 +15,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libetp.so")
-SOURCES = ["etp_abi.cu", "etp_graph.cu", "etp_conv.cu", "etp_fwd_tc.cu", "etp_bwd_tc.cu", "etp_noalloc.cu", "etp_dw.cu", "etp_fwd_cx.cu", "etp_ladder_full.cu", "etp_product.cu", "etp_general.cu"]
+SOURCES = ["etp_abi.cu", "etp_graph.cu", "etp_conv.cu", "etp_fwd_tc.cu", "etp_bwd_tc.cu", "etp_noalloc.cu", "etp_dw.cu", "etp_fwd_cx.cu", "etp_ladder_full.cu", "etp_product.cu", "etp_general.cu", "etp_general_tc.cu"]
 HEADERS = [os.path.join(ROOT, "include", "etp.h"), os.path.join(CSRC, "etp_internal.h"),
            os.path.join(CSRC, "generated", "etp_paths.h"), os.path.join(CSRC, "etp_device.h"), os.path.join(CSRC, "etp_tc_common.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -284,6 +284,7 @@ bool general_config(const std::vector<Block>& bin, int sh_lmax, const std::vecto
   }
   g.sh_lmax = sh_lmax;
   g.inv_rc = 1.0f / r_cut;
+  plan_general_tc(g);
   int mul = bin[0].mul;
   for (const Block& b : bin) mul = b.mul == mul ? mul : 0;
   for (const Block& b : bout) mul = b.mul == mul ? mul : 0;
@@ -554,8 +555,12 @@ etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_pt
     if (st != ETP_OK) return st;
   }
   if (n_nodes == 0) return ETP_OK;
-  if (h->c.general)
-    return launch_general_forward(h->c.gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, s);
+  if (h->c.general) {
+    st = launch_general_forward(h->c.gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, s,
+                                h->c.status_dev);
+    if (st == ETP_OK && validate_requested()) st = read_status(h->c, s, "general forward");
+    return st;
+  }
   if (use_tc_forward()) {
     if (!workspace || workspace_bytes < etp_workspace_bytes(h, n_nodes, n_edges)) {
       set_error("etp_forward: workspace missing or smaller than etp_workspace_bytes()");
@@ -644,7 +649,7 @@ etp_status etp_forward_masked(etp_handle h, int n_nodes, int n_edges, const int*
   if (n_nodes == 0) return ETP_OK;
   if (h->c.general)
     return launch_general_forward(h->c.gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, s,
-                                  n_edges > 0 ? path_mask : nullptr);
+                                  h->c.status_dev, n_edges > 0 ? path_mask : nullptr);
   void* tcws = static_cast<char*>(workspace) + ws_tc_offset(n_edges);
   st = tc::launch_forward_tc(h->c, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out, tcws, s,
                              n_edges > 0 ? path_mask : nullptr);

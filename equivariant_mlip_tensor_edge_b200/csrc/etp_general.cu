@@ -458,9 +458,11 @@ etp_status launch_general_weight_grad(const GenParams& g, int n_nodes, int n_edg
 
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                   const int* sender, const float* edge_vec, const float* x, const float* W,
-                                  float* out, cudaStream_t s, const uint32_t* path_mask) {
+                                  float* out, cudaStream_t s, int* err, const uint32_t* path_mask) {
   (void)n_edges;
   if (n_nodes == 0) return ETP_OK;
+  if (general_tc_selected(g, path_mask))
+    return launch_general_forward_tc(g, n_nodes, row_ptr, sender, edge_vec, x, W, out, s, err);
   int covered = 0;
   for (int q = 0; q < g.n_out_groups; ++q) covered += g.out_grp[q].size;
   if (covered < g.dim_out) {

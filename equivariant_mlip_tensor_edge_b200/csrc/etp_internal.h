@@ -29,6 +29,16 @@ struct GenGroup {
   int off, size;      // the block's row segment: offset and mul (2l + 1) floats
   int beg, end;       // its paths: order[beg .. end - 1]
 };
+// Tensor-core forward plan: the paths' channels cut into slices of 32 (path, first channel),
+// dealt to the four TMEM lane quadrants; MMA block b holds slice b of every quadrant (128 weight
+// columns as the rows of the A operand). n_blocks = 0: the plan does not fit and the FP32
+// forward serves the handle.
+constexpr int kGenTcMaxBlocks = 16;
+struct GenTcPlan {
+  int n_blocks = 0;
+  short path[kGenTcMaxBlocks][4] = {};   // path of quadrant q's slice in block b (-1: none)
+  short u0[kGenTcMaxBlocks][4] = {};     // its first channel
+};
 struct GenParams {
   int n_paths = 0;
   int dim_in = 0;
@@ -45,8 +55,9 @@ struct GenParams {
   GenGroup in_grp[kGenMaxBlocks];
   unsigned char order_out[kGenMaxPaths];
   unsigned char order_in[kGenMaxPaths];
+  GenTcPlan tcp;
 };
-static_assert(sizeof(GenParams) <= 4000, "the path table travels as a kernel parameter");
+static_assert(sizeof(GenParams) <= 3900, "the path table travels as a kernel parameter");
 
 struct Ctx {
   int lmax = 0;
@@ -153,9 +164,17 @@ etp_status launch_general_weight_grad(const GenParams& g, int n_nodes, int n_edg
                                       const int* sender, const float* edge_vec, const float* x,
                                       const float* grad_out, float* grad_W, int* recv, float* part,
                                       cudaStream_t s);
+// Runs the tensor-core forward (etp_general_tc.cu) when the handle has a plan, no mask is given and
+// ETP_GEN_FORWARD is not "fp32"; err: the handle's status word (bounded waits of that kernel).
 etp_status launch_general_forward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                   const int* sender, const float* edge_vec, const float* x, const float* W,
-                                  float* out, cudaStream_t s, const uint32_t* path_mask = nullptr);
+                                  float* out, cudaStream_t s, int* err, const uint32_t* path_mask = nullptr);
+// Fills g.tcp (n_blocks = 0 when the plan does not fit) from the path table.
+void plan_general_tc(GenParams& g);
+bool general_tc_selected(const GenParams& g, const uint32_t* path_mask);
+etp_status launch_general_forward_tc(const GenParams& g, int n_nodes, const int* row_ptr, const int* sender,
+                                     const float* edge_vec, const float* x, const float* W, float* out,
+                                     cudaStream_t s, int* err);
 etp_status launch_general_backward(const GenParams& g, int n_nodes, int n_edges, const int* row_ptr,
                                    const float* edge_vec, const int* t_row_ptr, const int* t_perm,
                                    const float* x, const float* W, const float* grad_out, float* grad_x,

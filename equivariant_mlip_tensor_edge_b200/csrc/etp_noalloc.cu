@@ -1,7 +1,8 @@
 // Forward entry point whose scratch lives in a fixed, statically sized device array of this
 // module instead of a caller-supplied workspace. For uniform handles it always runs the
 // edge-major tensor-core forward (whatever ETP_FORWARD says); general handles run the
-// table-driven forward, which needs no scratch.
+// general forward, which needs no scratch (its tensor-core form builds its split weights in
+// shared memory).
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -61,13 +62,13 @@ extern "C" etp_status etp_forward_noalloc(etp_handle h, int n_nodes, int n_edges
     return ETP_ERR_INVALID_ARG;
   }
   if (etp::gate(h, "etp_forward_noalloc") != ETP_OK) return ETP_ERR_CUDA;
-  if (c->general) {   // the general kernels need no scratch at all
+  if (c->general) {   // the general forward needs no scratch at all
     if (static_cast<long long>(n_nodes) * c->gen.dim_out >= (1LL << 31)) {
       set_error("etp_forward_noalloc: n_nodes * dim must stay below 2^31");
       return ETP_ERR_UNSUPPORTED;
     }
     return etp::launch_general_forward(c->gen, n_nodes, n_edges, row_ptr, sender, edge_vec, x, W, out,
-                                       static_cast<cudaStream_t>(stream));
+                                       static_cast<cudaStream_t>(stream), c->status_dev);
   }
   const size_t need = etp::tc::forward_tc_workspace_bytes(*c, n_nodes);
   if (need > etp::kScratchBytes) {

@@ -874,6 +874,78 @@ def emit_general(out):
     out.append("    default: break;")
     out.append("  }")
     out.append("}")
+    # forward over a round of staged edges with the radial weights supplied: wl(k0, w) fills w[0..3]
+    # with the channel's weights of edges k0..k0+3 (warp-uniform call); quads of edges run with all
+    # their loads ahead of the arithmetic, the ragged tail one edge at a time
+    out.append("constexpr int kGenYS = 25;   // staged harmonics per edge (to l = 4)")
+    for t, (l1, l2, l3) in enumerate(tri):
+        c = real_cg_any(l1, l2, l3)
+        groups = []
+        for m3 in range(2 * l3 + 1):
+            for m1 in range(2 * l1 + 1):
+                terms = [(c[m1, m2, m3], idx(l2, m2 - l2)) for m2 in range(2 * l2 + 1) if c[m1, m2, m3] != 0.0]
+                if terms:
+                    groups.append((m3, m1, terms))
+        rows = sorted({m3 for m3, _, _ in groups})
+
+        def body(ind, k, w):
+            lines = [f"{ind}{{ const float* Y = Ys + ({k}) * kGenYS;",
+                     f"{ind}  const float* x = xu + static_cast<size_t>(sj[{k}]) * dim_in;"]
+            for m1 in range(2 * l1 + 1):
+                lines.append(f"{ind}  const float x{m1} = x[{m1} * stride];")
+            for m3 in rows:
+                row = [(m1, terms) for (a3, m1, terms) in groups if a3 == m3]
+                first = True
+                for m1, terms in row:
+                    mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                    if first:
+                        lines.append(f"{ind}  float s{m3} = ({mexpr}) * x{m1};")
+                        first = False
+                    else:
+                        lines.append(f"{ind}  s{m3} = fmaf({mexpr}, x{m1}, s{m3});")
+                lines.append(f"{ind}  a{m3} = fmaf({w}, s{m3}, a{m3});")
+            lines.append(f"{ind}}}")
+            return lines
+
+        out.append("template <class WL>")
+        out.append(f"__device__ __forceinline__ void gfwdw_{t}(const float* Ys, const int* sj, int cnt,")
+        out.append("                                        const float* __restrict__ xu, int dim_in, int stride, WL&& wl,")
+        out.append("                                        bool act, float* acc) {")
+        for m3 in rows:
+            out.append(f"  float a{m3} = 0.0f;")
+        out.append("  int k0 = 0;")
+        out.append("  for (; k0 + 4 <= cnt; k0 += 4) {")
+        out.append("    float w[4];")
+        out.append("    wl(k0, w);")
+        out.append("    if (act) {")
+        out.append("      #pragma unroll")
+        out.append("      for (int kk = 0; kk < 4; ++kk)")
+        out.extend(body("        ", "k0 + kk", "w[kk]"))
+        out.append("    }")
+        out.append("  }")
+        out.append("  if (k0 < cnt) {")
+        out.append("    float w[4];")
+        out.append("    wl(k0, w);")
+        out.append("    if (act)")
+        out.append("      for (int kk = 0; k0 + kk < cnt; ++kk) {")
+        out.append("        const float wk = kk == 0 ? w[0] : (kk == 1 ? w[1] : w[2]);")
+        out.extend(body("        ", "k0 + kk", "wk"))
+        out.append("      }")
+        out.append("  }")
+        out.append("  if (act) {")
+        for m3 in rows:
+            out.append(f"    acc[{m3} * stride] += a{m3};")
+        out.append("  }")
+        out.append("}")
+    out.append("template <class WL>")
+    out.append("__device__ __forceinline__ void gen_fwd_w(int t, const float* Ys, const int* sj, int cnt, const float* xu,")
+    out.append("                                          int dim_in, int stride, WL&& wl, bool act, float* acc) {")
+    out.append("  switch (t) {")
+    for t in range(len(tri)):
+        out.append(f"    case {t}: gfwdw_{t}(Ys, sj, cnt, xu, dim_in, stride, wl, act, acc); break;")
+    out.append("    default: break;")
+    out.append("  }")
+    out.append("}")
     out.append("// mk: per-edge path masks of the chunk (null: every path on); bit: this path's bit")
     out.append("__device__ __forceinline__ void gen_fwd_chunk(int t, const float* geo, const int* sj, int cnt,")
     out.append("                                              const float* xu, int dim_in, int stride, const float* wb,")

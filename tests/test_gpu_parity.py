@@ -779,6 +779,61 @@ def test_general_irreps_parity_sampled_full_size(wls):
     assert_close_rel(gv[pos], rgv, "NequIP-L grad_edge_vec (sampled)")
 
 
+@pytest.mark.parametrize("impl", ["tc", "fp32"])
+@pytest.mark.parametrize("irin,sh,irout", GENERAL)
+def test_general_irreps_forward_ragged_both_kernels(irin, sh, irout, impl, monkeypatch):
+    """The general forward with its radial projection on the tensor cores (the default) and on the
+    FP32 pipe (ETP_GEN_FORWARD=fp32): degrees 0..150 (empty rows, one edge, quads and ragged tails
+    of the 32-edge rounds, several rounds) against the oracle, with the status word checked."""
+    if impl == "fp32":
+        monkeypatch.setenv("ETP_GEN_FORWARD", "fp32")
+    monkeypatch.setenv("ETP_VALIDATE", "1")
+    n = 12
+    degrees = np.array([0, 1, 3, 4, 5, 31, 32, 33, 0, 64, 97, 150])
+    recv, send, vec = _random_graph(n, degrees, seed=len(irin) + sh)
+    conv = etp.EdgeConv(irin, sh, irout, 8, 5.0)
+    spec = ConvSpec(irin, sh, irout, 8, 5.0)
+    x, W, _ = _general_inputs(spec, n, 5 + sh)
+    g = etp.build_csr(n, torch.from_numpy(recv).to(DEV), torch.from_numpy(send).to(DEV),
+                      torch.from_numpy(vec).to(DEV))
+    xd, Wd = torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)
+    ws = torch.empty(conv.workspace_bytes(n, g.n_edges), dtype=torch.uint8, device=DEV)
+    out = conv.forward(g, xd, Wd, workspace=ws)
+    order = np.lexsort((send, recv))
+    rp = np.concatenate([[0], np.cumsum(degrees)])
+    ref = conv_forward(spec, rp, send[order], vec[order], x, W)
+    on = _np(out)
+    assert np.all(on[degrees == 0] == 0.0)
+    assert_irrep_blocks_close(on, ref, spec, "out", f"{irin} ragged forward ({impl})")
+    assert torch.equal(conv.forward(g, xd, Wd, workspace=ws), out)   # bitwise repeatable
+    conv.check_status(DEV)
+
+
+def test_general_irreps_forward_kernels_differ_only_by_rounding(wls, monkeypatch):
+    """NequIP-L on the 1000-atom cell: the tensor-core general forward (default) and the FP32 one
+    agree to rounding but not bit for bit (so the default really is the tensor-core kernel), and
+    the no-workspace entry point runs the default kernel."""
+    wl = wls("diamond1k")
+    irr = "128x0e+64x1o+32x2e+32x3o"
+    conv = etp.EdgeConv(irr, 3, irr, 8, float(wl.r_cut))
+    spec = ConvSpec(irr, 3, irr, 8, float(wl.r_cut))
+    x, W, _ = _general_inputs(spec, wl.n_nodes, 78)
+    g = _gpu_graph(wl)
+    xd, Wd = torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)
+    out_tc = conv.forward(g, xd, Wd)
+    out_nw = torch.empty_like(out_tc)
+    st = etp.load_library().etp_forward_noalloc(conv._h, g.n_nodes, g.n_edges, etp._ptr(g.row_ptr),
+                                                etp._ptr(g.sender), etp._ptr(g.edge_vec), etp._ptr(xd),
+                                                etp._ptr(Wd), etp._ptr(out_nw), etp._stream(xd.device))
+    assert st == 0 and torch.equal(out_nw, out_tc)
+    monkeypatch.setenv("ETP_GEN_FORWARD", "fp32")
+    out_fp = conv.forward(g, xd, Wd)
+    assert not torch.equal(out_fp, out_tc)
+    # each is within 1e-5 max|ref| of the oracle (the tests above), so within twice that of the other
+    assert_irrep_blocks_close(_np(out_tc), _np(out_fp).astype(np.float64), spec, "out",
+                              "NequIP-L tensor-core vs FP32 forward", tol=2e-5)
+
+
 @pytest.mark.parametrize("irin,sh,irout", GENERAL)
 def test_general_irreps_weight_grad_parity(wls, irin, sh, irout):
     """dL/dW of general irreps handles against the oracle (small cell), and bitwise repeatable."""
@@ -824,8 +879,9 @@ def test_general_irreps_weight_grad_full_size(wls):
 
 @pytest.mark.parametrize("irin,sh,irout", [("16x0e+16x1o+16x1e+16x2e+16x2o", 2, "16x0e+16x1o+16x1e+16x2e+16x2o"),
                                           ("128x0e+64x1o+32x2e+32x3o", 3, "128x0e+64x1o+32x2e+32x3o")])
-def test_general_irreps_path_mask_parity(wls, irin, sh, irout):
-    """Per-edge path masks on general handles (at most 32 paths) against the oracle."""
+def test_general_irreps_path_mask_parity(wls, irin, sh, irout, monkeypatch):
+    """Per-edge path masks on general handles (at most 32 paths) against the oracle. Masked calls
+    run the FP32 general forward, so with every bit set they equal its unmasked call bit for bit."""
     wl = wls("tiny")
     conv = etp.EdgeConv(irin, sh, irout, 8, float(wl.r_cut))
     spec = ConvSpec(irin, sh, irout, 8, float(wl.r_cut))
@@ -845,8 +901,9 @@ def test_general_irreps_path_mask_parity(wls, irin, sh, irout):
     rgx, rgv = conv_vjp(spec, ref_g["row_ptr"], ref_g["sender"], ref_g["edge_vec"], x, W, gout, path_mask=mask)
     assert_irrep_blocks_close(_np(gx), rgx, spec, "in", f"{irin} masked grad_x")
     assert_close_rel(_np(gv), rgv, f"{irin} masked grad_edge_vec")
-    # all bits set is the unmasked call, bit for bit
+    # all bits set is the unmasked call of the same kernel, bit for bit
     ones = torch.full((g.n_edges,), -1, dtype=torch.int32, device=DEV)
+    monkeypatch.setenv("ETP_GEN_FORWARD", "fp32")
     assert torch.equal(conv.forward(g, xd, Wd, path_mask=ones), conv.forward(g, xd, Wd))
 
 
