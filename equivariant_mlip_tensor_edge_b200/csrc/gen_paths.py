@@ -876,7 +876,8 @@ def emit_general(out):
     out.append("}")
     # forward over a round of staged edges with the radial weights supplied: wl(k0, w) fills w[0..3]
     # with the channel's weights of edges k0..k0+3 (warp-uniform call); quads of edges run with all
-    # their loads ahead of the arithmetic, the ragged tail one edge at a time
+    # their loads ahead of the arithmetic, the ragged tail one edge at a time. Instantiated for the
+    # block strides 32, 64 and 128 (component loads at immediate offsets) and for any stride.
     out.append("constexpr int kGenYS = 25;   // staged harmonics per edge (to l = 4)")
     for t, (l1, l2, l3) in enumerate(tri):
         c = real_cg_any(l1, l2, l3)
@@ -907,10 +908,11 @@ def emit_general(out):
             lines.append(f"{ind}}}")
             return lines
 
-        out.append("template <class WL>")
+        out.append("template <int S, class WL>   // S: the block stride when known at compile time (0: stride_rt)")
         out.append(f"__device__ __forceinline__ void gfwdw_{t}(const float* Ys, const int* sj, int cnt,")
-        out.append("                                        const float* __restrict__ xu, int dim_in, int stride, WL&& wl,")
+        out.append("                                        const float* __restrict__ xu, int dim_in, int stride_rt, WL&& wl,")
         out.append("                                        bool act, float* acc) {")
+        out.append("  const int stride = S ? S : stride_rt;")
         for m3 in rows:
             out.append(f"  float a{m3} = 0.0f;")
         out.append("  int k0 = 0;")
@@ -942,7 +944,12 @@ def emit_general(out):
     out.append("                                          int dim_in, int stride, WL&& wl, bool act, float* acc) {")
     out.append("  switch (t) {")
     for t in range(len(tri)):
-        out.append(f"    case {t}: gfwdw_{t}(Ys, sj, cnt, xu, dim_in, stride, wl, act, acc); break;")
+        out.append(f"    case {t}:")
+        for st in (32, 64, 128):
+            kw = "if" if st == 32 else "else if"
+            out.append(f"      {kw} (stride == {st}) gfwdw_{t}<{st}>(Ys, sj, cnt, xu, dim_in, stride, wl, act, acc);")
+        out.append(f"      else gfwdw_{t}<0>(Ys, sj, cnt, xu, dim_in, stride, wl, act, acc);")
+        out.append("      break;")
     out.append("    default: break;")
     out.append("  }")
     out.append("}")
