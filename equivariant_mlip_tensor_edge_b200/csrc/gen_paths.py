@@ -768,9 +768,11 @@ def emit_general(out):
                     groups.append((m3, m1, terms))
         out.append(f"// ({l1},{l2},{l3})")
         # backward
+        out.append("template <int S>   // S: the block stride when known at compile time (0: stride_rt)")
         out.append(f"__device__ __forceinline__ void gbwd_{t}(const float* __restrict__ x, const float* __restrict__ g,")
-        out.append("                                       int stride, const float* Y, float w, float* gx, float* gY,")
+        out.append("                                       int stride_rt, const float* Y, float w, float* gx, float* gY,")
         out.append("                                       float& gw) {")
+        out.append("  const int stride = S ? S : stride_rt;")
         for m1 in range(2 * l1 + 1):
             out.append(f"  const float x{m1} = x[{m1} * stride];")
             out.append(f"  float a{m1} = 0.0f;")
@@ -840,9 +842,11 @@ def emit_general(out):
                 if terms:
                     groups.append((m3, m1, terms))
         rows = sorted({m3 for m3, _, _ in groups})
+        out.append("template <int S>   // S: the block stride when known at compile time (0: stride_rt)")
         out.append(f"__device__ __forceinline__ void gdwc_{t}(const float* geo, const int* sj, const int* si, int cnt,")
         out.append("                                       const float* __restrict__ xu, const float* __restrict__ gu,")
-        out.append("                                       int dim_in, int dim_out, int stride, float* acc8) {")
+        out.append("                                       int dim_in, int dim_out, int stride_rt, float* acc8) {")
+        out.append("  const int stride = S ? S : stride_rt;")
         out.append("  for (int k = 0; k < cnt; ++k) {")
         out.append("    const float* Y = geo + k * kGenGeoF;")
         out.append("    const float* x = xu + static_cast<size_t>(sj[k]) * dim_in;")
@@ -870,7 +874,12 @@ def emit_general(out):
     out.append("                                             int stride, float* acc8) {")
     out.append("  switch (t) {")
     for t in range(len(tri)):
-        out.append(f"    case {t}: gdwc_{t}(geo, sj, si, cnt, xu, gu, dim_in, dim_out, stride, acc8); break;")
+        out.append(f"    case {t}:")
+        for st in (32, 64, 128):
+            kw = "if" if st == 32 else "else if"
+            out.append(f"      {kw} (stride == {st}) gdwc_{t}<{st}>(geo, sj, si, cnt, xu, gu, dim_in, dim_out, stride, acc8);")
+        out.append(f"      else gdwc_{t}<0>(geo, sj, si, cnt, xu, gu, dim_in, dim_out, stride, acc8);")
+        out.append("      break;")
     out.append("    default: break;")
     out.append("  }")
     out.append("}")
@@ -967,7 +976,12 @@ def emit_general(out):
     out.append("                                        float w, float* gx, float* gY, float& gw) {")
     out.append("  switch (t) {")
     for t in range(len(tri)):
-        out.append(f"    case {t}: gbwd_{t}(x, g, stride, Y, w, gx, gY, gw); break;")
+        out.append(f"    case {t}:")
+        for st in (32, 64, 128):
+            kw = "if" if st == 32 else "else if"
+            out.append(f"      {kw} (stride == {st}) gbwd_{t}<{st}>(x, g, stride, Y, w, gx, gY, gw);")
+        out.append(f"      else gbwd_{t}<0>(x, g, stride, Y, w, gx, gY, gw);")
+        out.append("      break;")
     out.append("    default: break;")
     out.append("  }")
     out.append("}")
