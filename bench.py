@@ -116,6 +116,7 @@ KERNEL_SOURCES = {
     "k_dw_pair": ["etp_dw.cu", "etp_device.h", "generated/etp_paths.h"],
     "k_node_ladder": ["etp_product.cu", "etp_device.h", "generated/etp_paths.h"],
     "k_gen_fwd": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
+    "k_gen_fwd_tc": ["etp_general_tc.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
     "k_gen_bwd": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
     "k_gen_dw": ["etp_general.cu", "etp_device.h", "generated/etp_paths.h"],
     "k_ladder_mix": ["etp_ladder_full.cu", "etp_tc_common.h", "etp_device.h", "generated/etp_paths.h"],
@@ -514,11 +515,13 @@ def run_gpu(args, rank, world, local_rank):
         # edge reduction sum_e R_b gw (2 n_basis cols flop per edge)
         flop = (float(gi["flop_fwd"]) + 2.0 * gi["weight_numel"]) * e if kind == "dw" else float(gi[f"flop_{kind}"]) * e
         ach = flop / (ms * 1e-3) / 1e12
+        # the forward runs the tensor-core general kernel (radial projection on tcgen05)
+        kernel = "k_gen_fwd_tc" if kind == "fwd" else f"k_gen_{kind}"
         return {"workload": f"{gen_irreps}, harmonics to l = 3, {wl.name} graph ({e} edges)",
-                "kernel": f"k_gen_{kind}", "ms_per_launch": round(ms, 5), "bound": "alu", "achieved": round(ach, 3),
+                "kernel": kernel, "ms_per_launch": round(ms, 5), "bound": "alu", "achieved": round(ach, 3),
                 "peak": round(fp32_peak, 2), "unit": "TFLOP/s", "frac": round(ach / fp32_peak, 4),
                 "edges_per_s": round(e / (ms * 1e-3), 1),
-                "traffic": recorded_traffic(f"k_gen_{kind}", f"nequipl_{wl.name}")}
+                "traffic": recorded_traffic(kernel, f"nequipl_{wl.name}")}
 
     line = {
         "metric": METRIC,

@@ -102,7 +102,7 @@ typedef struct {
  *  - uniform (the tensor-core kernels): every block has the same multiplicity C (C % 4 == 0,
  *    4 <= C <= 256), blocks are l = 0..L in order with parity (-1)^l, irreps_out == irreps_in,
  *    sh_lmax == L, L in {1,2,3};
- *  - general (table-driven FP32 kernels, info.general = 1): any blocks with 0 <= l <= 4 and
+ *  - general (table-driven kernels, info.general = 1): any blocks with 0 <= l <= 4 and
  *    1 <= mul <= 1024 in any order and either parity, sh_lmax <= 4, node rows of at most 4096
  *    floats, 1 to 128 paths, at most 16 blocks a side. Paths join blocks of EQUAL multiplicity only (uvu: channel u to
  *    channel u), so irreps like NequIP's 128x0e+64x1o+32x2e+32x3o couple 2e with 3o but not 1o
@@ -114,7 +114,12 @@ typedef struct {
  *    etp_forward, etp_forward_noalloc (no scratch needed), etp_backward, etp_backward_weights and,
  *    for handles with at most 32 paths (the mask has 32 bits), etp_forward_masked and
  *    etp_backward_masked (more paths: ETP_ERR_UNSUPPORTED); etp_radial_weights returns
- *    ETP_ERR_UNSUPPORTED for them.
+ *    ETP_ERR_UNSUPPORTED for them. Their forward computes the radial weights on the tensor cores
+ *    (kind::tf32, three products of the tf32 split) when the handle's plan fits (the paths' 32-channel
+ *    slices fill at most 16 blocks of 128 weight columns, and the split weights, the output row
+ *    copies and the staging fit 227 KB of shared memory); masked calls, handles outside that plan
+ *    and ETP_GEN_FORWARD=fp32 run the FP32 kernel (the two agree with the float64 reference within
+ *    the same tolerance, not bit for bit). The backward and the weight gradient are FP32 kernels.
  * Both need n_basis == 8 and r_cut > 0. Malformed strings -> ETP_ERR_IRREPS; anything else
  * outside these sets -> ETP_ERR_UNSUPPORTED. The path list is the enumeration described above. */
 etp_status etp_create(const char* irreps_in, int sh_lmax, const char* irreps_out, int n_basis,
@@ -169,8 +174,8 @@ etp_status etp_forward(etp_handle h, int n_nodes, int n_edges, const int* row_pt
  * module, one per device, so the call allocates no memory and takes nothing from the caller but
  * the tensors. For uniform handles it always runs the edge-major tensor-core forward and ignores
  * ETP_FORWARD, so its bits can differ from etp_forward's default kernel (both agree with the
- * float64 reference within the same tolerance); general handles run the table-driven forward,
- * which needs no scratch.
+ * float64 reference within the same tolerance); general handles run the same kernel as their
+ * etp_forward, which needs no scratch (the tensor-core form splits its weights in shared memory).
  * The method has no such call; it is an interface convenience. It is for callers that cannot
  * provide device scratch: for instance a host program that reaches the model through a fixed
  * plugin interface that hands over only the input and output tensors, with no allocator of its
