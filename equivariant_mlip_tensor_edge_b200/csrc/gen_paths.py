@@ -778,6 +778,11 @@ def emit_general(out):
             out.append(f"  float a{m1} = 0.0f;")
         for m3 in range(2 * l3 + 1):
             out.append(f"  const float g{m3} = g[{m3} * stride];")
+        # dL/dY_i = w sum_terms C x g: the sums over the coupling's terms first, one product with w
+        # per harmonic component at the end
+        ys = sorted({i for _, _, terms in groups for _, i in terms})
+        for i in ys:
+            out.append(f"  float t{i} = 0.0f;")
         for m3, m1, terms in groups:
             mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
             out.append(f"  {{ const float mv = {mexpr};")
@@ -785,8 +790,10 @@ def emit_general(out):
             out.append(f"    const float xg = x{m1} * g{m3};")
             out.append("    gw = fmaf(mv, xg, gw);")
             for v, i in terms:
-                out.append(f"    gY[{i}] = fmaf({repr_f32(np.float32(v))} * w, xg, gY[{i}]);")
+                out.append(f"    t{i} = fmaf({repr_f32(np.float32(v))}, xg, t{i});")
             out.append("  }")
+        for i in ys:
+            out.append(f"  gY[{i}] = fmaf(w, t{i}, gY[{i}]);")
         for m1 in range(2 * l1 + 1):
             out.append(f"  gx[{m1} * stride] = fmaf(w, a{m1}, gx[{m1} * stride]);")
         out.append("}")
