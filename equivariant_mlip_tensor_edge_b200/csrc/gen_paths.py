@@ -783,17 +783,31 @@ def emit_general(out):
         ys = sorted({i for _, _, terms in groups for _, i in terms})
         for i in ys:
             out.append(f"  float t{i} = 0.0f;")
+        # two equivalent orders, the one with fewer operations is emitted:
+        #   A: mv = sum C Y per (m3, m1), a += mv g, xg = x g, t_i += C xg
+        #   B: cg = C g per (C, m3), then per term a += Y cg and t_i += x cg
+        cost_a = len({tuple(terms) for _, _, terms in groups}) + 2 * len(groups) + sum(len(t) for _, _, t in groups)
+        cost_b = len({(np.float32(v), m3) for m3, _, terms in groups for v, _ in terms}) + \
+            2 * sum(len(t) for _, _, t in groups)
         for m3, m1, terms in groups:
-            mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
-            out.append(f"  {{ const float mv = {mexpr};")
-            out.append(f"    a{m1} = fmaf(mv, g{m3}, a{m1});")
-            out.append(f"    const float xg = x{m1} * g{m3};")
-            out.append("    gw = fmaf(mv, xg, gw);")
-            for v, i in terms:
-                out.append(f"    t{i} = fmaf({repr_f32(np.float32(v))}, xg, t{i});")
-            out.append("  }")
+            if cost_a <= cost_b:
+                mexpr = " + ".join(f"{repr_f32(np.float32(v))}*Y[{i}]" for v, i in terms)
+                out.append(f"  {{ const float mv = {mexpr};")
+                out.append(f"    a{m1} = fmaf(mv, g{m3}, a{m1});")
+                out.append(f"    const float xg = x{m1} * g{m3};")
+                for v, i in terms:
+                    out.append(f"    t{i} = fmaf({repr_f32(np.float32(v))}, xg, t{i});")
+                out.append("  }")
+            else:
+                for v, i in terms:
+                    out.append(f"  {{ const float cg = {repr_f32(np.float32(v))} * g{m3};")
+                    out.append(f"    a{m1} = fmaf(Y[{i}], cg, a{m1});")
+                    out.append(f"    t{i} = fmaf(x{m1}, cg, t{i}); }}")
         for i in ys:
             out.append(f"  gY[{i}] = fmaf(w, t{i}, gY[{i}]);")
+        # dL/dw = sum_{m1, m3} x M g = sum_m1 x[m1] a[m1]
+        for m1 in range(2 * l1 + 1):
+            out.append(f"  gw = fmaf(x{m1}, a{m1}, gw);")
         for m1 in range(2 * l1 + 1):
             out.append(f"  gx[{m1} * stride] = fmaf(w, a{m1}, gx[{m1} * stride]);")
         out.append("}")
