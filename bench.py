@@ -124,14 +124,14 @@ KERNEL_SOURCES = {
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised in
 # profiles/<kernel>_<workload>.md, keyed by a hash of the kernel's sources at capture time.
 RECORDED_TRAFFIC = {
-    ("k_fwd_cx", "diamond1k"): (3838976 + 0, "53d21688231dedef"),
-    ("k_bwd_tc", "diamond1k"): (6546688 + 0, "63325d2c4afb1ec5"),
-    ("k_dw_pair", "diamond1k"): (6419072 + 0, "00a89d774a2c119d"),
-    ("k_node_ladder", "ladder4096_l2"): (18898176 + 0, "66f8b4ce79f9935b"),
-    ("k_gen_fwd", "nequipl_diamond1k"): (4371712 + 0, "dfd2b891a353c1c8"),
-    ("k_gen_bwd", "nequipl_diamond1k"): (7540224 + 0, "dfd2b891a353c1c8"),
-    ("k_gen_dw", "nequipl_diamond1k"): (7535616 + 0, "dfd2b891a353c1c8"),
-    ("k_ladder_mix", "ladder_full4096_l2"): (93743488 + 429184, "39ca551a22249767"),
+    ("k_fwd_cx", "diamond1k"): (3838976 + 0, "fd682e65b3f8446a"),
+    ("k_bwd_tc", "diamond1k"): (6546944 + 0, "4c7c1bd4b19ff2bd"),
+    ("k_dw_pair", "diamond1k"): (6419072 + 0, "38fbe4bab767f971"),
+    ("k_node_ladder", "ladder4096_l2"): (18898432 + 0, "1a24bdcf27b3ffd1"),
+    ("k_gen_fwd_tc", "nequipl_diamond1k"): (4433152 + 0, "367004bd86802b39"),
+    ("k_gen_bwd", "nequipl_diamond1k"): (7563520 + 0, "1a8eed53d06a16a3"),
+    ("k_gen_dw", "nequipl_diamond1k"): (7538176 + 0, "1a8eed53d06a16a3"),
+    ("k_ladder_mix", "ladder_full4096_l2"): (93743104 + 413952, "082af7a27a72565a"),
 }
 
 
