@@ -9,8 +9,9 @@
 // of the FP32 general forward, without its eight FMAs per edge, path and channel.
 //
 // A CTA of four warps takes one receiver at a time (receivers strided over the grid). Per round of
-// <= 32 edges: warp 0 stages the harmonics, warp 1 the radial basis as the B operand (tf32 hi / lo
-// rows), warp 2 the senders; thread 0 issues the MMAs; then every warp runs its slices over the
+// <= 32 edges (padded to whole quads with edges of zero weight and zero harmonics that read a real
+// sender's row): warp 0 stages the harmonics, warp 1 the radial basis as the B operand (tf32 hi /
+// lo rows), warp 2 the senders; thread 0 issues the MMAs; then every warp runs its slices over the
 // round's edges with the generated coupling code (gfwdw_t: quads of edges with their loads ahead
 // of the arithmetic), each slice's message summed in registers and added once per round into the
 // warp's own copy of the output row in shared memory. Per receiver the four copies are added in
@@ -152,10 +153,11 @@ __global__ void __launch_bounds__(kThr) k_gen_fwd_tc(const __grid_constant__ Gen
         ok = false;
         break;
       }
+      const int nk = (cnt + 3) & ~3;   // whole quads: the padding edges have w = 0 and Y = 0
       const bool valid = lane < cnt;
       const int e = c0 + lane;
       if (warp == 2) {
-        if (valid) sj[lane] = sender[e];
+        if (lane < nk) sj[lane] = sender[valid ? e : c0];   // a padding edge reads a real sender's row
       } else if (warp < 2) {
         float vx = 0.0f, vy = 0.0f, vz = 0.0f;
         if (valid) {
@@ -165,12 +167,12 @@ __global__ void __launch_bounds__(kThr) k_gen_fwd_tc(const __grid_constant__ Gen
         }
         const float d = sqrtf(vx * vx + vy * vy + vz * vz);
         if (warp == 0) {
-          if (valid) {
+          if (lane < nk) {
             const float inv_d = d > 0.0f ? 1.0f / d : 0.0f;
             float Y[kYS];
             sh_upto(g.sh_lmax, vx * inv_d, vy * inv_d, vz * inv_d, Y);
 #pragma unroll
-            for (int c = 0; c < kYS; ++c) Ys[lane * kYS + c] = Y[c];
+            for (int c = 0; c < kYS; ++c) Ys[lane * kYS + c] = valid ? Y[c] : 0.0f;
           }
         } else {
           float R[kNumBasis], dR[kNumBasis];
@@ -222,7 +224,7 @@ __global__ void __launch_bounds__(kThr) k_gen_fwd_tc(const __grid_constant__ Gen
           tmem_ld4(taddr + static_cast<uint32_t>(k0), w);
           tc::tmem_wait_ld();
         };
-        etp_gen::gen_fwd_w(P.tri, Ys, sj, cnt, x + P.in_off + u, g.dim_in, P.mul, wl, act,
+        etp_gen::gen_fwd_w(P.tri, Ys, sj, nk, x + P.in_off + u, g.dim_in, P.mul, wl, act,
                            accw + (P.out_off + u));
       }
     }

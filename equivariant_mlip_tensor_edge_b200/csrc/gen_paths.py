@@ -905,9 +905,10 @@ def emit_general(out):
     out.append("  }")
     out.append("}")
     # forward over a round of staged edges with the radial weights supplied: wl(k0, w) fills w[0..3]
-    # with the channel's weights of edges k0..k0+3 (warp-uniform call); quads of edges run with all
-    # their loads ahead of the arithmetic, the ragged tail one edge at a time. Instantiated for the
-    # block strides 32, 64 and 128 (component loads at immediate offsets) and for any stride.
+    # with the channel's weights of edges k0..k0+3 (warp-uniform call); the edges run in quads with
+    # all their loads ahead of the arithmetic (the caller pads the round to whole quads with edges
+    # of zero weight and zero harmonics). Instantiated for the block strides 32, 64 and 128
+    # (component loads at immediate offsets) and for any stride.
     out.append("constexpr int kGenYS = 25;   // staged harmonics per edge (to l = 4)")
     for t, (l1, l2, l3) in enumerate(tri):
         c = real_cg_any(l1, l2, l3)
@@ -945,8 +946,7 @@ def emit_general(out):
         out.append("  const int stride = S ? S : stride_rt;")
         for m3 in rows:
             out.append(f"  float a{m3} = 0.0f;")
-        out.append("  int k0 = 0;")
-        out.append("  for (; k0 + 4 <= cnt; k0 += 4) {")
+        out.append("  for (int k0 = 0; k0 < cnt; k0 += 4) {   // cnt: a multiple of 4 (padding edges weigh zero)")
         out.append("    float w[4];")
         out.append("    wl(k0, w);")
         out.append("    if (act) {")
@@ -954,15 +954,6 @@ def emit_general(out):
         out.append("      for (int kk = 0; kk < 4; ++kk)")
         out.extend(body("        ", "k0 + kk", "w[kk]"))
         out.append("    }")
-        out.append("  }")
-        out.append("  if (k0 < cnt) {")
-        out.append("    float w[4];")
-        out.append("    wl(k0, w);")
-        out.append("    if (act)")
-        out.append("      for (int kk = 0; k0 + kk < cnt; ++kk) {")
-        out.append("        const float wk = kk == 0 ? w[0] : (kk == 1 ? w[1] : w[2]);")
-        out.extend(body("        ", "k0 + kk", "wk"))
-        out.append("      }")
         out.append("  }")
         out.append("  if (act) {")
         for m3 in rows:
