@@ -124,14 +124,14 @@ KERNEL_SOURCES = {
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch, from the ncu captures summarised in
 # profiles/<kernel>_<workload>.md, keyed by a hash of the kernel's sources at capture time.
 RECORDED_TRAFFIC = {
-    ("k_fwd_cx", "diamond1k"): (3838976 + 0, "fd682e65b3f8446a"),
-    ("k_bwd_tc", "diamond1k"): (6546944 + 0, "4c7c1bd4b19ff2bd"),
-    ("k_dw_pair", "diamond1k"): (6419072 + 0, "38fbe4bab767f971"),
-    ("k_node_ladder", "ladder4096_l2"): (18898432 + 0, "1a24bdcf27b3ffd1"),
-    ("k_gen_fwd_tc", "nequipl_diamond1k"): (4433152 + 0, "367004bd86802b39"),
-    ("k_gen_bwd", "nequipl_diamond1k"): (7563520 + 0, "1a8eed53d06a16a3"),
-    ("k_gen_dw", "nequipl_diamond1k"): (7538176 + 0, "1a8eed53d06a16a3"),
-    ("k_ladder_mix", "ladder_full4096_l2"): (93743104 + 413952, "082af7a27a72565a"),
+    ("k_fwd_cx", "diamond1k"): (3838720 + 0, "40b5d99bc09974bb"),
+    ("k_bwd_tc", "diamond1k"): (6546944 + 0, "b52ffa427ab48b75"),
+    ("k_dw_pair", "diamond1k"): (6418816 + 0, "86c17c159f9a5c2f"),
+    ("k_node_ladder", "ladder4096_l2"): (18898432 + 0, "e21b6756156138a7"),
+    ("k_gen_fwd_tc", "nequipl_diamond1k"): (4399872 + 0, "ee151666faecb84b"),
+    ("k_gen_bwd", "nequipl_diamond1k"): (7565824 + 0, "fcb3a1d2171be5f7"),
+    ("k_gen_dw", "nequipl_diamond1k"): (7538176 + 0, "fcb3a1d2171be5f7"),
+    ("k_ladder_mix", "ladder_full4096_l2"): (93742976 + 397440, "f4fd8ff8fff3e133"),
 }
 
 
