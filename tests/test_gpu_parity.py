@@ -834,6 +834,24 @@ def test_general_irreps_forward_kernels_differ_only_by_rounding(wls, monkeypatch
                               "NequIP-L tensor-core vs FP32 forward", tol=2e-5)
 
 
+@pytest.mark.parametrize("irr,sh", [("64x0e+64x1o+64x1e+64x2e+64x2o", 2), ("32x0e+32x1o+32x2e+32x3o+32x4e", 4)])
+def test_general_irreps_forward_tc_full_size_sampled(wls, irr, sh):
+    """Handles whose tensor-core plan holds 13 and 11 MMA blocks (one CTA per SM, 512 TMEM columns)
+    on the 1000-atom cell: sampled receivers against the oracle, computed one by one, and the
+    status word clean."""
+    wl = wls("diamond1k")
+    conv = etp.EdgeConv(irr, sh, irr, 8, float(wl.r_cut))
+    spec = ConvSpec(irr, sh, irr, 8, float(wl.r_cut))
+    x, W, _ = _general_inputs(spec, wl.n_nodes, 79 + sh)
+    g = _gpu_graph(wl)
+    out = _np(conv.forward(g, torch.from_numpy(x).to(DEV), torch.from_numpy(W).to(DEV)))
+    conv.check_status(DEV)
+    rng = np.random.default_rng(19 + sh)
+    sample = np.sort(rng.choice(wl.n_nodes, size=N_SAMPLE // 4, replace=False))
+    ref, _ = forward_ref(wl, spec, x, W, sample=sample)
+    assert_irrep_blocks_close(out[sample], ref, spec, "out", f"{irr} forward (sampled)")
+
+
 @pytest.mark.parametrize("irin,sh,irout", GENERAL)
 def test_general_irreps_weight_grad_parity(wls, irin, sh, irout):
     """dL/dW of general irreps handles against the oracle (small cell), and bitwise repeatable."""
